@@ -1,0 +1,208 @@
+/*
+ * ue.h -- C ABI of libue, the B200 (sm_100a) implementation of UltraEP's
+ * per-layer, per-microbatch exact-load rebalancing hot path:
+ *
+ *   ue_gate_topk -> ue_count -> ue_plan -> ue_reroute -> ue_permute
+ *   (experts, outside this library) -> ue_combine
+ *
+ * Sources (page title, section):
+ *   "UltraEP" project README, "Interface / 1. Initialization" (one manager
+ *     per EP group, redundant slots reserved per rank, no runtime
+ *     allocation), "Interface / 2. Forward and backward" (router ->
+ *     update_placement -> reroute -> dispatch -> experts -> combine),
+ *     "Performance Tuning / NVSHMEM" (global-load metadata before planning);
+ *   "Xiaohongshu's UltraEP Balances MoE Experts in 300 us, Reaching 94.3% of
+ *     Ideal", "How balancing in 300 microseconds works" (quota-driven
+ *     scheduler, rebalancing every microbatch and every layer);
+ *   "UltraEP: Real-Time Load Balancing for Large-Scale MoE Training and
+ *     Inference", "What Happened" (exact routing, hot experts replicated per
+ *     microbatch and per layer).
+ *
+ * One context simulates one EP group of R ranks on one GPU. Sizes:
+ *   R ranks, T tokens per rank, N = R*T tokens (token n lives on rank n/T),
+ *   E experts (E % R == 0), M = E/R masters per rank (expert e's master is on
+ *   rank e/M), K top-k, S redundant slots per rank, d hidden size (bf16),
+ *   Q = N*K token-expert pairs (pair i = n*K + k, "global order"),
+ *   G = R*S redundant slots (slot g = r*S + s lives on rank r),
+ *   P = R*(M+S) physical slots, rank-major: rank r owns
+ *   p = r*(M+S) + m (its masters, m < M) then p = r*(M+S) + M + s.
+ *
+ * Conventions, for every call below:
+ *   - Pointers are device pointers unless stated otherwise. The caller owns
+ *     every input and output buffer; the context owns only its scratch.
+ *   - Every call is asynchronous on the given stream (0 = legacy default
+ *     stream), performs no host synchronisation and allocates nothing.
+ *     Output sizes never depend on the data.
+ *   - Host-side errors (null or misaligned pointers, sizes out of range,
+ *     a destroyed context) are returned at once and nothing is launched.
+ *   - Device-side errors (an expert id out of range, a row index out of
+ *     range, a wait that ran out) are recorded in the context's error word;
+ *     the kernel skips the offending element or returns early. They are
+ *     read (and cleared) with ue_get_error. No device code traps.
+ *   - One context must not be used from two streams at once.
+ */
+#ifndef UE_H
+#define UE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    UE_OK = 0,
+    UE_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or config   */
+    UE_ERR_CUDA = 2,          /* a CUDA runtime call failed               */
+    UE_ERR_NOMEM = 3,         /* scratch allocation failed in ue_init     */
+    UE_ERR_DEVICE_BOUNDS = 4, /* a kernel met an out-of-range id or row   */
+    UE_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out       */
+    UE_ERR_UNSUPPORTED = 6    /* no sm_100 device, or sizes beyond limits */
+} ue_status;
+
+/* Sizes of one simulated EP group. Limits: 1 <= R <= 128; 1 <= E <= 256;
+ * E % R == 0; 1 <= K <= min(E, 32); 0 <= S <= 8 and R*S <= 256; T >= 1;
+ * Q = R*T*K < 2^30; d >= 8, d % 8 == 0 (rows are whole 16-byte units) and
+ * d <= 16384. */
+typedef struct {
+    int32_t R, T, E, K, S, d;
+} ue_config;
+
+/* The replication plan of one layer instance ("placement": the pages'
+ * update_placement). All arrays are int32 device buffers owned by the
+ * caller, written by ue_plan and read by ue_reroute.
+ *   slot_expert [G]   expert held by redundant slot g, -1 when empty
+ *   n_copies    [E]   copies of expert e (master included), >= 1
+ *   slot_quota  [P]   pairs assigned to physical slot p
+ *   slot_offset [P+1] exclusive running sum of slot_quota: slot p's rows in
+ *                     the dispatch buffer are [slot_offset[p],
+ *                     slot_offset[p+1]); rank r's receive buffer is
+ *                     [slot_offset[r*(M+S)], slot_offset[(r+1)*(M+S)])
+ *   rank_load   [R]   pairs each rank processes under the plan
+ *   stats       [4]   {iterations, max rank load before (masters only),
+ *                      max rank load after, copies placed on a rank that
+ *                      already held a copy of the same expert}
+ * slot_expert may be NULL when S == 0. */
+typedef struct {
+    int32_t* slot_expert;
+    int32_t* n_copies;
+    int32_t* slot_quota;
+    int32_t* slot_offset;
+    int32_t* rank_load;
+    int32_t* stats;
+} ue_placement;
+
+typedef struct ue_ctx ue_ctx; /* opaque */
+
+/* Create a context for `cfg` on CUDA device `device` (made current) and
+ * allocate its scratch once: the error word and the reroute's look-back
+ * status words (ceil(Q/2048)*E 32-bit words plus a tile counter). Nothing
+ * is allocated after this call ("Interface / 1. Initialization": buffers
+ * reserved up front, no dynamic allocation at runtime).
+ * Returns UE_ERR_INVALID_ARG for a null `out` or a config outside the
+ * limits (checked before any CUDA call), UE_ERR_UNSUPPORTED if the device
+ * is not compute capability 10.x, UE_ERR_CUDA / UE_ERR_NOMEM on failure.
+ * On error *out is set to NULL. */
+ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out);
+
+/* Free the context's scratch (synchronises the device first). NULL is
+ * accepted and ignored. */
+ue_status ue_destroy(ue_ctx* ctx);
+
+/* Synchronise `stream`, then read and clear the context's device error
+ * word. Returns UE_OK, UE_ERR_DEVICE_BOUNDS, UE_ERR_TIMEOUT, or UE_ERR_CUDA
+ * if the synchronisation itself failed. */
+ue_status ue_get_error(ue_ctx* ctx, void* stream);
+
+/* Router gating ("Interface / 2. Forward and backward": probs, routing_map
+ * = router(hidden); "What Happened": exact routing probabilities).
+ *   logits fp32 [N][E] row-major, 4-byte aligned.
+ *   idx    int32 [N][K]: per token the K experts with the largest logits,
+ *          in descending logit order; equal logits (IEEE ==, -0.0 == +0.0)
+ *          go to the lower expert id. Logits must be finite.
+ *   w      fp32 [N][K]: softmax over the K selected logits,
+ *          w_k = exp(v_k - v_0) / sum_j exp(v_j - v_0), evaluated in fp64
+ *          and rounded once to fp32. */
+ue_status ue_gate_topk(ue_ctx* ctx, const float* logits, int32_t* idx,
+                       float* w, void* stream);
+
+/* Exact per-expert load ("UltraEP" README intro: rebalance on the exact
+ * post-gating load; "Performance Tuning / NVSHMEM": per-rank load metadata
+ * gathered before planning).
+ *   idx     int32 [N][K] expert ids (from ue_gate_topk).
+ *   load_re int32 [R][E]: pairs of source rank r routed to expert e.
+ *   load_e  int32 [E]: sum over r of load_re.
+ * Both outputs are overwritten (zeroed on the stream first). An id outside
+ * [0, E) is skipped and sets UE_ERR_DEVICE_BOUNDS. */
+ue_status ue_count(ue_ctx* ctx, const int32_t* idx, int32_t* load_re,
+                   int32_t* load_e, void* stream);
+
+/* Quota-driven replication plan ("How balancing in 300 microseconds works";
+ * "Interface / 2. Forward and backward": update_placement).
+ *   load_e int32 [E] exact per-expert pair counts, Q = sum(load_e).
+ * Rule: start with the masters only; quota of copy j of expert e (j = 0 the
+ * master, then replicas by ascending g) is floor(L_e/c_e) plus one for the
+ * first L_e mod c_e copies; a rank's load is the sum of its copies' quotas.
+ * Repeat: stop if 50*R*max_r load_r <= 51*Q (max <= 1.02 x mean) or no slot
+ * is free; else take e* = argmax L_e/c_e (exact integer comparison, ties to
+ * the lowest e) and give it a copy in the lowest free slot of the least
+ * loaded rank that has one (ties to the lowest r).
+ * Writes every array of `out` (device pointers, see ue_placement). Runs as
+ * a single CTA. */
+ue_status ue_plan(ue_ctx* ctx, const int32_t* load_e, const ue_placement* out,
+                  void* stream);
+
+/* Logical -> physical routing ("Interface / 2. Forward and backward":
+ * reroute expands logical routing to physical replicas).
+ *   idx       int32 [N][K] expert ids.
+ *   plan      a placement written by ue_plan for the same idx.
+ *   phys_slot int32 [N][K]: physical slot of each pair.
+ *   dest_row  int32 [N][K]: row of each pair in the dispatch buffer.
+ * Pairs in global order fill each expert's copies by prefix sum (master
+ * first, then replicas by ascending g): the o-th pair of expert e goes to
+ * the copy whose quota range holds o, at row slot_offset[p] + (o - start).
+ * dest_row is a permutation of [0, Q). Single pass: a stable counting sort
+ * with a decoupled look-back scan over tiles of 2048 pairs; its waits are
+ * bounded and end with UE_ERR_TIMEOUT. Ids outside [0, E) set
+ * UE_ERR_DEVICE_BOUNDS. */
+ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
+                     int32_t* phys_slot, int32_t* dest_row, void* stream);
+
+/* Token dispatch into per-slot contiguous buffers ("Interface / 2. Forward
+ * and backward": dispatch(hidden, probs, routing_map), here a single-GPU
+ * gather/scatter).
+ *   hidden   bf16 [N][d] (raw 16-bit words), 16-byte aligned.
+ *   dest_row int32 [N][K] from ue_reroute (a permutation of [0, Q)).
+ *   dispatch bf16 [Q][d], 16-byte aligned, must not overlap hidden:
+ *            dispatch[dest_row[n*K+k]] = hidden[n], bit for bit.
+ * Rows outside [0, Q) are skipped and set UE_ERR_DEVICE_BOUNDS. */
+ue_status ue_permute(ue_ctx* ctx, const uint16_t* hidden,
+                     const int32_t* dest_row, uint16_t* dispatch,
+                     void* stream);
+
+/* Gate-weighted combine / unpermute ("Interface / 2. Forward and
+ * backward": combine(recv_tokens)).
+ *   y        bf16 [Q][d] expert outputs in dispatch order, 16-byte aligned.
+ *   dest_row int32 [N][K], w fp32 [N][K].
+ *   out      fp32 [N][d], 16-byte aligned:
+ *            out[n] = sum_{k=0..K-1} w[n][k] * y[dest_row[n*K+k]],
+ *            accumulated in fp32 with one fused multiply-add per term,
+ *            k ascending, starting from 0.
+ * Rows outside [0, Q) contribute nothing and set UE_ERR_DEVICE_BOUNDS. */
+ue_status ue_combine(ue_ctx* ctx, const uint16_t* y, const int32_t* dest_row,
+                     const float* w, float* out, void* stream);
+
+/* Test hooks for the bounded waits (no counterpart on the pages).
+ * ue_debug_set_lookback_limit sets the number of polls a reroute tile makes
+ * on a predecessor before it gives up with UE_ERR_TIMEOUT (default 1<<22,
+ * with a sleep between polls). ue_debug_drop_first_publish(ctx, 1) makes the
+ * first reroute tile skip publishing its counts, so that its successor's
+ * wait runs out; 0 restores normal behaviour. */
+ue_status ue_debug_set_lookback_limit(ue_ctx* ctx, int64_t polls);
+ue_status ue_debug_drop_first_publish(ue_ctx* ctx, int enable);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UE_H */

@@ -1,0 +1,112 @@
+"""The oracle's pins catch plausible mistakes (CPU only).
+
+Each case plants one mistake in a private copy of oracle.c (a flipped tie
+break, an off-by-one in the quota remainder, a loosened stop test, a wrong
+index...), builds it, and runs the pin tests against it: at least one pin
+must fail. The real oracle is never modified.
+"""
+import ctypes
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+from tests import test_oracle_gate as tg
+from tests import test_oracle_plan as tp
+from tests import test_oracle_rows as tr
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTANTS = {
+    "topk_tie_to_higher_id": ("if (a->e < b->e) return -1;\n    if (a->e > b->e) return 1;",
+                              "if (a->e < b->e) return 1;\n    if (a->e > b->e) return -1;"),
+    "topk_signed_zero_not_tied": (
+        "if (a->v > b->v) return -1;\n    if (a->v < b->v) return 1;",
+        "if (a->v > b->v || (a->v == b->v && signbit(b->v) && !signbit(a->v))) return -1;\n"
+        "    if (a->v < b->v || (a->v == b->v && signbit(a->v) && !signbit(b->v))) return 1;"),
+    "topk_weight_unshifted": ("w[n * K + k] = exp((double)row[k].v - v0) / z;",
+                              "w[n * K + k] = exp((double)row[k].v) / z;"),
+    "count_rank_from_pair": ("int64_t r = n / T;", "int64_t r = i / T;"),
+    "quota_remainder_off_by_one": ("return L / c + (j < L % c ? 1 : 0);",
+                                   "return L / c + (j <= L % c ? 1 : 0);"),
+    "stop_strict": ("if (50 * (int64_t)R * maxl <= 51 * Q) break;",
+                    "if (50 * (int64_t)R * maxl < 51 * Q) break;"),
+    "stop_looser": ("if (50 * (int64_t)R * maxl <= 51 * Q) break;",
+                    "if (50 * (int64_t)R * maxl <= 52 * Q) break;"),
+    "rank_tie_to_higher_r": ("if (used < S && (rstar < 0 || load[r] < load[rstar])) rstar = r;",
+                             "if (used < S && (rstar < 0 || load[r] <= load[rstar])) rstar = r;"),
+    "expert_tie_to_higher_e": ("(int64_t)load_e[e] * n_copies[estar] >\n",
+                               "(int64_t)load_e[e] * n_copies[estar] >=\n"),
+    "remainder_by_descending_slot": ("for (int32_t g = 0; g < G; ++g) {\n            if (slot_expert[g] == e) {\n                load[g / S]",
+                                     "for (int32_t g = G - 1; g >= 0; --g) {\n            if (slot_expert[g] == e) {\n                load[g / S]"),
+    "reroute_row_without_start": ("dest_row[i] = slot_offset[found] + (int32_t)(o - start);",
+                                  "dest_row[i] = slot_offset[found] + (int32_t)o;"),
+    "permute_wrong_token": ("memcpy(dispatch + row * d, hidden + (i / K) * d,",
+                            "memcpy(dispatch + row * d, hidden + (i % K) * d,"),
+    "combine_first_weight_only": ("double wk = w[n * K + k];", "double wk = w[n * K];"),
+}
+
+
+def run_pins(golden_dir):
+    """Every pin of the oracle; returns the names of those that failed."""
+    pins = [
+        ("hand_row", tg.test_hand_row_closed_form),
+        ("signed_zero", tg.test_signed_zero_ties_to_lower_id),
+        ("all_equal", tg.test_all_equal_rows_pick_lowest_ids_and_uniform_weights),
+        ("brute_topk", lambda: tg.test_matches_brute_force_with_many_ties(64, 4)),
+        ("softmax", lambda: tg.test_weights_equal_renormalised_full_softmax(128, 8)),
+        ("count_uniform", tg.test_count_constructed_uniform_routing),
+        ("count_random", tg.test_count_random_matches_bincount),
+        ("hand_plans", lambda: tp.test_hand_worked_plans(golden_dir)),
+        ("plan_invariants", lambda: tp.test_plan_invariants_random(8, 64, 2, 1.2)),
+        ("plan_hot", tp.test_plan_single_hot_expert_closed_form),
+        ("hand_reroute", lambda: tp.test_reroute_hand_worked(golden_dir)),
+        ("reroute_invariants", lambda: tp.test_reroute_invariants_random(4, 33, 16, 3, 2)),
+        ("permute", tr.test_permute_definition_small),
+        ("combine_exact", tr.test_combine_exact_dyadic_case),
+        ("combine_identity", tr.test_combine_identity_experts_reproduce_hidden),
+    ]
+    failed = []
+    for name, fn in pins:
+        try:
+            fn()
+        except (AssertionError, ValueError):
+            failed.append(name)
+    return failed
+
+
+def test_real_oracle_passes_every_pin(golden_dir):
+    assert run_pins(golden_dir) == []
+
+
+_CHILD = """
+import ctypes, sys
+sys.path.insert(0, {root!r})
+import oracle
+from tests import test_oracle_mutants as m
+oracle._lib = oracle._bind(ctypes.CDLL({so!r}))
+failed = m.run_pins({golden!r})
+print("FAILED_PINS", failed)
+sys.exit(1 if failed else 0)
+"""
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, golden_dir, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fPIC",
+                           "-shared", "-o", str(so), str(path), "-lm"])
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    # a child process, so that a mutant that writes out of bounds and crashes
+    # (which also counts as caught) cannot take the test run down with it
+    res = subprocess.run([sys.executable, "-c",
+                          _CHILD.format(root=root, so=str(so), golden=golden_dir)],
+                         capture_output=True, text=True, timeout=300)
+    assert res.returncode != 0, f"no pin caught the planted mistake '{name}':\n{res.stdout}"

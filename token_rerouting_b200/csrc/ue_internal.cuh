@@ -1,0 +1,84 @@
+// ue_internal.cuh -- internal declarations shared by the libue translation
+// units (kernels + C ABI). Not installed, not part of the ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "ue.h"
+
+namespace ue {
+
+// Device error word layout: err[0] = first ue_status code raised,
+// err[1] = a detail value (the offending index or tile).
+__device__ __forceinline__ void raise_error(int* err, int code, int detail)
+{
+    if (atomicCAS(err, 0, code) == 0) {
+        atomicExch(err + 1, detail);
+    }
+}
+
+constexpr int kWarp = 32;
+constexpr unsigned kFull = 0xffffffffu;
+
+// Reroute tiling: pairs per tile and threads per tile.
+constexpr int kRerouteTile = 2048;
+constexpr int kRerouteThreads = 256;
+constexpr int kRerouteWarps = kRerouteThreads / kWarp;
+
+// Look-back status word: [31:30] flag, [29:0] count.
+constexpr uint32_t kFlagInvalid = 0u;
+constexpr uint32_t kFlagAggregate = 1u;
+constexpr uint32_t kFlagPrefix = 2u;
+constexpr uint32_t kFlagError = 3u;
+constexpr uint32_t kValueMask = (1u << 30) - 1u;
+
+// Upper limits of the config (checked on the host).
+constexpr int kMaxR = 128;
+constexpr int kMaxE = 256;
+constexpr int kMaxK = 32;
+constexpr int kMaxS = 8;
+constexpr int kMaxG = 256;
+constexpr int kMaxD = 16384;
+
+struct Sizes {
+    int R, T, E, K, S, d;
+    int M, G, P;
+    int64_t N, Q;
+};
+
+inline Sizes make_sizes(const ue_config& c)
+{
+    Sizes s;
+    s.R = c.R; s.T = c.T; s.E = c.E; s.K = c.K; s.S = c.S; s.d = c.d;
+    s.M = c.E / c.R;
+    s.G = c.R * c.S;
+    s.P = c.R * (s.M + c.S);
+    s.N = (int64_t)c.R * c.T;
+    s.Q = s.N * c.K;
+    return s;
+}
+
+// Launch helpers, one per kernel family. Each returns the CUDA error of the
+// launch (cudaSuccess if nothing was launched because there was no work).
+cudaError_t launch_gate_topk(const Sizes& z, const float* logits, int32_t* idx,
+                             float* w, int grid, cudaStream_t st);
+cudaError_t launch_count(const Sizes& z, const int32_t* idx, int32_t* load_re,
+                         int32_t* load_e, int* err, cudaStream_t st);
+cudaError_t launch_plan(const Sizes& z, const int32_t* load_e,
+                        const ue_placement& out, int* err, cudaStream_t st);
+cudaError_t launch_reroute(const Sizes& z, const int32_t* idx,
+                           const ue_placement& plan, int32_t* phys_slot,
+                           int32_t* dest_row, uint32_t* status,
+                           uint32_t* tile_counter, int64_t spin_limit,
+                           int drop_first, int* err, cudaStream_t st);
+cudaError_t launch_permute(const Sizes& z, const uint16_t* hidden,
+                           const int32_t* dest_row, uint16_t* dispatch,
+                           int num_sms, int* err, cudaStream_t st);
+cudaError_t launch_combine(const Sizes& z, const uint16_t* y,
+                           const int32_t* dest_row, const float* w, float* out,
+                           int num_sms, int* err, cudaStream_t st);
+
+int gate_topk_grid(const Sizes& z, int num_sms);
+
+}  // namespace ue
