@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-load expert rebalancing hot path on B200.
+
+One step = one layer instance through the whole path on the device:
+gate top-k -> exact histogram -> replication plan -> reroute -> permute ->
+gate-weighted combine (identity experts: the combine reads the dispatch
+buffer), on the Qwen3-235B-shaped layer (R=64 simulated EP ranks x 4096
+tokens, E=128, K=8, S=2, d=4096) with synthetic skewed routing (pre-balance
+max/mean rank load 2.5).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ue|reference]
+
+Prints one JSON line (rank 0). ``value`` is routed token-expert pairs per
+second over all GPUs, device-timed with CUDA events (max over ranks).
+With N > 1 (torchrun) every GPU runs its own layer instance (a different
+microbatch): weak scaling, no data-path collective.
+``--impl reference`` times the CPU oracle on a bounded sample of the same
+workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("routed token-expert pairs/s and µs/layer (gate→plan→permute), "
+          "% of HBM roofline")
+UNIT = "pairs/s"
+DEFAULT_WORKLOAD = "qwen3_layer_r64_e128"
+KERNELS = ("gate_topk", "count", "plan", "reroute", "permute", "combine")
+FALLBACK_HBM_GBS = 6650.0
+
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture, with the SHA-256 of the kernel source it was taken on; a
+# kernel changed since then reports null.
+TRAFFIC = {}
+
+
+def sha_of(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+KERNEL_SRC = {
+    "gate_topk": "k_gate.cu", "count": "k_count.cu", "plan": "k_plan.cu",
+    "reroute": "k_reroute.cu", "permute": "k_permute.cu", "combine": "k_combine.cu",
+}
+
+
+def algorithmic_bytes(w):
+    """Bytes each step must move per kernel (reads + writes of its operands)."""
+    N, E, K, d, Q = w.N, w.E, w.K, w.d, w.Q
+    return {
+        "gate_topk": 4 * N * E + 8 * Q,          # logits in; idx + w out
+        "count": 4 * Q,                          # idx in (counts are tiny)
+        "plan": 0,                               # latency bound: reported in us
+        "reroute": 4 * Q + 8 * Q,                # idx in; phys_slot + dest_row out
+        "permute": 2 * N * d + 2 * Q * d,        # each row read once, written K times
+        "combine": 2 * Q * d + 8 * Q + 4 * N * d,  # K rows + dest/w in; fp32 row out
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------- clocks ----
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the bench runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="ue_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        pw = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        # samples under load: power above the midpoint of what was seen
+        if pw and len(pw) == len(sm):
+            cut = (min(pw) + max(pw)) / 2
+            loaded = [s for s, p in zip(sm, pw) if p >= cut] or sm
+        else:
+            loaded = sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# ----------------------------------------------------------- distributed ----
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if n_gpus > 1 and world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} needs torchrun with {n_gpus} processes "
+                         f"(WORLD_SIZE={world})")
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Largest value over all ranks (the slowest rank sets the time)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- oracle -----
+def oracle_slices(w, logits, hidden, tokens_per_rank, budget_s, max_slices):
+    """Run the CPU oracle over slices of the workload (every rank's tokens
+    [j*t, (j+1)*t)), each as one layer instance: gate -> count -> plan ->
+    reroute -> permute -> combine. Stops after budget_s seconds or
+    max_slices slices. Returns (pairs, seconds, slices)."""
+    import oracle
+    t = tokens_per_rank
+    pairs, elapsed, done = 0, 0.0, 0
+    nsl = max(1, w.T // t)
+    lg3 = logits.reshape(w.R, w.T, w.E)
+    hd3 = hidden.reshape(w.R, w.T, w.d)
+    for j in range(min(nsl, max_slices)):
+        lg = lg3[:, j * t:(j + 1) * t].reshape(-1, w.E).copy()
+        hd = hd3[:, j * t:(j + 1) * t].reshape(-1, w.d).copy()
+        t0 = time.perf_counter()
+        o = oracle.run_path(lg, w.R, t, w.S, w.K)
+        disp = oracle.permute(hd, w.K, o["dest_row"])
+        oracle.combine(disp, w.R * t, w.K, o["dest_row"], o["w"])
+        elapsed += time.perf_counter() - t0
+        pairs += w.R * t * w.K
+        done += 1
+        del disp
+        if elapsed >= budget_s:
+            break
+    return pairs, elapsed, done
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_setup(args.gpus)
+    if rank != 0:
+        return
+    import synth
+    logits = synth.logits(w, mb=0)
+    hidden = synth.hidden(w)
+    # size each step so that warm-up + timed steps take about two minutes
+    per_step_s = max(0.05, 120.0 / max(1, args.steps + args.warmup))
+    t = 512
+    while t > 8 and 2.2 * (t / 512) > per_step_s:
+        t //= 2
+    for _ in range(args.warmup):
+        oracle_slices(w, logits, hidden, t, 0.0, 1)
+    pairs, secs, n = 0, 0.0, 0
+    for _ in range(args.steps):
+        p, s, _k = oracle_slices(w, logits, hidden, t, 0.0, 1)
+        pairs += p
+        secs += s
+        n += 1
+    value = pairs / secs
+    sample = (f"{t} tokens per rank x {w.R} ranks ({w.R * t * w.K} pairs) per step, the first "
+              f"slice of the {w.name} workload, whole path incl. permute and combine")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / max(1, n), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "R": w.R, "T": w.T, "N": w.N, "E": w.E, "K": w.K, "S": w.S,
+            "d": w.d, "pairs_per_step": w.Q,
+            "routing": "logits N(0,1) + Zipf(s=1.0) log-weight bias scaled to a masters-only "
+                       "max/mean rank load of 2.5, seed 0 (microbatch = rank)",
+            "l2": "inputs larger than L2 (logits 134 MB, hidden 2.1 GB, dispatch 17.2 GB)",
+            "experts": "identity (combine reads the dispatch buffer)"}
+
+
+# ------------------------------------------------------------------ main ----
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ue", "reference"), default="ue")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    world, rank, local = dist_setup(args.gpus)
+    import numpy as np
+    import torch
+
+    import token_rerouting_b200 as ue
+    from token_rerouting_b200 import build as ue_build
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    if rank == 0:
+        ue_build.build()
+    if world > 1:
+        dist.barrier()
+    ue.load_library()
+
+    # inputs: each rank is a different microbatch of the same layer
+    logits_h = synth.logits(w, mb=rank)
+    hidden_h = synth.hidden(w, seed=rank)
+    L = ue.Layer(w.R, w.T, w.E, w.K, w.S, w.d, device=local)
+    L.logits.copy_(torch.from_numpy(logits_h))
+    L.hidden.copy_(torch.from_numpy(hidden_h.view(np.int16)).to(dev).view(torch.bfloat16))
+    stream = torch.cuda.current_stream(dev)
+
+    steps_fn = [L.gate, L.count, L.plan_step, L.reroute, L.permute, L.combine]
+
+    def step():
+        for f in steps_fn:
+            f(stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    rc = L.error(stream)
+    if rc != 0:
+        raise SystemExit(f"device error after warm-up: {ue.STATUS.get(rc, rc)}")
+    plan0 = L.plan_arrays()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.2)
+    # kernel-level events: ev[s][k] .. ev[s][k+1] brackets kernel k of step s
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(steps_fn) + 1)]
+           for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(args.steps):
+        ev = evs[s]
+        ev[0].record(stream)
+        for k, f in enumerate(steps_fn):
+            f(stream=stream)
+            ev[k + 1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = start.elapsed_time(end)
+    rc = L.error(stream)
+    if rc != 0:
+        raise SystemExit(f"device error in the timed region: {ue.STATUS.get(rc, rc)}")
+
+    per_kernel_ms = {name: statistics.fmean(evs[s][k].elapsed_time(evs[s][k + 1])
+                                            for s in range(args.steps))
+                     for k, name in enumerate(KERNELS)}
+    ms_step_local = total_ms / args.steps
+    ms_step = max_over_ranks(ms_step_local, world, dev)
+    value = world * w.Q / (ms_step / 1e3)
+
+    # dominant kernel and its roofline
+    abytes = algorithmic_bytes(w)
+    dom = max(("permute", "combine", "gate_topk", "reroute"), key=lambda k: per_kernel_ms[k])
+    peak, peak_kind = load_peaks()
+    achieved = abytes[dom] / (per_kernel_ms[dom] / 1e3) / 1e9
+    tr = TRAFFIC.get(dom)
+    src = os.path.join(ROOT, "token_rerouting_b200", "csrc", KERNEL_SRC[dom])
+    traffic = tr["bytes_per_launch"] if tr and tr.get("source_sha") == sha_of(src) else None
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "peak_kind": f"of {peak_kind}",
+                "traffic": traffic, "algorithmic_bytes": abytes[dom]}
+    kernels = {}
+    for k in KERNELS:
+        ms = per_kernel_ms[k]
+        kernels[k] = {"us": 1e3 * ms, "share": ms / sum(per_kernel_ms.values())}
+        if abytes[k]:
+            gbs = abytes[k] / (ms / 1e3) / 1e9
+            kernels[k].update(gbs=gbs, frac_of_peak=gbs / peak)
+
+    cfg = workload_config(w)
+    gate_to_permute = sum(per_kernel_ms[k] for k in KERNELS[:5])
+    cfg.update(us_per_layer_gate_to_permute=1e3 * gate_to_permute,
+               us_per_layer_incl_combine=1e3 * sum(per_kernel_ms.values()),
+               parallelism=f"replicas: {world} independent layer instance(s), one per GPU")
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        lg_pin = torch.from_numpy(logits_h).pin_memory()
+        hd_pin = torch.from_numpy(hidden_h.view(np.int16)).pin_memory()
+        out_pin = torch.empty(L.out.shape, dtype=torch.float32).pin_memory()
+        st_pin = torch.empty(4, dtype=torch.int32).pin_memory()
+        rl_pin = torch.empty(w.R, dtype=torch.int32).pin_memory()
+
+        def e2e_step():
+            L.logits.copy_(lg_pin, non_blocking=True)
+            L.hidden.view(torch.int16).copy_(hd_pin, non_blocking=True)
+            step()
+            out_pin.copy_(L.out, non_blocking=True)
+            st_pin.copy_(L.stats, non_blocking=True)
+            rl_pin.copy_(L.rank_load, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, world, dev)
+        h2d = lg_pin.numel() * 4 + hd_pin.numel() * 2
+        d2h = out_pin.numel() * 4 + 4 * 4 + w.R * 4
+        e2e = {"value": world * w.Q / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "what": "pinned host logits + hidden -> device, full path, combine output + "
+                       "plan stats -> host, every step"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        pairs, secs, nsl = oracle_slices(w, logits_h, hidden_h, 512, 10.0, 8)
+        cpu = {"value": pairs / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{nsl} slice(s) of 512 tokens per rank x {w.R} ranks "
+                         f"({pairs} pairs, {secs:.1f} s), each a whole layer instance "
+                         f"through the single-threaded C oracle incl. permute and combine"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": len(steps_fn) * args.steps,
+            "clocks": clk, "kernels": kernels,
+            "imbalance": {"max_over_mean_before": float(plan0["stats"][1]) / (w.Q / w.R),
+                          "max_over_mean_after": float(plan0["stats"][2]) / (w.Q / w.R),
+                          "copies": int(plan0["stats"][0]),
+                          "colocated_copies": int(plan0["stats"][3])},
+        }
+        print(json.dumps(line), flush=True)
+    L.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,100 @@
+"""Device-side error paths, without faulting the GPU.
+
+Bad ids and rows are caught by the kernels' own bounds checks (the access is
+skipped and UE_ERR_DEVICE_BOUNDS recorded); a look-back wait is made to run
+out by a test hook that keeps the first reroute tile from publishing (a flag
+nothing sets) with a short poll limit, and must end with UE_ERR_TIMEOUT. After
+each error the same context keeps working and matches the oracle again.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import token_rerouting_b200 as ue
+from tests import gpu_helpers as gh
+
+pytestmark = pytest.mark.gpu
+
+R, T, E, K, S, d = 8, 512, 64, 4, 2, 64
+
+
+@pytest.fixture()
+def layer():
+    L = gh.make_layer(R, T, E, K, S, d)
+    yield L
+    L.close()
+
+
+def check_clean_run(L, logits):
+    gh.load_inputs(L, logits)
+    L.run_routing()
+    assert L.error() == ue.UE_OK
+    gh.assert_routing_equal(gh.routing_results(L), oracle.run_path(logits, R, T, S, K))
+
+
+def test_bad_expert_id_in_count_and_reroute(layer):
+    w = synth.custom(R, T, E, K, S, d, cid=501)
+    logits = synth.logits(w)
+    gh.load_inputs(layer, logits)
+    layer.run_routing()
+    assert layer.error() == ue.UE_OK
+    layer.idx[3, 1] = E + 7
+    layer.idx[100, 0] = -2
+    layer.count()
+    assert layer.error() == ue.UE_ERR_DEVICE_BOUNDS
+    layer.reroute()
+    assert layer.error() == ue.UE_ERR_DEVICE_BOUNDS
+    # the bad pairs get no slot and no row
+    assert int(layer.dest_row[3, 1]) == -1 and int(layer.phys_slot[100, 0]) == -1
+    check_clean_run(layer, logits)
+
+
+def test_rows_out_of_range_in_permute_and_combine(layer):
+    w = synth.custom(R, T, E, K, S, d, cid=502)
+    logits = synth.logits(w)
+    gh.load_inputs(layer, logits, synth.hidden(w))
+    layer.run_routing()
+    layer.dispatch.zero_()
+    layer.dest_row[0, 0] = -1
+    layer.dest_row[7, 2] = R * T * K + 5
+    layer.permute()
+    assert layer.error() == ue.UE_ERR_DEVICE_BOUNDS
+    layer.combine()
+    assert layer.error() == ue.UE_ERR_DEVICE_BOUNDS
+    check_clean_run(layer, logits)
+
+
+def test_negative_load_in_plan(layer):
+    load = torch.full((E,), 10, dtype=torch.int32, device=layer.device)
+    load[5] = -3
+    ue.ue_plan(layer.ctx, load, layer.plan)
+    assert layer.error() == ue.UE_ERR_DEVICE_BOUNDS
+
+
+def test_lookback_wait_runs_out_and_context_recovers(layer):
+    w = synth.custom(R, T, E, K, S, d, cid=503)
+    logits = synth.logits(w)
+    gh.load_inputs(layer, logits)
+    layer.run_routing()
+    assert layer.error() == ue.UE_OK
+    ue.ue_debug_set_lookback_limit(layer.ctx, 1000)
+    ue.ue_debug_drop_first_publish(layer.ctx, True)
+    layer.reroute()
+    assert layer.error() == ue.UE_ERR_TIMEOUT
+    ue.ue_debug_drop_first_publish(layer.ctx, False)
+    ue.ue_debug_set_lookback_limit(layer.ctx, 1 << 22)
+    check_clean_run(layer, logits)
+
+
+def test_host_rejects_misaligned_and_overlapping_rows(layer):
+    base = layer.hidden.view(torch.int16)
+    with pytest.raises(ue.UEError):
+        ue.ue_permute(layer.ctx, base.data_ptr() + 2, layer.dest_row, layer.dispatch)
+    with pytest.raises(ue.UEError):
+        ue.ue_permute(layer.ctx, layer.dispatch, layer.dest_row, layer.dispatch)
+    with pytest.raises(ue.UEError):
+        ue.ue_combine(layer.ctx, layer.dispatch, layer.dest_row, layer.w,
+                      layer.out.data_ptr() + 4)
+    assert layer.error() == ue.UE_OK

@@ -1,0 +1,235 @@
+// ue_api.cu -- the C ABI declared in include/ue.h: context, host-side
+// argument checks, and kernel launches. See ue.h for the contract of every
+// call.
+#include <cstdio>
+#include <cstdlib>
+#include <new>
+
+#include "ue_internal.cuh"
+
+struct ue_ctx {
+    ue_config cfg;
+    ue::Sizes z;
+    int device;
+    int num_sms;
+    int gate_grid;
+    ue::PermuteShape perm;
+    ue::CombineShape comb;
+    int* d_err;             // [2] error code, detail
+    uint32_t* d_status;     // [tiles][E] reroute look-back words
+    uint32_t* d_counter;    // reroute tile ticket
+    int64_t tiles;
+    int64_t spin_limit;
+    int drop_first;
+    uint32_t magic;
+};
+
+namespace {
+
+constexpr uint32_t kMagic = 0x75656331u;  // "uec1"
+
+bool config_ok(const ue_config& c)
+{
+    if (c.R < 1 || c.R > ue::kMaxR) return false;
+    if (c.E < 1 || c.E > ue::kMaxE || c.E % c.R != 0) return false;
+    if (c.K < 1 || c.K > ue::kMaxK || c.K > c.E) return false;
+    if (c.S < 0 || c.S > ue::kMaxS || c.R * c.S > ue::kMaxG) return false;
+    if (c.T < 1) return false;
+    if (c.d < 8 || c.d % 8 != 0 || c.d > ue::kMaxD) return false;
+    const int64_t Q = (int64_t)c.R * c.T * c.K;
+    if (Q >= (int64_t(1) << 30)) return false;
+    return true;
+}
+
+bool ctx_ok(const ue_ctx* ctx) { return ctx != nullptr && ctx->magic == kMagic; }
+
+bool aligned(const void* p, size_t a) { return p != nullptr && ((uintptr_t)p % a) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// make the context's device current (cheap when it already is)
+ue_status use_device(const ue_ctx* ctx)
+{
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return UE_ERR_CUDA;
+    if (cur != ctx->device && cudaSetDevice(ctx->device) != cudaSuccess) return UE_ERR_CUDA;
+    return UE_OK;
+}
+
+ue_status from_cuda(cudaError_t e) { return e == cudaSuccess ? UE_OK : UE_ERR_CUDA; }
+
+bool placement_ok(const ue_ctx* ctx, const ue_placement* p)
+{
+    if (p == nullptr) return false;
+    if (ctx->z.G > 0 && !aligned(p->slot_expert, 4)) return false;
+    return aligned(p->n_copies, 4) && aligned(p->slot_quota, 4) && aligned(p->slot_offset, 4) &&
+           aligned(p->rank_load, 4) && aligned(p->stats, 4);
+}
+
+}  // namespace
+
+extern "C" {
+
+ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
+{
+    if (out == nullptr) return UE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (cfg == nullptr || !config_ok(*cfg)) return UE_ERR_INVALID_ARG;
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess) return UE_ERR_CUDA;
+    if (device < 0 || device >= ndev) return UE_ERR_INVALID_ARG;
+    if (cudaSetDevice(device) != cudaSuccess) return UE_ERR_CUDA;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return UE_ERR_CUDA;
+    if (prop.major != 10) return UE_ERR_UNSUPPORTED;
+
+    ue_ctx* ctx = new (std::nothrow) ue_ctx();
+    if (ctx == nullptr) return UE_ERR_NOMEM;
+    ctx->cfg = *cfg;
+    ctx->z = ue::make_sizes(*cfg);
+    ctx->device = device;
+    ctx->num_sms = prop.multiProcessorCount;
+    ctx->gate_grid = ue::gate_topk_grid(ctx->z, ctx->num_sms);
+    ctx->tiles = (ctx->z.Q + ue::kRerouteTile - 1) / ue::kRerouteTile;
+    ctx->spin_limit = 1LL << 22;
+    ctx->drop_first = 0;
+
+    if (ue::plan_permute_shape(ctx->z, ctx->num_sms, &ctx->perm) != cudaSuccess ||
+        ue::plan_combine_shape(ctx->z, ctx->num_sms, &ctx->comb) != cudaSuccess) {
+        delete ctx;
+        cudaGetLastError();
+        return UE_ERR_CUDA;
+    }
+
+    const size_t status_words = (size_t)std::max<int64_t>(ctx->tiles, 1) * ctx->z.E;
+    if (cudaMalloc(&ctx->d_err, 2 * sizeof(int)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_status, status_words * sizeof(uint32_t)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_counter, sizeof(uint32_t)) != cudaSuccess) {
+        cudaFree(ctx->d_err);
+        cudaFree(ctx->d_status);
+        cudaFree(ctx->d_counter);
+        delete ctx;
+        cudaGetLastError();
+        return UE_ERR_NOMEM;
+    }
+    if (cudaMemset(ctx->d_err, 0, 2 * sizeof(int)) != cudaSuccess ||
+        cudaMemset(ctx->d_status, 0, status_words * sizeof(uint32_t)) != cudaSuccess ||
+        cudaMemset(ctx->d_counter, 0, sizeof(uint32_t)) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess) {
+        cudaFree(ctx->d_err);
+        cudaFree(ctx->d_status);
+        cudaFree(ctx->d_counter);
+        delete ctx;
+        return UE_ERR_CUDA;
+    }
+    ctx->magic = kMagic;
+    *out = ctx;
+    return UE_OK;
+}
+
+ue_status ue_destroy(ue_ctx* ctx)
+{
+    if (ctx == nullptr) return UE_OK;
+    if (!ctx_ok(ctx)) return UE_ERR_INVALID_ARG;
+    ue_status st = use_device(ctx);
+    if (st == UE_OK && cudaDeviceSynchronize() != cudaSuccess) st = UE_ERR_CUDA;
+    cudaFree(ctx->d_err);
+    cudaFree(ctx->d_status);
+    cudaFree(ctx->d_counter);
+    ctx->magic = 0;
+    delete ctx;
+    return st;
+}
+
+ue_status ue_get_error(ue_ctx* ctx, void* stream)
+{
+    if (!ctx_ok(ctx)) return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    int h[2] = {0, 0};
+    if (cudaStreamSynchronize(st) != cudaSuccess) return UE_ERR_CUDA;
+    if (cudaMemcpyAsync(h, ctx->d_err, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return UE_ERR_CUDA;
+    if (cudaMemsetAsync(ctx->d_err, 0, sizeof(h), st) != cudaSuccess) return UE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return UE_ERR_CUDA;
+    return (ue_status)h[0];
+}
+
+ue_status ue_gate_topk(ue_ctx* ctx, const float* logits, int32_t* idx, float* w, void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(logits, 4) || !aligned(idx, 4) || !aligned(w, 4))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_gate_topk(ctx->z, logits, idx, w, ctx->gate_grid,
+                                          as_stream(stream)));
+}
+
+ue_status ue_count(ue_ctx* ctx, const int32_t* idx, int32_t* load_re, int32_t* load_e,
+                   void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(idx, 4) || !aligned(load_re, 4) || !aligned(load_e, 4))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_count(ctx->z, idx, load_re, load_e, ctx->d_err,
+                                      as_stream(stream)));
+}
+
+ue_status ue_plan(ue_ctx* ctx, const int32_t* load_e, const ue_placement* out, void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(load_e, 4) || !placement_ok(ctx, out))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_plan(ctx->z, load_e, *out, ctx->d_err, as_stream(stream)));
+}
+
+ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
+                     int32_t* phys_slot, int32_t* dest_row, void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(idx, 4) || !placement_ok(ctx, plan) ||
+        !aligned(phys_slot, 4) || !aligned(dest_row, 4))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_reroute(ctx->z, idx, *plan, phys_slot, dest_row, ctx->d_status,
+                                        ctx->d_counter, ctx->spin_limit, ctx->drop_first,
+                                        ctx->d_err, as_stream(stream)));
+}
+
+ue_status ue_permute(ue_ctx* ctx, const uint16_t* hidden, const int32_t* dest_row,
+                     uint16_t* dispatch, void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(hidden, 16) || !aligned(dest_row, 4) || !aligned(dispatch, 16))
+        return UE_ERR_INVALID_ARG;
+    const size_t hb = (size_t)ctx->z.N * ctx->z.d * 2, db = (size_t)ctx->z.Q * ctx->z.d * 2;
+    const uintptr_t h0 = (uintptr_t)hidden, d0 = (uintptr_t)dispatch;
+    if (h0 < d0 + db && d0 < h0 + hb) return UE_ERR_INVALID_ARG;  // overlap
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_permute(ctx->z, ctx->perm, hidden, dest_row, dispatch,
+                                        ctx->d_err, as_stream(stream)));
+}
+
+ue_status ue_combine(ue_ctx* ctx, const uint16_t* y, const int32_t* dest_row, const float* w,
+                     float* out, void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(y, 16) || !aligned(dest_row, 4) || !aligned(w, 4) ||
+        !aligned(out, 16))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_combine(ctx->z, ctx->comb, y, dest_row, w, out, ctx->d_err,
+                                        as_stream(stream)));
+}
+
+ue_status ue_debug_set_lookback_limit(ue_ctx* ctx, int64_t polls)
+{
+    if (!ctx_ok(ctx) || polls < 0) return UE_ERR_INVALID_ARG;
+    ctx->spin_limit = polls;
+    return UE_OK;
+}
+
+ue_status ue_debug_drop_first_publish(ue_ctx* ctx, int enable)
+{
+    if (!ctx_ok(ctx)) return UE_ERR_INVALID_ARG;
+    ctx->drop_first = enable ? 1 : 0;
+    return UE_OK;
+}
+
+}  // extern "C"

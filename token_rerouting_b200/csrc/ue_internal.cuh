@@ -2,6 +2,8 @@
 // units (kernels + C ABI). Not installed, not part of the ABI.
 #pragma once
 
+#include <algorithm>
+#include <climits>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -72,12 +74,25 @@ cudaError_t launch_reroute(const Sizes& z, const int32_t* idx,
                            int32_t* dest_row, uint32_t* status,
                            uint32_t* tile_counter, int64_t spin_limit,
                            int drop_first, int* err, cudaStream_t st);
-cudaError_t launch_permute(const Sizes& z, const uint16_t* hidden,
-                           const int32_t* dest_row, uint16_t* dispatch,
-                           int num_sms, int* err, cudaStream_t st);
-cudaError_t launch_combine(const Sizes& z, const uint16_t* y,
-                           const int32_t* dest_row, const float* w, float* out,
-                           int num_sms, int* err, cudaStream_t st);
+// Launch shapes of the row kernels, fixed once per context (ue_init) so that
+// a call only enqueues work (nothing else touches the runtime, which keeps
+// the calls safe under stream capture).
+struct PermuteShape {
+    int grid, warps, nst;
+    size_t smem;
+};
+struct CombineShape {
+    int grid, tpt;
+};
+cudaError_t plan_permute_shape(const Sizes& z, int num_sms, PermuteShape* out);
+cudaError_t plan_combine_shape(const Sizes& z, int num_sms, CombineShape* out);
+
+cudaError_t launch_permute(const Sizes& z, const PermuteShape& sh, const uint16_t* hidden,
+                           const int32_t* dest_row, uint16_t* dispatch, int* err,
+                           cudaStream_t st);
+cudaError_t launch_combine(const Sizes& z, const CombineShape& sh, const uint16_t* y,
+                           const int32_t* dest_row, const float* w, float* out, int* err,
+                           cudaStream_t st);
 
 int gate_topk_grid(const Sizes& z, int num_sms);
 
