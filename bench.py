@@ -247,14 +247,20 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ue", "reference"), default="ue")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--tokens-per-rank", type=int, default=0,
+                    help="shrink T (profiling runs on a small case)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
+    import dataclasses
+
     import synth
     w = synth.WORKLOADS[args.workload]
+    if args.tokens_per_rank:
+        w = dataclasses.replace(w, T=args.tokens_per_rank, name=f"{w.name}_t{args.tokens_per_rank}")
     if args.impl == "reference":
         run_reference(args, w)
         return
