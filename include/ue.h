@@ -192,6 +192,28 @@ ue_status ue_permute(ue_ctx* ctx, const uint16_t* hidden,
 ue_status ue_combine(ue_ctx* ctx, const uint16_t* y, const int32_t* dest_row,
                      const float* w, float* out, void* stream);
 
+/* ue_reroute, without a context and without allocating anything (the
+ * pages have no counterpart to this call). For callers that cannot call
+ * cudaMalloc: code running inside an allocator's hooks or under a memory
+ * pool that forbids outside allocations, or code that keeps no context.
+ * The look-back scratch is a fixed device array inside libue (2 MiB plus a
+ * few words, held on every GPU that loads the library until the process
+ * exits): sizes with ceil(R*T*K / 2048) * E > 524288 are rejected with
+ * UE_ERR_UNSUPPORTED before anything is launched. The first call made with
+ * a given device current looks up that array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture. Every call shares the array: it clears the words it uses
+ * on `stream` first, and calls that overlap on the GPU (other streams, other
+ * threads) race and give wrong results. Calls no cudaMalloc or cudaFree.
+ *   cfg, idx, plan, phys_slot, dest_row, stream: as for ue_init + ue_reroute
+ *   (cfg is a host pointer, read during the call).
+ *   error: device int32[2], zeroed by the caller; a device-side error writes
+ *   {code, detail} into it (the first one only). NULL: errors are dropped.
+ * Host-side errors are returned at once, as for ue_reroute. */
+ue_status ue_reroute_noalloc(const ue_config* cfg, const int32_t* idx,
+                             const ue_placement* plan, int32_t* phys_slot,
+                             int32_t* dest_row, int32_t* error, void* stream);
+
 /* Test hooks for the bounded waits (no counterpart on the pages).
  * ue_debug_set_lookback_limit sets the number of polls a reroute tile makes
  * on a predecessor before it gives up with UE_ERR_TIMEOUT (default 1<<22,

@@ -32,7 +32,7 @@ UE_ERR_DEVICE_BOUNDS, UE_ERR_TIMEOUT, UE_ERR_UNSUPPORTED = 4, 5, 6
 
 # every symbol include/ue.h declares
 EXPORTS = ("ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count",
-           "ue_plan", "ue_reroute", "ue_permute", "ue_combine",
+           "ue_plan", "ue_reroute", "ue_permute", "ue_combine", "ue_reroute_noalloc",
            "ue_debug_set_lookback_limit", "ue_debug_drop_first_publish")
 
 
@@ -76,6 +76,8 @@ def load_library(path: str | None = None):
     lib.ue_reroute.argtypes = [vp, vp, ctypes.POINTER(ue_placement), vp, vp, vp]
     lib.ue_permute.argtypes = [vp, vp, vp, vp, vp]
     lib.ue_combine.argtypes = [vp, vp, vp, vp, vp, vp]
+    lib.ue_reroute_noalloc.argtypes = [ctypes.POINTER(ue_config), vp,
+                                       ctypes.POINTER(ue_placement), vp, vp, vp, vp]
     lib.ue_debug_set_lookback_limit.argtypes = [vp, i64]
     lib.ue_debug_drop_first_publish.argtypes = [vp, i32]
     for name in EXPORTS:
@@ -166,6 +168,15 @@ def ue_combine(ctx, y, dest_row, w, out, stream=None):
                                                 _ptr(out), _stream(stream)))
 
 
+def ue_reroute_noalloc(cfg: ue_config, idx, plan: ue_placement, phys_slot, dest_row,
+                       error=None, stream=None):
+    """ue_reroute without a context; allocates nothing (see include/ue.h)."""
+    _ok("ue_reroute_noalloc",
+        load_library().ue_reroute_noalloc(ctypes.byref(cfg), _ptr(idx), ctypes.byref(plan),
+                                          _ptr(phys_slot), _ptr(dest_row), _ptr(error),
+                                          _stream(stream)))
+
+
 def ue_debug_set_lookback_limit(ctx, polls: int):
     _ok("ue_debug_set_lookback_limit",
         load_library().ue_debug_set_lookback_limit(ctx, polls))
@@ -179,6 +190,7 @@ def ue_debug_drop_first_publish(ctx, enable: bool):
 from .layer import Layer  # noqa: E402  (buffers + one call per step)
 
 __all__ = ["ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count", "ue_plan",
-           "ue_reroute", "ue_permute", "ue_combine", "ue_debug_set_lookback_limit",
+           "ue_reroute", "ue_permute", "ue_combine", "ue_reroute_noalloc",
+           "ue_debug_set_lookback_limit",
            "ue_debug_drop_first_publish", "ue_config", "ue_placement", "make_config",
            "placement", "load_library", "Layer", "UEError", "STATUS", "EXPORTS"]
