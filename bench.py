@@ -40,9 +40,36 @@ KERNELS = ("gate_topk", "count", "plan", "reroute", "permute", "combine")
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# one ncu capture, with the SHA-256 of the kernel source it was taken on; a
-# kernel changed since then reports null.
-TRAFFIC = {}
+# one ncu --set full capture of the same workload at 512 tokens per rank,
+# scaled by 8 to the full 4096 tokens per rank (every kernel's traffic grows
+# in proportion to the tokens), with the SHA-256 prefix of the kernel source
+# it was taken on; a kernel changed since then reports null.
+TRAFFIC = {
+    "gate_topk": {
+        "bytes_per_launch": 134512000,
+        "source_sha": "eecff9157bbb7231"
+    },
+    "count": {
+        "bytes_per_launch": 8736000,
+        "source_sha": "27ba6f511329134d"
+    },
+    "plan": {
+        "bytes_per_launch": 224000,
+        "source_sha": "d88f84a3510d0295"
+    },
+    "reroute": {
+        "bytes_per_launch": 8888000,
+        "source_sha": "897786029bfb7b7a"
+    },
+    "permute": {
+        "bytes_per_launch": 18861456000,
+        "source_sha": "ec9d69b3006e5e8d"
+    },
+    "combine": {
+        "bytes_per_launch": 21233264000,
+        "source_sha": "c91a07d4eae7b00b"
+    },
+}
 
 
 def sha_of(path):
@@ -348,7 +375,8 @@ def main():
     achieved = abytes[dom] / (per_kernel_ms[dom] / 1e3) / 1e9
     tr = TRAFFIC.get(dom)
     src = os.path.join(ROOT, "token_rerouting_b200", "csrc", KERNEL_SRC[dom])
-    traffic = tr["bytes_per_launch"] if tr and tr.get("source_sha") == sha_of(src) else None
+    traffic = (tr["bytes_per_launch"] if tr and tr.get("source_sha") == sha_of(src)
+               and w.name == DEFAULT_WORKLOAD else None)
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "peak_kind": f"of {peak_kind}",
                 "traffic": traffic, "algorithmic_bytes": abytes[dom]}
