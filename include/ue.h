@@ -96,7 +96,7 @@ typedef struct ue_ctx ue_ctx; /* opaque */
 
 /* Create a context for `cfg` on CUDA device `device` (made current) and
  * allocate its scratch once: the error word and the reroute's look-back
- * status words (ceil(Q/2048)*E 32-bit words plus a tile counter). Nothing
+ * status words (ceil(Q/4096)*E 32-bit words plus a tile counter). Nothing
  * is allocated after this call ("Interface / 1. Initialization": buffers
  * reserved up front, no dynamic allocation at runtime).
  * Returns UE_ERR_INVALID_ARG for a null `out` or a config outside the
@@ -162,7 +162,7 @@ ue_status ue_plan(ue_ctx* ctx, const int32_t* load_e, const ue_placement* out,
  * first, then replicas by ascending g): the o-th pair of expert e goes to
  * the copy whose quota range holds o, at row slot_offset[p] + (o - start).
  * dest_row is a permutation of [0, Q). Single pass: a stable counting sort
- * with a decoupled look-back scan over tiles of 2048 pairs; its waits are
+ * with a decoupled look-back scan over tiles of 4096 pairs; its waits are
  * bounded and end with UE_ERR_TIMEOUT. Ids outside [0, E) set
  * UE_ERR_DEVICE_BOUNDS. */
 ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
@@ -198,7 +198,7 @@ ue_status ue_combine(ue_ctx* ctx, const uint16_t* y, const int32_t* dest_row,
  * pool that forbids outside allocations, or code that keeps no context.
  * The look-back scratch is a fixed device array inside libue (2 MiB plus a
  * few words, held on every GPU that loads the library until the process
- * exits): sizes with ceil(R*T*K / 2048) * E > 524288 are rejected with
+ * exits): sizes with ceil(R*T*K / 4096) * E > 524288 are rejected with
  * UE_ERR_UNSUPPORTED before anything is launched. The first call made with
  * a given device current looks up that array's device address
  * (cudaGetSymbolAddress) and caches it; make that first call before any

@@ -39,11 +39,67 @@ __device__ __forceinline__ float key_value(uint32_t k)
     return __uint_as_float(u);
 }
 
-template <int VPL>
-__global__ void __launch_bounds__(kGateThreads)
-gate_topk_kernel(const float* __restrict__ logits, int64_t N, int E, int K,
-                 int rpg, int32_t* __restrict__ idx, float* __restrict__ w)
+// Selection of one row's top-K from the lane's VPL logits (expert ids
+// lane + 32 j); lane (base + k) records round k's winner.
+template <int VPL, int KT>
+__device__ __forceinline__ void select_row(const float (&v)[VPL], int E, int K, int base,
+                                           int lane, uint32_t& cap_key, uint32_t& cap_e)
 {
+    uint32_t key[VPL];
+    uint32_t ke[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        const int e = lane + 32 * j;
+        key[j] = (e < E) ? order_key(v[j]) : 0u;
+        ke[j] = (uint32_t)e;
+    }
+    // stable descending sort of the lane's keys; ids ascend with j, so equal
+    // keys keep the lower id first
+#pragma unroll
+    for (int pass = 0; pass < VPL - 1; ++pass) {
+#pragma unroll
+        for (int j = 0; j < VPL - 1 - pass; ++j) {
+            const bool sw = key[j + 1] > key[j];
+            const uint32_t k0 = key[j], k1 = key[j + 1];
+            const uint32_t e0 = ke[j], e1 = ke[j + 1];
+            key[j] = sw ? k1 : k0;
+            key[j + 1] = sw ? k0 : k1;
+            ke[j] = sw ? e1 : e0;
+            ke[j + 1] = sw ? e0 : e1;
+        }
+    }
+    constexpr int KU = KT > 0 ? KT : kMaxK;
+#pragma unroll
+    for (int k = 0; k < KU; ++k) {
+        if (KT == 0 && k >= K) break;
+        const uint32_t m = __reduce_max_sync(kFull, key[0]);
+        const uint32_t cand = (key[0] == m) ? ke[0] : 0xffffffffu;
+        const uint32_t ew = __reduce_min_sync(kFull, cand);
+        if (lane == base + k) {
+            cap_key = m;
+            cap_e = ew;
+        }
+        const bool pop = (ke[0] == ew);
+#pragma unroll
+        for (int j = 0; j < VPL - 1; ++j) {
+            key[j] = pop ? key[j + 1] : key[j];
+            ke[j] = pop ? ke[j + 1] : ke[j];
+        }
+        if (pop) {
+            key[VPL - 1] = 0u;
+            ke[VPL - 1] = 0xfffffffeu;
+        }
+    }
+}
+
+// KT > 0: K == KT at compile time; KT == 0: any K <= 32.
+template <int VPL, int KT>
+__global__ void __launch_bounds__(kGateThreads)
+gate_topk_kernel(const float* __restrict__ logits, int64_t N, int E, int Krt,
+                 int32_t* __restrict__ idx, float* __restrict__ w)
+{
+    const int K = KT > 0 ? KT : Krt;
+    const int rpg = 32 / K;  // rows per warp group
     const int lane = threadIdx.x & 31;
     const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -68,52 +124,16 @@ gate_topk_kernel(const float* __restrict__ logits, int64_t N, int E, int K,
                     v[b][j] = (rowok && e < E) ? __ldcs(src + e) : 0.0f;
                 }
             }
+            if (rb + kGateBatch <= rows) {
+                // full batch: no row-count branches, consecutive rows interleave
 #pragma unroll
-            for (int b = 0; b < kGateBatch; ++b) {
-                if (rb + b >= rows) break;  // warp-uniform
-                uint32_t key[VPL];
-                uint32_t ke[VPL];
+                for (int b = 0; b < kGateBatch; ++b)
+                    select_row<VPL, KT>(v[b], E, K, (rb + b) * K, lane, cap_key, cap_e);
+            } else {
 #pragma unroll
-                for (int j = 0; j < VPL; ++j) {
-                    const int e = lane + 32 * j;
-                    key[j] = (e < E) ? order_key(v[b][j]) : 0u;
-                    ke[j] = (uint32_t)e;
-                }
-                // stable descending sort of the lane's keys; ids ascend with
-                // j, so equal keys keep the lower id first
-#pragma unroll
-                for (int pass = 0; pass < VPL - 1; ++pass) {
-#pragma unroll
-                    for (int j = 0; j < VPL - 1 - pass; ++j) {
-                        const bool sw = key[j + 1] > key[j];
-                        const uint32_t k0 = key[j], k1 = key[j + 1];
-                        const uint32_t e0 = ke[j], e1 = ke[j + 1];
-                        key[j] = sw ? k1 : k0;
-                        key[j + 1] = sw ? k0 : k1;
-                        ke[j] = sw ? e1 : e0;
-                        ke[j + 1] = sw ? e0 : e1;
-                    }
-                }
-                const int base = (rb + b) * K;
-                for (int k = 0; k < K; ++k) {
-                    const uint32_t m = __reduce_max_sync(kFull, key[0]);
-                    const uint32_t cand = (key[0] == m) ? ke[0] : 0xffffffffu;
-                    const uint32_t ew = __reduce_min_sync(kFull, cand);
-                    if (lane == base + k) {
-                        cap_key = m;
-                        cap_e = ew;
-                    }
-                    const bool pop = (ke[0] == ew);
-#pragma unroll
-                    for (int j = 0; j < VPL - 1; ++j) {
-                        key[j] = pop ? key[j + 1] : key[j];
-                        ke[j] = pop ? ke[j + 1] : ke[j];
-                    }
-                    if (pop) {
-                        key[VPL - 1] = 0u;
-                        ke[VPL - 1] = 0xfffffffeu;
-                    }
-                }
+                for (int b = 0; b < kGateBatch; ++b)
+                    if (rb + b < rows)
+                        select_row<VPL, KT>(v[b], E, K, (rb + b) * K, lane, cap_key, cap_e);
             }
         }
 
@@ -126,7 +146,12 @@ gate_topk_kernel(const float* __restrict__ logits, int64_t N, int E, int K,
         const double v0 = __shfl_sync(kFull, v_own, lead);
         const double x = act ? exp(v_own - v0) : 0.0;
         double z = 0.0;
-        for (int kk = 0; kk < K; ++kk) z += __shfl_sync(kFull, x, act ? lead + kk : 0);
+        constexpr int KU = KT > 0 ? KT : kMaxK;
+#pragma unroll
+        for (int kk = 0; kk < KU; ++kk) {
+            if (KT == 0 && kk >= K) break;
+            z += __shfl_sync(kFull, x, act ? lead + kk : 0);
+        }
         if (act) {
             const int64_t pos = (row0 + r) * (int64_t)K + k;
             idx[pos] = (int32_t)cap_e;
@@ -139,9 +164,12 @@ template <int VPL>
 cudaError_t launch_vpl(const Sizes& z, const float* logits, int32_t* idx,
                        float* w, int grid, cudaStream_t st)
 {
-    const int rpg = 32 / z.K;
-    gate_topk_kernel<VPL><<<grid, kGateThreads, 0, st>>>(logits, z.N, z.E, z.K,
-                                                         rpg, idx, w);
+    if (z.K == 8)
+        gate_topk_kernel<VPL, 8><<<grid, kGateThreads, 0, st>>>(logits, z.N, z.E, z.K, idx, w);
+    else if (z.K == 4)
+        gate_topk_kernel<VPL, 4><<<grid, kGateThreads, 0, st>>>(logits, z.N, z.E, z.K, idx, w);
+    else
+        gate_topk_kernel<VPL, 0><<<grid, kGateThreads, 0, st>>>(logits, z.N, z.E, z.K, idx, w);
     return cudaGetLastError();
 }
 

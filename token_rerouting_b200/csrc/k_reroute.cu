@@ -9,17 +9,20 @@
 // With the plan's quotas q_j = b + [j < rem] (b = floor(L/c), rem = L mod c),
 // j and the offset follow from o by one division.
 //
-// Design (B200): a single-pass stable counting sort. Each CTA takes a tile of
-// 2048 pairs by an atomic ticket (so every tile it waits on is already
-// running), stages the tile's ids in shared memory, and counts them per warp
-// sub-range with __match_any_sync. It publishes its per-expert tile counts
-// and then looks back over predecessor tiles, one thread per expert column,
-// until it finds an inclusive prefix (decoupled look-back). Every wait is
-// bounded: when it runs out the tile publishes an error flag, records
-// UE_ERR_TIMEOUT and writes nothing. Finally each warp re-walks its 256 pairs
-// in order, ranking equal ids within 32 lanes by popcount, and writes the
-// physical slot and dispatch row. The plan's copy lists are rebuilt per CTA
-// from slot_expert / slot_quota / slot_offset (at most 512 entries).
+// Design (B200): a single-pass stable counting sort with a decoupled
+// look-back. Each CTA takes a tile of 4096 pairs by an atomic ticket (so every
+// tile it waits on is already running), stages the ids in shared memory and
+// counts them per warp sub-range, then publishes its per-expert tile counts
+// at once so that successors never wait on its later work. While its
+// predecessors finish, it rebuilds the plan's copy lists (at most 512
+// entries). The look-back runs one thread per expert column and reads a
+// window of 16 predecessors per step with independent loads, adding their
+// counts until it meets an inclusive prefix; with every tile resident at
+// once this cuts the serial chain of L2 round trips by the window width.
+// Every wait is bounded: when it runs out the tile publishes an error flag,
+// records UE_ERR_TIMEOUT and writes nothing. Finally each warp re-walks its
+// 512 pairs in order, ranking equal ids within 32 lanes by popcount of the
+// lanes that match, and writes the physical slot and dispatch row.
 #include "ue_internal.cuh"
 
 namespace ue {
@@ -30,6 +33,7 @@ constexpr int kThreads = kRerouteThreads;
 constexpr int kWarps = kRerouteWarps;
 constexpr int kPerWarp = kTile / kWarps;
 constexpr int kRounds = kPerWarp / 32;
+constexpr int kWindow = 16;  // predecessors read per look-back step
 
 __device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p)
 {
@@ -50,13 +54,17 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
                uint32_t* tile_counter, int64_t spin_limit, int drop_first,
                int* err)
 {
-    __shared__ int s_idx[kTile];
+    __shared__ short s_idx[kTile];        // expert ids of the tile (-1: none)
     __shared__ int s_wh[kWarps][kMaxE];   // per-warp counts, then start offsets
-    __shared__ int s_agg[kMaxE];          // tile counts, then tile prefix
+    __shared__ int s_pre[kMaxE];          // tile prefix per expert
+    __shared__ int s_cnt[kMaxE], s_lrep[kMaxE], s_run[kMaxE];
     __shared__ int s_L[kMaxE], s_b[kMaxE], s_rem[kMaxE];
     __shared__ int s_master[kMaxE], s_repstart[kMaxE];
     __shared__ int s_rep[kMaxG];          // replica slots, by expert then g
     __shared__ int s_off[kMaxE + kMaxG + 1];
+    __shared__ int s_se[kMaxG];           // plan: slot_expert
+    __shared__ int s_sq[kMaxE + kMaxG];   // plan: slot_quota
+    __shared__ int s_wsum[kWarps];
     __shared__ int s_tile;
     __shared__ int s_fail;
 
@@ -66,29 +74,69 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
-    int* cnt = s_wh[0];   // prologue scratch, reset before the histogram
-    int* lrep = s_wh[1];
-    int* run = s_wh[2];
 
     if (tid == 0) {
         s_tile = (int)atomicAdd(tile_counter, 1u);
         s_fail = 0;
     }
-    for (int p = tid; p <= P; p += kThreads) s_off[p] = __ldg(plan.slot_offset + p);
+    for (int x = tid; x < kWarps * kMaxE; x += kThreads) (&s_wh[0][0])[x] = 0;
     for (int e = tid; e < E; e += kThreads) {
-        cnt[e] = 0;
-        lrep[e] = 0;
-        run[e] = 0;
+        s_cnt[e] = 0;
+        s_lrep[e] = 0;
+        s_run[e] = 0;
     }
     __syncthreads();
 
-    // ---- copy lists of every expert, from the plan ----
+    // ---- stage the tile and count it per warp sub-range ----
+    const int tile = s_tile;
+    const int64_t t0 = (int64_t)tile * kTile;
+    const int cnt_tile = (int)min((int64_t)kTile, Q - t0);
+    for (int x = tid; x < kTile; x += kThreads) {
+        int e = -1;
+        if (x < cnt_tile) {
+            e = __ldg(idx + t0 + x);
+            if ((unsigned)e >= (unsigned)E) {
+                raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(t0 + x, (int64_t)INT_MAX));
+                e = -1;
+            }
+        }
+        s_idx[x] = (short)e;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int rd = 0; rd < kRounds; ++rd) {
+        const int e = s_idx[warp * kPerWarp + rd * 32 + lane];
+        if (e >= 0) atomicAdd(&s_wh[warp][e], 1);
+    }
+    __syncthreads();
+
+    // ---- publish this tile's counts ----
+    int acc = 0;
+    uint32_t* mine = status + (size_t)tile * E + tid;
+    if (tid < E) {
+        for (int w = 0; w < kWarps; ++w) {
+            const int t = s_wh[w][tid];
+            s_wh[w][tid] = acc;
+            acc += t;
+        }
+        if (tile == 0) {
+            if (!drop_first) st_relaxed(mine, (kFlagPrefix << 30) | (uint32_t)acc);
+        } else {
+            st_relaxed(mine, (kFlagAggregate << 30) | (uint32_t)acc);
+        }
+    }
+
+    // ---- copy lists of every expert, from the plan (overlaps the wait) ----
+    for (int p = tid; p <= P; p += kThreads) s_off[p] = __ldg(plan.slot_offset + p);
+    for (int p = tid; p < P; p += kThreads) s_sq[p] = __ldg(plan.slot_quota + p);
+    for (int g = tid; g < G; g += kThreads) s_se[g] = __ldg(plan.slot_expert + g);
+    __syncthreads();
     for (int g = tid; g < G; g += kThreads) {
-        const int e = __ldg(plan.slot_expert + g);
+        const int e = s_se[g];
         if (e >= 0 && e < E) {
             const int p = (g / S) * (M + S) + M + (g % S);
-            atomicAdd(&cnt[e], 1);
-            atomicAdd(&lrep[e], __ldg(plan.slot_quota + p));
+            atomicAdd(&s_cnt[e], 1);
+            atomicAdd(&s_lrep[e], s_sq[p]);
         } else if (e >= E) {
             raise_error(err, UE_ERR_DEVICE_BOUNDS, g);
         }
@@ -96,22 +144,22 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     __syncthreads();
     {
         // exclusive scan of replica counts over experts (E <= kThreads)
-        const int c = tid < E ? cnt[tid] : 0;
+        const int c = tid < E ? s_cnt[tid] : 0;
         int incl = c;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int o = __shfl_up_sync(kFull, incl, off);
             if (lane >= off) incl += o;
         }
-        if (lane == 31) s_agg[warp] = incl;
+        if (lane == 31) s_wsum[warp] = incl;
         __syncthreads();
         int wofs = 0;
-        for (int w = 0; w < warp; ++w) wofs += s_agg[w];
+        for (int w = 0; w < warp; ++w) wofs += s_wsum[w];
         if (tid < E) {
             const int e = tid;
             const int mp = (e / M) * (M + S) + (e % M);
             const int copies = 1 + c;
-            const int L = __ldg(plan.slot_quota + mp) + lrep[e];
+            const int L = s_sq[mp] + s_lrep[e];
             const int b = L / copies;
             s_L[e] = L;
             s_b[e] = b;
@@ -127,98 +175,70 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
             const int g = g0 + lane;
             int e = -1;
             if (g < G) {
-                e = __ldg(plan.slot_expert + g);
+                e = s_se[g];
                 if (e >= E) e = -1;
             }
             const unsigned peers = __match_any_sync(kFull, e);
             if (e >= 0) {
-                const int pos = run[e] + __popc(peers & ((1u << lane) - 1u));
+                const int pos = s_run[e] + __popc(peers & ((1u << lane) - 1u));
                 s_rep[s_repstart[e] + pos] = (g / S) * (M + S) + M + (g % S);
             }
             __syncwarp();
-            if (e >= 0 && lane == __ffs(peers) - 1) run[e] += __popc(peers);
+            if (e >= 0 && lane == __ffs(peers) - 1) s_run[e] += __popc(peers);
             __syncwarp();
         }
     }
-    __syncthreads();
 
-    // ---- stage the tile, count per warp sub-range ----
-    const int tile = s_tile;
-    const int64_t t0 = (int64_t)tile * kTile;
-    const int cnt_tile = (int)min((int64_t)kTile, Q - t0);
-    for (int x = tid; x < kTile; x += kThreads) {
-        int e = -1;
-        if (x < cnt_tile) {
-            e = __ldg(idx + t0 + x);
-            if ((unsigned)e >= (unsigned)E) {
-                raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(t0 + x, (int64_t)INT_MAX));
-                e = -1;
-            }
-        }
-        s_idx[x] = e;
-    }
-    for (int x = tid; x < kWarps * kMaxE; x += kThreads) (&s_wh[0][0])[x] = 0;
-    __syncthreads();
-#pragma unroll 1
-    for (int rd = 0; rd < kRounds; ++rd) {
-        const int e = s_idx[warp * kPerWarp + rd * 32 + lane];
-        const unsigned peers = __match_any_sync(kFull, e);
-        if (e >= 0 && lane == __ffs(peers) - 1) s_wh[warp][e] += __popc(peers);
-        __syncwarp();
-    }
-    __syncthreads();
-
-    // ---- publish tile counts, look back, publish inclusive prefix ----
+    // ---- look back over predecessor tiles, publish the inclusive prefix ----
     if (tid < E) {
-        int acc = 0;
-        for (int w = 0; w < kWarps; ++w) {
-            const int t = s_wh[w][tid];
-            s_wh[w][tid] = acc;
-            acc += t;
-        }
-        uint32_t* mine = status + (size_t)tile * E + tid;
         if (tile == 0) {
-            if (!drop_first) st_relaxed(mine, (kFlagPrefix << 30) | (uint32_t)acc);
-            s_agg[tid] = 0;
+            s_pre[tid] = 0;
         } else {
-            st_relaxed(mine, (kFlagAggregate << 30) | (uint32_t)acc);
             uint32_t excl = 0;
-            int pred = tile - 1;
+            int base = tile - 1;  // nearest predecessor not yet added
             int64_t polls = 0;
-            bool fail = false;
-            for (;;) {
-                const uint32_t sw = ld_relaxed(status + (size_t)pred * E + tid);
-                const uint32_t flag = sw >> 30;
-                if (flag == kFlagInvalid) {
-                    if (++polls > spin_limit) {
-                        raise_error(err, UE_ERR_TIMEOUT, tile);
-                        fail = true;
-                        break;
+            bool fail = false, done = false;
+            while (!done && !fail) {
+                uint32_t v[kWindow];
+#pragma unroll
+                for (int i = 0; i < kWindow; ++i)
+                    v[i] = (base - i >= 0) ? ld_relaxed(status + (size_t)(base - i) * E + tid)
+                                           : (kFlagPrefix << 30);
+#pragma unroll
+                for (int i = 0; i < kWindow; ++i) {
+                    if (!done && !fail) {
+                        uint32_t sw = v[i];
+                        while ((sw >> 30) == kFlagInvalid && !fail) {
+                            if (++polls > spin_limit) {
+                                raise_error(err, UE_ERR_TIMEOUT, tile);
+                                fail = true;
+                            } else {
+                                __nanosleep(64);
+                                sw = ld_relaxed(status + (size_t)(base - i) * E + tid);
+                            }
+                        }
+                        if ((sw >> 30) == kFlagError) fail = true;
+                        if (!fail) {
+                            if (base - i >= 0) excl += sw & kValueMask;
+                            if ((sw >> 30) == kFlagPrefix) done = true;
+                        }
                     }
-                    __nanosleep(64);
-                    continue;
                 }
-                if (flag == kFlagError) {
-                    fail = true;
-                    break;
-                }
-                excl += sw & kValueMask;
-                if (flag == kFlagPrefix) break;
-                --pred;
+                base -= kWindow;
             }
             if (fail) {
                 st_relaxed(mine, kFlagError << 30);
                 atomicOr(&s_fail, 1);
             } else {
                 st_relaxed(mine, (kFlagPrefix << 30) | ((excl + (uint32_t)acc) & kValueMask));
-                s_agg[tid] = (int)excl;
+                s_pre[tid] = (int)excl;
             }
         }
     }
     __syncthreads();
     if (s_fail) return;
     if (tid < E) {
-        const int pre = s_agg[tid];
+        const int pre = s_pre[tid];
         for (int w = 0; w < kWarps; ++w) s_wh[w][tid] += pre;
     }
     __syncthreads();

@@ -24,7 +24,7 @@ constexpr int kWarp = 32;
 constexpr unsigned kFull = 0xffffffffu;
 
 // Reroute tiling: pairs per tile and threads per tile.
-constexpr int kRerouteTile = 2048;
+constexpr int kRerouteTile = 4096;
 constexpr int kRerouteThreads = 256;
 constexpr int kRerouteWarps = kRerouteThreads / kWarp;
 
@@ -78,8 +78,7 @@ cudaError_t launch_reroute(const Sizes& z, const int32_t* idx,
 // a call only enqueues work (nothing else touches the runtime, which keeps
 // the calls safe under stream capture).
 struct PermuteShape {
-    int grid, warps, nst;
-    size_t smem;
+    int grid, threads, cw;  // cw: threads per token (one 16-byte chunk each)
 };
 struct CombineShape {
     int grid, tpt;
