@@ -62,8 +62,8 @@ TRAFFIC = {
         "source_sha": "897786029bfb7b7a"
     },
     "permute": {
-        "bytes_per_launch": 18861456000,
-        "source_sha": "ec9d69b3006e5e8d"
+        "bytes_per_launch": 18877864000,
+        "source_sha": "07222823ab0e9db7"
     },
     "combine": {
         "bytes_per_launch": 21233264000,
