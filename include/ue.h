@@ -96,8 +96,8 @@ typedef struct ue_ctx ue_ctx; /* opaque */
 
 /* Create a context for `cfg` on CUDA device `device` (made current) and
  * allocate its scratch once: the error word and the reroute's look-back
- * status words (ceil(Q/4096)*E 32-bit words plus a tile counter). Nothing
- * is allocated after this call ("Interface / 1. Initialization": buffers
+ * status words (ceil(Q/8192)*E 64-bit words plus a ticket, a counter and an
+ * epoch). Nothing is allocated after this call ("Interface / 1. Initialization": buffers
  * reserved up front, no dynamic allocation at runtime).
  * Returns UE_ERR_INVALID_ARG for a null `out` or a config outside the
  * limits (checked before any CUDA call), UE_ERR_UNSUPPORTED if the device
@@ -162,7 +162,7 @@ ue_status ue_plan(ue_ctx* ctx, const int32_t* load_e, const ue_placement* out,
  * first, then replicas by ascending g): the o-th pair of expert e goes to
  * the copy whose quota range holds o, at row slot_offset[p] + (o - start).
  * dest_row is a permutation of [0, Q). Single pass: a stable counting sort
- * with a decoupled look-back scan over tiles of 4096 pairs; its waits are
+ * with a decoupled look-back scan over tiles of 8192 pairs; its waits are
  * bounded and end with UE_ERR_TIMEOUT. Ids outside [0, E) set
  * UE_ERR_DEVICE_BOUNDS. */
 ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
@@ -198,13 +198,15 @@ ue_status ue_combine(ue_ctx* ctx, const uint16_t* y, const int32_t* dest_row,
  * pool that forbids outside allocations, or code that keeps no context.
  * The look-back scratch is a fixed device array inside libue (2 MiB plus a
  * few words, held on every GPU that loads the library until the process
- * exits): sizes with ceil(R*T*K / 4096) * E > 524288 are rejected with
+ * exits): sizes with ceil(R*T*K / 8192) * E > 262144 are rejected with
  * UE_ERR_UNSUPPORTED before anything is launched. The first call made with
  * a given device current looks up that array's device address
  * (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture. Every call shares the array: it clears the words it uses
- * on `stream` first, and calls that overlap on the GPU (other streams, other
- * threads) race and give wrong results. Calls no cudaMalloc or cudaFree.
+ * stream capture. Every call shares the array and it is never cleared: its
+ * status words carry the call's epoch, so words left by an earlier call read
+ * as unpublished, and each call's last CTA resets the tile ticket. Calls
+ * that overlap on the GPU (other streams, other threads) race and give
+ * wrong results. Calls no cudaMalloc or cudaFree.
  *   cfg, idx, plan, phys_slot, dest_row, stream: as for ue_init + ue_reroute
  *   (cfg is a host pointer, read during the call).
  *   error: device int32[2], zeroed by the caller; a device-side error writes

@@ -50,8 +50,8 @@ def test_noalloc_reroute_matches_context_reroute(name):
 def test_noalloc_refuses_sizes_beyond_its_scratch():
     gh.ensure_built()
     lib = ue.load_library()
-    # 64 x 32768 tokens x 8 = 16.8M pairs: 4096 tiles x 256 experts > 524288 words
-    cfg = ue.make_config(64, 32768, 256, 8, 2, 64)
+    # 64 x 32768 tokens x 16 = 33.5M pairs: 4096 tiles x 256 experts > 262144 words
+    cfg = ue.make_config(64, 32768, 256, 16, 2, 64)
     dummy = torch.zeros(16, dtype=torch.int32, device="cuda")
     pl = ue.placement(dummy, dummy, dummy, dummy, dummy, dummy)
     rc = lib.ue_reroute_noalloc(ctypes.byref(cfg), dummy.data_ptr(), ctypes.byref(pl),

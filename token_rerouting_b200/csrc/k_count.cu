@@ -8,37 +8,69 @@
 // Design (B200): each CTA owns a chunk of one source rank's pairs and counts
 // them in shared memory, one private histogram per warp so that a hot expert
 // contends only within a warp; shared-memory atomics resolve the rest. Each
-// CTA then adds its non-zero bins to global memory with one atomic per bin. The outputs are zeroed on the stream first. Integer atomics
-// are exact, so the result does not depend on their order.
+// CTA then adds its non-zero bins to the outputs (zeroed on the stream
+// first) with one global atomic per bin. Chunks are large (16384 pairs), so
+// few CTAs contend for each bin of load_e. Every thread issues all its loads
+// before it counts. Integer sums are exact, so the result does not depend on
+// the order of the additions.
 #include "ue_internal.cuh"
 
 namespace ue {
 namespace {
 
-constexpr int kCountThreads = 256;
+constexpr int kCountThreads = 512;
 constexpr int kCountWarps = kCountThreads / 32;
-constexpr int kCountChunk = 2048;  // pairs per CTA
+constexpr int kCountChunk = 16384;  // pairs per CTA (few CTAs add into each bin)
 
+template <bool VEC>
 __global__ void __launch_bounds__(kCountThreads)
 count_kernel(const int32_t* __restrict__ idx, int64_t TK, int E, int chunks_per_rank,
              int32_t* __restrict__ load_re, int32_t* __restrict__ load_e, int* err)
 {
-    __shared__ int hist[kCountWarps][kMaxE];  // one private histogram per warp
+    __shared__ int hist[kCountWarps][kMaxE];  // one private histogram per warp (16 KB)
     const int r = blockIdx.x / chunks_per_rank;
     const int c = blockIdx.x - r * chunks_per_rank;
     const int64_t beg = (int64_t)r * TK + (int64_t)c * kCountChunk;
-    const int64_t end = min((int64_t)(r + 1) * TK, beg + kCountChunk);
+    const int n = (int)min((int64_t)kCountChunk, (int64_t)(r + 1) * TK - beg);
     const int warp = threadIdx.x >> 5;
     for (int x = threadIdx.x; x < kCountWarps * kMaxE; x += blockDim.x) (&hist[0][0])[x] = 0;
     __syncthreads();
-    for (int64_t i = beg + threadIdx.x; i < end; i += blockDim.x) {
-        const int e = __ldg(idx + i);
+    const int32_t* src = idx + beg;
+    // issue all of this thread's loads before using any of them
+    constexpr int kPer = kCountChunk / kCountThreads;
+    int v[kPer];
+    if (VEC) {
+        // beg and n are multiples of 4 here: 16-byte loads
+#pragma unroll
+        for (int q = 0; q < kPer / 4; ++q) {
+            const int x = 4 * (threadIdx.x + q * kCountThreads);
+            int4 w4 = make_int4(-1, -1, -1, -1);
+            if (x < n) w4 = __ldg(reinterpret_cast<const int4*>(src + x));
+            v[4 * q] = w4.x;
+            v[4 * q + 1] = w4.y;
+            v[4 * q + 2] = w4.z;
+            v[4 * q + 3] = w4.w;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int x = threadIdx.x + q * kCountThreads;
+            v[q] = x < n ? __ldg(src + x) : -1;
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int x = VEC ? 4 * (threadIdx.x + (q / 4) * kCountThreads) + (q % 4)
+                          : threadIdx.x + q * kCountThreads;
+        if (x >= n) continue;
+        const int e = v[q];
         if ((unsigned)e < (unsigned)E)
             atomicAdd(&hist[warp][e], 1);
         else
-            raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(i, (int64_t)INT_MAX));
+            raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(beg + x, (int64_t)INT_MAX));
     }
     __syncthreads();
+    // add this CTA's bins to the outputs (zeroed on the stream first)
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int h = 0;
 #pragma unroll
@@ -60,10 +92,14 @@ cudaError_t launch_count(const Sizes& z, const int32_t* idx, int32_t* load_re,
     ce = cudaMemsetAsync(load_e, 0, sizeof(int32_t) * (size_t)z.E, st);
     if (ce != cudaSuccess) return ce;
     const int64_t TK = (int64_t)z.T * z.K;
-    if (TK == 0) return cudaSuccess;
-    const int chunks = (int)((TK + kCountChunk - 1) / kCountChunk);
-    count_kernel<<<z.R * chunks, kCountThreads, 0, st>>>(idx, TK, z.E, chunks, load_re, load_e,
-                                                         err);
+    const int chunks = (int)std::max<int64_t>(1, (TK + kCountChunk - 1) / kCountChunk);
+    const bool vec = (TK % 4 == 0) && ((uintptr_t)idx % 16 == 0);
+    if (vec)
+        count_kernel<true><<<z.R * chunks, kCountThreads, 0, st>>>(idx, TK, z.E, chunks,
+                                                                   load_re, load_e, err);
+    else
+        count_kernel<false><<<z.R * chunks, kCountThreads, 0, st>>>(idx, TK, z.E, chunks,
+                                                                    load_re, load_e, err);
     return cudaGetLastError();
 }
 

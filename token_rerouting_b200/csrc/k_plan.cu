@@ -14,26 +14,30 @@
 // (exact, ties to the lowest e), r* = argmin load_r over ranks with a free
 // slot (ties to the lowest r); the copy goes into r*'s lowest free slot.
 //
-// Design (B200): the greedy is serial (at most G iterations), so its speed is
-// the latency of one iteration, and one warp runs it entirely in registers.
-// Lane l owns experts l, l+32, ... (load, copies, selection key) and ranks
-// l, l+32, ... together with those ranks' redundant slots (expert held,
-// quota). Every load change then lands in the lane that owns the rank, so an
-// iteration needs no shared memory and no atomics:
-//  - Expert side: L/c is compared through the integer key floor(L*2^24/c),
-//    one 64-bit multiply-high with a table of ceil(2^64/c). For c <= 257 and
-//    L < 2^30 this map is exact and order preserving (two different ratios
-//    differ by more than 1/66049, i.e. by more than 250 after scaling, and
-//    equal ratios give equal keys). The expert id is packed below the key, so
-//    the argmax with ties to the lowest e is two warp `redux` max reductions.
-//  - Rank side: the stop test (max load) and the least-loaded rank with a
-//    free slot are `redux` reductions, issued together with the expert one.
-//  - Update: the replicas of e* are found by ballots over the slot registers
-//    in ascending slot order; each replica's new quota changes its owner
-//    lane's rank load locally. The master's quota goes from ceil(L/(c-1)) to
-//    ceil(L/c); every lane knows that change and the master's owner applies
-//    it.
-// The other warps write the outputs and scan the slot offsets at the end.
+// Design (B200): the greedy is serial, so its speed is the latency of one
+// iteration. The choice of e* depends only on the copy counts, never on the
+// ranks: the sequence of experts the greedy picks is fixed by the loads
+// alone (a highest-ratio apportionment). So two warps of one CTA run it as a
+// pipeline:
+//  - warp 1 (expert side) produces the picks in order: e*, its new copy
+//    count and the quota parameters of that step, pushed into a shared-memory
+//    queue with a ready flag per entry. L/c is compared through the integer
+//    key floor(L*2^24/c), one 64-bit multiply-high with a table of
+//    ceil(2^64/c); for c <= 257 and L < 2^30 the map is exact and order
+//    preserving (two different ratios differ by more than 1/66049, i.e. by
+//    more than 250 after scaling; equal ratios give equal keys). The expert id
+//    sits below the key, so the argmax with ties to the lowest e is two warp
+//    `redux` max reductions.
+//  - warp 0 (rank side) keeps the rank loads and the redundant slots in
+//    registers (lane l owns ranks l, l+32, ... and their slots, so every
+//    load change lands in the lane that owns the rank). Per iteration: the
+//    stop test and the least loaded rank with a free slot (three `redux`
+//    reductions), the placement, and the new quotas of e*'s copies: its
+//    replicas are found by ballots in ascending slot order; the master's
+//    quota goes from ceil(L/(c-1)) to ceil(L/c).
+// Warp 1 needs far fewer instructions per step, so warp 0 rarely waits; its
+// wait on a queue entry is bounded. The rest of the CTA writes the outputs
+// and scans the slot offsets at the end.
 #include "ue_internal.cuh"
 
 namespace ue {
@@ -42,6 +46,7 @@ namespace {
 constexpr int kPlanThreads = 256;
 constexpr int kPlanWarps = kPlanThreads / 32;
 constexpr int kKeyShift = 24;
+constexpr long long kPickWaitLimit = 1LL << 24;
 
 __device__ __forceinline__ unsigned div_by(unsigned x, unsigned c, const unsigned long long* recip)
 {
@@ -59,7 +64,14 @@ __device__ __forceinline__ unsigned long long packed_key(unsigned L, unsigned c,
     return (k << 9) | (unsigned long long)(511 - e);
 }
 
-template <int NJ, int SM>
+struct Pick {
+    int e;         // expert receiving the copy
+    unsigned qb;   // floor(L / c) with the new copy count c
+    unsigned rem;  // L mod c
+    unsigned dq0;  // master quota change: ceil(L/c) - ceil(L/(c-1)) (two's complement)
+};
+
+template <int NJE, int NJR, int SM>
 __global__ void __launch_bounds__(kPlanThreads)
 plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placement out, int* err)
 {
@@ -69,6 +81,10 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
     __shared__ int sRank[kMaxR];    // rank loads (initial, then final)
     __shared__ int sSlotE[kMaxG];   // expert of redundant slot g, -1 empty (final)
     __shared__ int sSlotQ[kMaxG];   // quota of redundant slot g (final)
+    __shared__ Pick sPick[kMaxG];   // the expert side's picks, in order
+    __shared__ volatile int sReady[kMaxG];
+    __shared__ volatile int sDone;  // the rank side has stopped
+    __shared__ int sUsedPicks;
     __shared__ unsigned long long sQ;
     __shared__ int sStats[4];
     __shared__ int sWarpSum[kPlanWarps];
@@ -78,8 +94,13 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
     const int P = R * (M + S);
     const int tid = threadIdx.x;
 
-    if (tid == 0) sQ = 0ull;
+    if (tid == 0) {
+        sQ = 0ull;
+        sUsedPicks = 0;
+        sDone = 0;
+    }
     for (int r = tid; r < R; r += blockDim.x) sRank[r] = 0;
+    for (int g = tid; g < G; g += blockDim.x) sReady[g] = 0;
     for (int c = tid + 2; c <= G + 1; c += blockDim.x)
         sRecip[c] = (0xffffffffffffffffull / (unsigned long long)c) + 1ull;
     __syncthreads();
@@ -97,21 +118,65 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
     if (part) atomicAdd(&sQ, part);
     __syncthreads();
 
-    if (tid < 32) {
-        const int lane = tid;
-        const long long Q = (long long)sQ;
-        const long long stop_rhs = 51LL * Q;
-        unsigned Lr[NJ], cr[NJ];
-        unsigned long long key[NJ];
-        unsigned load[NJ];
-        int used[NJ];
-        int slotE[NJ][SM], slotQ[NJ][SM];
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    if (warp == 1) {
+        // ---- expert side: the greedy's picks, independent of the ranks ----
+        unsigned Lr[NJE], cr[NJE];
+        unsigned long long key[NJE];
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) {
+        for (int j = 0; j < NJE; ++j) {
             const int e = lane + 32 * j;
             Lr[j] = e < E ? (unsigned)sL[e] : 0u;
             cr[j] = 1u;
             key[j] = e < E ? packed_key(Lr[j], 1u, e, sRecip) : 0ull;
+        }
+        for (int t = 0; t < G; ++t) {
+            if (__any_sync(kFull, sDone != 0)) break;
+            unsigned long long best = 0ull;
+#pragma unroll
+            for (int j = 0; j < NJE; ++j) best = key[j] > best ? key[j] : best;
+            const unsigned hi = __reduce_max_sync(kFull, (unsigned)(best >> 32));
+            const unsigned lo = __reduce_max_sync(kFull, (unsigned)(best >> 32) == hi ? (unsigned)best : 0u);
+            const int estar = 511 - (int)(lo & 511u);
+            const int ej = estar >> 5;
+            unsigned Le = 0u, ce = 0u;
+#pragma unroll
+            for (int j = 0; j < NJE; ++j)
+                if (j == ej) {
+                    Le = Lr[j];
+                    ce = cr[j];
+                }
+            Le = __shfl_sync(kFull, Le, estar & 31);
+            ce = __shfl_sync(kFull, ce, estar & 31) + 1u;
+            const unsigned long long nk = packed_key(Le, ce, estar, sRecip);
+            if (lane == (estar & 31)) {
+#pragma unroll
+                for (int j = 0; j < NJE; ++j)
+                    if (j == ej) {
+                        cr[j] = ce;
+                        key[j] = nk;
+                    }
+            }
+            if (lane == 0) {
+                const unsigned qb = div_by(Le, ce, sRecip);
+                const unsigned rem = Le - qb * ce;
+                const unsigned q0_new = qb + (rem > 0u ? 1u : 0u);
+                const unsigned q0_old = div_by(Le + ce - 2u, ce - 1u, sRecip);
+                sPick[t] = Pick{estar, qb, rem, q0_new - q0_old};
+                __threadfence_block();
+                sReady[t] = 1;
+            }
+        }
+    } else if (warp == 0) {
+        // ---- rank side: stop test, least loaded free rank, bookkeeping ----
+        const long long Q = (long long)sQ;
+        const long long stop_rhs = 51LL * Q;
+        unsigned load[NJR];
+        int used[NJR];
+        int slotE[NJR][SM], slotQ[NJR][SM];
+#pragma unroll
+        for (int j = 0; j < NJR; ++j) {
             const int r = lane + 32 * j;
             load[j] = r < R ? (unsigned)sRank[r] : 0u;
             used[j] = r < R ? 0 : S;  // ranks beyond R never offer a slot
@@ -125,35 +190,40 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
         unsigned max_before = 0u;
         for (;;) {
             unsigned maxl = 0u, bestl = 0xffffffffu, bestr = 0xffffffffu;
-            unsigned long long best = 0ull;
 #pragma unroll
-            for (int j = 0; j < NJ; ++j) {
+            for (int j = 0; j < NJR; ++j) {
                 maxl = max(maxl, load[j]);
                 if (used[j] < S && load[j] < bestl) {
                     bestl = load[j];
                     bestr = (unsigned)(lane + 32 * j);
                 }
-                best = key[j] > best ? key[j] : best;
             }
             maxl = __reduce_max_sync(kFull, maxl);
             const unsigned ml = __reduce_min_sync(kFull, bestl);
-            const unsigned hi = __reduce_max_sync(kFull, (unsigned)(best >> 32));
             if (iters == 0) max_before = maxl;
             if (50LL * R * (long long)maxl <= stop_rhs) break;
             if (ml == 0xffffffffu) break;  // no free slot anywhere
             const int rstar = (int)__reduce_min_sync(kFull, bestl == ml ? bestr : 0xffffffffu);
-            const unsigned lo = __reduce_max_sync(kFull, (unsigned)(best >> 32) == hi ? (unsigned)best : 0u);
-            const int estar = 511 - (int)(lo & 511u);
+
+            // this iteration's expert, from the expert side's queue
+            int ready = sReady[iters];
+            for (long long spin = 0; !ready && spin < kPickWaitLimit; ++spin) ready = sReady[iters];
+            ready = __all_sync(kFull, ready);
+            if (!ready) {
+                if (lane == 0) raise_error(err, UE_ERR_TIMEOUT, iters);
+                break;
+            }
+            __threadfence_block();
+            const Pick pk = sPick[iters];
+            const int estar = pk.e;
             const int rj = rstar >> 5;
             const bool rown = lane == (rstar & 31);
-            const int ej = estar >> 5;
-            const bool eown = lane == (estar & 31);
 
             // r*'s lowest free slot; does r* already hold a copy of e*?
             int s_new = 0;
             bool held = false;
 #pragma unroll
-            for (int j = 0; j < NJ; ++j)
+            for (int j = 0; j < NJR; ++j)
                 if (j == rj) {
                     s_new = used[j];
 #pragma unroll
@@ -163,7 +233,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
             if (estar / M == rstar || __any_sync(kFull, held)) colocated += 1;
             if (rown) {
 #pragma unroll
-                for (int j = 0; j < NJ; ++j)
+                for (int j = 0; j < NJR; ++j)
                     if (j == rj) {
                         used[j] += 1;
 #pragma unroll
@@ -171,57 +241,32 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
                             if (s == s_new) slotE[j][s] = estar;
                     }
             }
-
-            // e* gains a copy: new key and quotas
-            unsigned Le = 0u, ce = 0u;
-#pragma unroll
-            for (int j = 0; j < NJ; ++j)
-                if (j == ej) {
-                    Le = Lr[j];
-                    ce = cr[j];
-                }
-            Le = __shfl_sync(kFull, Le, estar & 31);
-            ce = __shfl_sync(kFull, ce, estar & 31) + 1u;
-            const unsigned long long nk = packed_key(Le, ce, estar, sRecip);
-            if (eown) {
-#pragma unroll
-                for (int j = 0; j < NJ; ++j)
-                    if (j == ej) {
-                        cr[j] = ce;
-                        key[j] = nk;
-                    }
-            }
-            const unsigned qb = div_by(Le, ce, sRecip);
-            const unsigned rem = Le - qb * ce;
-            // master: ceil(L/(c-1)) -> ceil(L/c), applied by the master rank's owner
+            // master quota change, on the master rank's owner
             const int rm = estar / M;
-            const unsigned q0_new = qb + (rem > 0u ? 1u : 0u);
-            const unsigned q0_old = div_by(Le + ce - 2u, ce - 1u, sRecip);
             if (lane == (rm & 31)) {
 #pragma unroll
-                for (int j = 0; j < NJ; ++j)
-                    if (j == (rm >> 5)) load[j] = load[j] + q0_new - q0_old;
+                for (int j = 0; j < NJR; ++j)
+                    if (j == (rm >> 5)) load[j] += pk.dq0;
             }
             // replicas, ascending slot g = r*S + s (r = lane + 32 j)
             unsigned before = 0u;
             const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-            for (int j = 0; j < NJ; ++j) {
+            for (int j = 0; j < NJR; ++j) {
                 unsigned lower = 0u;   // e* replicas in lower lanes of group j
                 unsigned total = 0u;   // e* replicas in group j
-                unsigned msk[SM];
 #pragma unroll
                 for (int s = 0; s < SM; ++s) {
-                    msk[s] = __ballot_sync(kFull, s < S && slotE[j][s] == estar);
-                    lower += __popc(msk[s] & lt);
-                    total += __popc(msk[s]);
+                    const unsigned msk = __ballot_sync(kFull, s < S && slotE[j][s] == estar);
+                    lower += __popc(msk & lt);
+                    total += __popc(msk);
                 }
                 unsigned mine = 0u;  // e* replicas in this lane's lower slots
 #pragma unroll
                 for (int s = 0; s < SM; ++s) {
                     if (s < S && slotE[j][s] == estar) {
                         const unsigned pos = 1u + before + lower + mine;
-                        const int qn = (int)(qb + (pos < rem ? 1u : 0u));
+                        const int qn = (int)(pk.qb + (pos < pk.rem ? 1u : 0u));
                         load[j] = load[j] + (unsigned)(qn - slotQ[j][s]);
                         slotQ[j][s] = qn;
                         mine += 1u;
@@ -233,19 +278,18 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
         }
         unsigned mx = 0u;
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-            const int idx = lane + 32 * j;
-            if (idx < R) {
+        for (int j = 0; j < NJR; ++j) {
+            const int r = lane + 32 * j;
+            if (r < R) {
                 mx = max(mx, load[j]);
-                sRank[idx] = (int)load[j];
+                sRank[r] = (int)load[j];
 #pragma unroll
                 for (int s = 0; s < SM; ++s)
                     if (s < S) {
-                        sSlotE[idx * S + s] = slotE[j][s];
-                        sSlotQ[idx * S + s] = slotQ[j][s];
+                        sSlotE[r * S + s] = slotE[j][s];
+                        sSlotQ[r * S + s] = slotQ[j][s];
                     }
             }
-            if (idx < E) sC[idx] = (int)cr[j];
         }
         mx = __reduce_max_sync(kFull, mx);
         if (lane == 0) {
@@ -253,8 +297,17 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
             sStats[1] = (int)max_before;
             sStats[2] = (int)mx;
             sStats[3] = colocated;
+            sUsedPicks = iters;
+            sDone = 1;
         }
     }
+    __syncthreads();
+
+    // copies per expert: 1 + its picks among the first `iters` of the queue
+    const int iters = sUsedPicks;
+    for (int e = tid; e < E; e += blockDim.x) sC[e] = 1;
+    __syncthreads();
+    for (int t = tid; t < iters; t += blockDim.x) atomicAdd(&sC[sPick[t].e], 1);
     __syncthreads();
 
     for (int e = tid; e < E; e += blockDim.x) out.n_copies[e] = sC[e];
@@ -284,7 +337,6 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
         }
         q2[h] = q;
     }
-    const int lane = tid & 31, warp = tid >> 5;
     const int mine = q2[0] + q2[1];
     int incl = mine;
 #pragma unroll
@@ -302,19 +354,24 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
     if (tid == 0) out.slot_offset[P] = (int)sQ;
 }
 
-template <int NJ>
-cudaError_t launch_nj(const Sizes& z, const int32_t* load_e, const ue_placement& out, int* err,
-                      cudaStream_t st)
+template <int NJE, int NJR>
+cudaError_t launch_s(const Sizes& z, const int32_t* load_e, const ue_placement& out, int* err,
+                     cudaStream_t st)
 {
-    if (z.S <= 1)
-        plan_kernel<NJ, 1><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, out, err);
-    else if (z.S <= 2)
-        plan_kernel<NJ, 2><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, out, err);
-    else if (z.S <= 4)
-        plan_kernel<NJ, 4><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, out, err);
+    if (z.S <= 2)
+        plan_kernel<NJE, NJR, 2><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, out, err);
     else
-        plan_kernel<NJ, 8><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, out, err);
+        plan_kernel<NJE, NJR, 8><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, out, err);
     return cudaGetLastError();
+}
+
+template <int NJE>
+cudaError_t launch_r(const Sizes& z, const int32_t* load_e, const ue_placement& out, int* err,
+                     cudaStream_t st)
+{
+    if (z.R <= 32) return launch_s<NJE, 1>(z, load_e, out, err, st);
+    if (z.R <= 64) return launch_s<NJE, 2>(z, load_e, out, err, st);
+    return launch_s<NJE, 4>(z, load_e, out, err, st);
 }
 
 }  // namespace
@@ -322,11 +379,10 @@ cudaError_t launch_nj(const Sizes& z, const int32_t* load_e, const ue_placement&
 cudaError_t launch_plan(const Sizes& z, const int32_t* load_e,
                         const ue_placement& out, int* err, cudaStream_t st)
 {
-    const int need = std::max(z.E, z.R);
-    if (need <= 32) return launch_nj<1>(z, load_e, out, err, st);
-    if (need <= 64) return launch_nj<2>(z, load_e, out, err, st);
-    if (need <= 128) return launch_nj<4>(z, load_e, out, err, st);
-    return launch_nj<8>(z, load_e, out, err, st);
+    if (z.E <= 32) return launch_r<1>(z, load_e, out, err, st);
+    if (z.E <= 64) return launch_r<2>(z, load_e, out, err, st);
+    if (z.E <= 128) return launch_r<4>(z, load_e, out, err, st);
+    return launch_r<8>(z, load_e, out, err, st);
 }
 
 }  // namespace ue

@@ -10,19 +10,25 @@
 // j and the offset follow from o by one division.
 //
 // Design (B200): a single-pass stable counting sort with a decoupled
-// look-back. Each CTA takes a tile of 4096 pairs by an atomic ticket (so every
+// look-back. Each CTA takes a tile of 8192 pairs by an atomic ticket (so every
 // tile it waits on is already running), stages the ids in shared memory and
 // counts them per warp sub-range, then publishes its per-expert tile counts
 // at once so that successors never wait on its later work. While its
 // predecessors finish, it rebuilds the plan's copy lists (at most 512
-// entries). The look-back runs one thread per expert column and reads a
-// window of 16 predecessors per step with independent loads, adding their
-// counts until it meets an inclusive prefix; with every tile resident at
-// once this cuts the serial chain of L2 round trips by the window width.
+// entries). The look-back runs H = min(4, 512/E) threads per expert column;
+// each reads 16 predecessors per step with independent loads, so one step
+// covers 16*H tiles, and the column adds their counts up to the nearest
+// inclusive prefix. With every tile resident at once this cuts the serial
+// chain of L2 round trips by the window width.
 // Every wait is bounded: when it runs out the tile publishes an error flag,
 // records UE_ERR_TIMEOUT and writes nothing. Finally each warp re-walks its
-// 512 pairs in order, ranking equal ids within 32 lanes by popcount of the
-// lanes that match, and writes the physical slot and dispatch row.
+// 512 pairs in order, ranking equal ids within 32 lanes (the lanes holding
+// the same id come from nine ballots over the id's bits), and writes the
+// physical slot and dispatch row; the copy index comes from one exact
+// multiply-high by a per-expert reciprocal.
+// The status words carry the launch's tag, so nothing is cleared between
+// launches: words of earlier launches read as "not yet published". The last
+// CTA to finish resets the ticket and the counter and advances the epoch.
 #include "ue_internal.cuh"
 
 namespace ue {
@@ -33,39 +39,97 @@ constexpr int kThreads = kRerouteThreads;
 constexpr int kWarps = kRerouteWarps;
 constexpr int kPerWarp = kTile / kWarps;
 constexpr int kRounds = kPerWarp / 32;
-constexpr int kWindow = 16;  // predecessors read per look-back step
+constexpr int kWindow = 16;  // predecessors read per thread per look-back step
+constexpr int kMaxH = 4;     // threads per expert column in the look-back
 
-__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p)
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p)
 {
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 
-__device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v)
+__device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long long v)
 {
-    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// status word of this launch: tag, flag, count
+__device__ __forceinline__ unsigned long long status_word(uint32_t tag, uint32_t flag, uint32_t v)
+{
+    return ((unsigned long long)tag << 32) | (flag << 30) | (v & kValueMask);
+}
+
+// the lanes of the warp holding the same key (9-bit keys): one ballot per bit
+__device__ __forceinline__ unsigned same_key_lanes(int key)
+{
+    unsigned peers = kFull;
+#pragma unroll
+    for (int b = 0; b < 9; ++b) {
+        const bool bit = (key >> b) & 1;
+        const unsigned m = __ballot_sync(kFull, bit);
+        peers &= bit ? m : ~m;
+    }
+    return peers;
+}
+
+// per-expert data used for every pair of the tile (16-byte aligned records)
+struct alignas(16) ExpA {
+    int pre;   // exclusive prefix of this expert before the tile
+    int L;     // total pairs of the expert (sum of its quotas)
+    int thr;   // rem * (b + 1): pairs held by the copies with quota b + 1
+    int rem;   // copies with quota b + 1
+};
+struct alignas(16) ExpB {
+    unsigned long long m1;  // ceil(2^64 / (b + 1))
+    unsigned long long m0;  // ceil(2^64 / b) (b >= 1), unused when b == 0
+};
+struct alignas(8) ExpC {
+    int b;   // floor(L / c)
+    int cb;  // first entry of the expert in the copy table
+};
+
+// ceil(2^64 / d) for d >= 2; floor(x / d) = umul64hi(x, m) exactly when x*d < 2^64
+__device__ __forceinline__ unsigned long long recip64(unsigned d)
+{
+    return d <= 1u ? 0ull : (0xffffffffffffffffull / d) + 1ull;
+}
+
+__device__ __forceinline__ unsigned div_m(unsigned x, unsigned d, unsigned long long m)
+{
+    return d == 1u ? x : (unsigned)__umul64hi((unsigned long long)x, m);
 }
 
 __global__ void __launch_bounds__(kThreads)
 reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
                ue_placement plan, int32_t* __restrict__ phys_slot,
-               int32_t* __restrict__ dest_row, uint32_t* status,
-               uint32_t* tile_counter, int64_t spin_limit, int drop_first,
+               int32_t* __restrict__ dest_row, unsigned long long* status,
+               uint32_t* sync, int64_t spin_limit, int drop_first,
                int* err)
 {
     __shared__ short s_idx[kTile];        // expert ids of the tile (-1: none)
-    __shared__ int s_wh[kWarps][kMaxE];   // per-warp counts, then start offsets
-    __shared__ int s_pre[kMaxE];          // tile prefix per expert
-    __shared__ int s_cnt[kMaxE], s_lrep[kMaxE], s_run[kMaxE];
-    __shared__ int s_L[kMaxE], s_b[kMaxE], s_rem[kMaxE];
-    __shared__ int s_master[kMaxE], s_repstart[kMaxE];
-    __shared__ int s_rep[kMaxG];          // replica slots, by expert then g
-    __shared__ int s_off[kMaxE + kMaxG + 1];
-    __shared__ int s_se[kMaxG];           // plan: slot_expert
-    __shared__ int s_sq[kMaxE + kMaxG];   // plan: slot_quota
+    __shared__ short s_wh[kWarps][kMaxE]; // per-warp counts, then in-tile offsets
+    __shared__ ExpA s_a[kMaxE];
+    __shared__ ExpB s_bm[kMaxE];
+    __shared__ ExpC s_c[kMaxE];
+    __shared__ int s_cp[kMaxE + kMaxG];   // copy table: physical slot, copies of
+    __shared__ int s_cr[kMaxE + kMaxG];   // each expert in order; first dispatch row
+    __shared__ union {
+        struct {  // building the copy table
+            int cnt[kMaxE], lrep[kMaxE], run[kMaxE];
+            int off[kMaxE + kMaxG + 1];   // plan: slot_offset
+            int se[kMaxG];                // plan: slot_expert
+            int sq[kMaxE + kMaxG];        // plan: slot_quota
+        } pro;
+        struct {  // look-back: one window segment per (h, e)
+            uint32_t part[kMaxH][kMaxE];
+            unsigned char state[kMaxH][kMaxE];
+            unsigned char cdone[kMaxE];  // column finished
+        } lb;
+    } u;
     __shared__ int s_wsum[kWarps];
     __shared__ int s_tile;
+    __shared__ uint32_t s_tag;
     __shared__ int s_fail;
 
     const int M = E / R;
@@ -76,75 +140,89 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     const int warp = tid >> 5;
 
     if (tid == 0) {
-        s_tile = (int)atomicAdd(tile_counter, 1u);
+        s_tile = (int)atomicAdd(&sync[0], 1u);
+        // this launch's tag; the epoch only moves after every CTA has read it
+        const uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(&sync[2]);
+        s_tag = epoch + 1u == 0u ? 1u : epoch + 1u;
         s_fail = 0;
     }
     for (int x = tid; x < kWarps * kMaxE; x += kThreads) (&s_wh[0][0])[x] = 0;
     for (int e = tid; e < E; e += kThreads) {
-        s_cnt[e] = 0;
-        s_lrep[e] = 0;
-        s_run[e] = 0;
+        u.pro.cnt[e] = 0;
+        u.pro.lrep[e] = 0;
+        u.pro.run[e] = 0;
     }
     __syncthreads();
 
     // ---- stage the tile and count it per warp sub-range ----
     const int tile = s_tile;
+    const uint32_t tag = s_tag;
     const int64_t t0 = (int64_t)tile * kTile;
     const int cnt_tile = (int)min((int64_t)kTile, Q - t0);
-    for (int x = tid; x < kTile; x += kThreads) {
-        int e = -1;
-        if (x < cnt_tile) {
-            e = __ldg(idx + t0 + x);
-            if ((unsigned)e >= (unsigned)E) {
+    {
+        // issue all of this thread's loads before using any of them
+        constexpr int kPer = kTile / kThreads;
+        int v[kPer];
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int x = tid + q * kThreads;
+            v[q] = x < cnt_tile ? __ldg(idx + t0 + x) : -1;
+        }
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int x = tid + q * kThreads;
+            int e = v[q];
+            if (x < cnt_tile && (unsigned)e >= (unsigned)E) {
                 raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(t0 + x, (int64_t)INT_MAX));
                 e = -1;
             }
+            s_idx[x] = (short)e;
         }
-        s_idx[x] = (short)e;
     }
     __syncthreads();
 #pragma unroll 4
     for (int rd = 0; rd < kRounds; ++rd) {
         const int e = s_idx[warp * kPerWarp + rd * 32 + lane];
-        if (e >= 0) atomicAdd(&s_wh[warp][e], 1);
+        if (e >= 0) atomicAdd_block(reinterpret_cast<int*>(&s_wh[warp][0]) + (e >> 1),
+                                    (e & 1) ? (1 << 16) : 1);
     }
     __syncthreads();
 
     // ---- publish this tile's counts ----
     int acc = 0;
-    uint32_t* mine = status + (size_t)tile * E + tid;
+    unsigned long long* mine = status + (size_t)tile * E + tid;
     if (tid < E) {
         for (int w = 0; w < kWarps; ++w) {
             const int t = s_wh[w][tid];
-            s_wh[w][tid] = acc;
+            s_wh[w][tid] = (short)acc;
             acc += t;
         }
         if (tile == 0) {
-            if (!drop_first) st_relaxed(mine, (kFlagPrefix << 30) | (uint32_t)acc);
+            if (!drop_first) st_relaxed(mine, status_word(tag, kFlagPrefix, (uint32_t)acc));
         } else {
-            st_relaxed(mine, (kFlagAggregate << 30) | (uint32_t)acc);
+            st_relaxed(mine, status_word(tag, kFlagAggregate, (uint32_t)acc));
         }
     }
 
-    // ---- copy lists of every expert, from the plan (overlaps the wait) ----
-    for (int p = tid; p <= P; p += kThreads) s_off[p] = __ldg(plan.slot_offset + p);
-    for (int p = tid; p < P; p += kThreads) s_sq[p] = __ldg(plan.slot_quota + p);
-    for (int g = tid; g < G; g += kThreads) s_se[g] = __ldg(plan.slot_expert + g);
+    // ---- copy table of every expert, from the plan (overlaps the wait) ----
+    for (int p = tid; p <= P; p += kThreads) u.pro.off[p] = __ldg(plan.slot_offset + p);
+    for (int p = tid; p < P; p += kThreads) u.pro.sq[p] = __ldg(plan.slot_quota + p);
+    for (int g = tid; g < G; g += kThreads) u.pro.se[g] = __ldg(plan.slot_expert + g);
     __syncthreads();
     for (int g = tid; g < G; g += kThreads) {
-        const int e = s_se[g];
+        const int e = u.pro.se[g];
         if (e >= 0 && e < E) {
             const int p = (g / S) * (M + S) + M + (g % S);
-            atomicAdd(&s_cnt[e], 1);
-            atomicAdd(&s_lrep[e], s_sq[p]);
+            atomicAdd(&u.pro.cnt[e], 1);
+            atomicAdd(&u.pro.lrep[e], u.pro.sq[p]);
         } else if (e >= E) {
             raise_error(err, UE_ERR_DEVICE_BOUNDS, g);
         }
     }
     __syncthreads();
     {
-        // exclusive scan of replica counts over experts (E <= kThreads)
-        const int c = tid < E ? s_cnt[tid] : 0;
+        // exclusive scan of copies per expert (1 + replicas) over experts
+        const int c = tid < E ? 1 + u.pro.cnt[tid] : 0;
         int incl = c;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -158,126 +236,175 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         if (tid < E) {
             const int e = tid;
             const int mp = (e / M) * (M + S) + (e % M);
-            const int copies = 1 + c;
-            const int L = s_sq[mp] + s_lrep[e];
-            const int b = L / copies;
-            s_L[e] = L;
-            s_b[e] = b;
-            s_rem[e] = L - b * copies;
-            s_master[e] = mp;
-            s_repstart[e] = wofs + incl - c;
+            const int L = u.pro.sq[mp] + u.pro.lrep[e];
+            const unsigned b = (unsigned)L / (unsigned)c;
+            const int rem = L - (int)b * c;
+            const int cb = wofs + incl - c;
+            s_a[e] = ExpA{0, L, rem * (int)(b + 1u), rem};
+            s_bm[e] = ExpB{recip64(b + 1u), recip64(b)};
+            s_c[e] = ExpC{(int)b, cb};
+            s_cp[cb] = mp;                 // copy 0: the master
+            s_cr[cb] = u.pro.off[mp];
+            u.pro.run[e] = cb + 1;         // next replica entry
         }
         __syncthreads();
     }
     if (warp == 0) {
-        // replica slots in ascending g within each expert
+        // replicas in ascending g after each expert's master
         for (int g0 = 0; g0 < G; g0 += 32) {
             const int g = g0 + lane;
             int e = -1;
             if (g < G) {
-                e = s_se[g];
+                e = u.pro.se[g];
                 if (e >= E) e = -1;
             }
             const unsigned peers = __match_any_sync(kFull, e);
             if (e >= 0) {
-                const int pos = s_run[e] + __popc(peers & ((1u << lane) - 1u));
-                s_rep[s_repstart[e] + pos] = (g / S) * (M + S) + M + (g % S);
+                const int ci = u.pro.run[e] + __popc(peers & ((1u << lane) - 1u));
+                const int p = (g / S) * (M + S) + M + (g % S);
+                s_cp[ci] = p;
+                s_cr[ci] = u.pro.off[p];
             }
             __syncwarp();
-            if (e >= 0 && lane == __ffs(peers) - 1) s_run[e] += __popc(peers);
+            if (e >= 0 && lane == __ffs(peers) - 1) u.pro.run[e] += __popc(peers);
             __syncwarp();
         }
     }
+    __syncthreads();  // the union switches from the copy table to look-back
 
     // ---- look back over predecessor tiles, publish the inclusive prefix ----
-    if (tid < E) {
-        if (tile == 0) {
-            s_pre[tid] = 0;
-        } else {
-            uint32_t excl = 0;
-            int base = tile - 1;  // nearest predecessor not yet added
-            int64_t polls = 0;
-            bool fail = false, done = false;
-            while (!done && !fail) {
-                uint32_t v[kWindow];
+    // H threads per expert column; thread (h, e) reads predecessors
+    // base - h*W .. base - h*W - (W-1) of each step, so one step covers H*W
+    // tiles with independent loads.
+    const int H = min(kMaxH, kThreads / E);
+    const int h = tid / E;
+    const int e = tid - h * E;
+    const bool lb = h < H;
+    uint32_t excl = 0;
+    if (lb && h == 0) u.lb.cdone[e] = (tile == 0) ? 1 : 0;
+    __syncthreads();
+    bool done = lb ? (u.lb.cdone[e] != 0) : true;
+    int base = tile - 1;  // nearest predecessor not yet added
+    int64_t polls = 0;
+    while (__syncthreads_or(!done)) {
+        if (!done) {
+            uint32_t sum = 0;
+            unsigned char st = 0;  // 0: no prefix in my segment, 1: prefix, 2: error
+            unsigned long long v[kWindow];
 #pragma unroll
-                for (int i = 0; i < kWindow; ++i)
-                    v[i] = (base - i >= 0) ? ld_relaxed(status + (size_t)(base - i) * E + tid)
-                                           : (kFlagPrefix << 30);
+            for (int i = 0; i < kWindow; ++i) {
+                const int pred = base - h * kWindow - i;
+                v[i] = pred >= 0 ? ld_relaxed(status + (size_t)pred * E + e)
+                                 : status_word(tag, kFlagPrefix, 0u);
+            }
 #pragma unroll
-                for (int i = 0; i < kWindow; ++i) {
-                    if (!done && !fail) {
-                        uint32_t sw = v[i];
-                        while ((sw >> 30) == kFlagInvalid && !fail) {
-                            if (++polls > spin_limit) {
-                                raise_error(err, UE_ERR_TIMEOUT, tile);
-                                fail = true;
-                            } else {
-                                __nanosleep(64);
-                                sw = ld_relaxed(status + (size_t)(base - i) * E + tid);
-                            }
+            for (int i = 0; i < kWindow; ++i) {
+                if (st == 0) {
+                    const int pred = base - h * kWindow - i;
+                    unsigned long long sw = v[i];
+                    // not yet published in this launch (older tag or none)
+                    while (((uint32_t)(sw >> 32) != tag ||
+                            (((uint32_t)sw >> 30) == kFlagInvalid)) && st == 0) {
+                        if (++polls > spin_limit) {
+                            raise_error(err, UE_ERR_TIMEOUT, tile);
+                            st = 2;
+                        } else {
+                            __nanosleep(64);
+                            sw = ld_relaxed(status + (size_t)pred * E + e);
                         }
-                        if ((sw >> 30) == kFlagError) fail = true;
-                        if (!fail) {
-                            if (base - i >= 0) excl += sw & kValueMask;
-                            if ((sw >> 30) == kFlagPrefix) done = true;
+                    }
+                    if (st == 0) {
+                        const uint32_t flag = (uint32_t)sw >> 30;
+                        if (flag == kFlagError) {
+                            st = 2;
+                        } else {
+                            if (pred >= 0) sum += (uint32_t)sw & kValueMask;
+                            if (flag == kFlagPrefix) st = 1;
                         }
                     }
                 }
-                base -= kWindow;
             }
-            if (fail) {
-                st_relaxed(mine, kFlagError << 30);
-                atomicOr(&s_fail, 1);
-            } else {
-                st_relaxed(mine, (kFlagPrefix << 30) | ((excl + (uint32_t)acc) & kValueMask));
-                s_pre[tid] = (int)excl;
-            }
+            u.lb.part[h][e] = sum;
+            u.lb.state[h][e] = st;
         }
+        __syncthreads();
+        if (!done && h == 0) {
+            // add the segments in order up to the first one holding a prefix
+            bool stop = false;
+            for (int hh = 0; hh < H && !stop; ++hh) {
+                const unsigned char st = u.lb.state[hh][e];
+                if (st == 2) {
+                    atomicOr(&s_fail, 1);
+                    stop = true;
+                } else {
+                    excl += u.lb.part[hh][e];
+                    if (st == 1) stop = true;
+                }
+            }
+            u.lb.cdone[e] = stop ? 1 : 0;
+        }
+        __syncthreads();
+        if (!done) done = u.lb.cdone[e] != 0;
+        base -= H * kWindow;
     }
-    __syncthreads();
-    if (s_fail) return;
-    if (tid < E) {
-        const int pre = s_pre[tid];
-        for (int w = 0; w < kWarps; ++w) s_wh[w][tid] += pre;
+    if (tid < E && tile > 0) {
+        if (s_fail)
+            st_relaxed(mine, status_word(tag, kFlagError, 0u));
+        else
+            st_relaxed(mine, status_word(tag, kFlagPrefix, excl + (uint32_t)acc));
     }
+    if (tid < E) s_a[tid].pre = (int)excl;
     __syncthreads();
+    const bool write_out = !s_fail;
 
     // ---- in-order ranks, copy, dispatch row ----
-#pragma unroll 1
-    for (int rd = 0; rd < kRounds; ++rd) {
+    // the o-th pair of expert e: copy j = o / (b+1) while o < rem*(b+1), else
+    // rem + (o - rem*(b+1)) / b; row = first row of that copy + (o - start_j)
+#pragma unroll 2
+    for (int rd = 0; rd < (write_out ? kRounds : 0); ++rd) {
         const int x = warp * kPerWarp + rd * 32 + lane;
-        const int e = s_idx[x];
-        const unsigned peers = __match_any_sync(kFull, e);
-        int o = 0;
-        if (e >= 0) o = s_wh[warp][e] + __popc(peers & ((1u << lane) - 1u));
+        const int ex = s_idx[x];
+        const unsigned peers = same_key_lanes(ex & 511);
+        int p = -1, row = -1;
+        if (ex >= 0) {
+            const ExpA a = s_a[ex];
+            const int o = a.pre + s_wh[warp][ex] + __popc(peers & ((1u << lane) - 1u));
+            if (o < a.L) {
+                const ExpB bm = s_bm[ex];
+                const ExpC c = s_c[ex];
+                const bool big = o < a.thr;
+                const unsigned d = big ? (unsigned)c.b + 1u : (unsigned)c.b;
+                const unsigned x0 = big ? (unsigned)o : (unsigned)(o - a.thr);
+                const unsigned q = div_m(x0, d, big ? bm.m1 : bm.m0);
+                const int j = big ? (int)q : a.rem + (int)q;
+                const int start = j * c.b + min(j, a.rem);
+                const int ci = c.cb + j;
+                p = s_cp[ci];
+                row = s_cr[ci] + (o - start);
+            } else {
+                // the plan does not cover this pair (plan from other ids)
+                raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(t0 + x, (int64_t)INT_MAX));
+            }
+        }
         __syncwarp();
-        if (e >= 0 && lane == __ffs(peers) - 1) s_wh[warp][e] += __popc(peers);
+        if (ex >= 0 && lane == __ffs(peers) - 1) s_wh[warp][ex] += (short)__popc(peers);
         __syncwarp();
         if (x < cnt_tile) {
-            int p = -1, row = -1;
-            if (e >= 0) {
-                if (o < s_L[e]) {
-                    const int b = s_b[e], rem = s_rem[e];
-                    const int thr = rem * (b + 1);
-                    int j, off;
-                    if (o < thr) {
-                        j = o / (b + 1);
-                        off = o - j * (b + 1);
-                    } else {
-                        const int o2 = o - thr;
-                        j = rem + o2 / b;
-                        off = o2 - (j - rem) * b;
-                    }
-                    p = (j == 0) ? s_master[e] : s_rep[s_repstart[e] + j - 1];
-                    row = s_off[p] + off;
-                } else {
-                    // the plan does not cover this pair (plan from other ids)
-                    raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(t0 + x, (int64_t)INT_MAX));
-                }
-            }
             phys_slot[t0 + x] = p;
             dest_row[t0 + x] = row;
+        }
+    }
+
+    // the last CTA to finish leaves the ticket, the counter and the epoch
+    // ready for the next launch
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        if (atomicAdd(&sync[1], 1u) == gridDim.x - 1) {
+            sync[0] = 0u;
+            sync[1] = 0u;
+            __threadfence();
+            atomicExch(&sync[2], tag);
         }
     }
 }
@@ -286,18 +413,14 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
 
 cudaError_t launch_reroute(const Sizes& z, const int32_t* idx,
                            const ue_placement& plan, int32_t* phys_slot,
-                           int32_t* dest_row, uint32_t* status,
-                           uint32_t* tile_counter, int64_t spin_limit,
+                           int32_t* dest_row, unsigned long long* status,
+                           uint32_t* sync, int64_t spin_limit,
                            int drop_first, int* err, cudaStream_t st)
 {
     if (z.Q == 0) return cudaSuccess;
     const int64_t tiles = (z.Q + kTile - 1) / kTile;
-    cudaError_t ce = cudaMemsetAsync(status, 0, sizeof(uint32_t) * (size_t)tiles * z.E, st);
-    if (ce != cudaSuccess) return ce;
-    ce = cudaMemsetAsync(tile_counter, 0, sizeof(uint32_t), st);
-    if (ce != cudaSuccess) return ce;
     reroute_kernel<<<(unsigned)tiles, kThreads, 0, st>>>(
-        idx, z.Q, z.R, z.E, z.S, plan, phys_slot, dest_row, status, tile_counter,
+        idx, z.Q, z.R, z.E, z.S, plan, phys_slot, dest_row, status, sync,
         spin_limit, drop_first, err);
     return cudaGetLastError();
 }

@@ -16,8 +16,8 @@ struct ue_ctx {
     ue::PermuteShape perm;
     ue::CombineShape comb;
     int* d_err;             // [2] error code, detail
-    uint32_t* d_status;     // [tiles][E] reroute look-back words
-    uint32_t* d_counter;    // reroute tile ticket
+    unsigned long long* d_status;  // [tiles][E] reroute look-back words
+    uint32_t* d_sync;       // [4] reroute ticket, finished CTAs, epoch
     int64_t tiles;
     int64_t spin_limit;
     int drop_first;
@@ -103,22 +103,22 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
 
     const size_t status_words = (size_t)std::max<int64_t>(ctx->tiles, 1) * ctx->z.E;
     if (cudaMalloc(&ctx->d_err, 2 * sizeof(int)) != cudaSuccess ||
-        cudaMalloc(&ctx->d_status, status_words * sizeof(uint32_t)) != cudaSuccess ||
-        cudaMalloc(&ctx->d_counter, sizeof(uint32_t)) != cudaSuccess) {
+        cudaMalloc(&ctx->d_status, status_words * sizeof(unsigned long long)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_sync, 4 * sizeof(uint32_t)) != cudaSuccess) {
         cudaFree(ctx->d_err);
         cudaFree(ctx->d_status);
-        cudaFree(ctx->d_counter);
+        cudaFree(ctx->d_sync);
         delete ctx;
         cudaGetLastError();
         return UE_ERR_NOMEM;
     }
     if (cudaMemset(ctx->d_err, 0, 2 * sizeof(int)) != cudaSuccess ||
-        cudaMemset(ctx->d_status, 0, status_words * sizeof(uint32_t)) != cudaSuccess ||
-        cudaMemset(ctx->d_counter, 0, sizeof(uint32_t)) != cudaSuccess ||
+        cudaMemset(ctx->d_status, 0, status_words * sizeof(unsigned long long)) != cudaSuccess ||
+        cudaMemset(ctx->d_sync, 0, 4 * sizeof(uint32_t)) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess) {
         cudaFree(ctx->d_err);
         cudaFree(ctx->d_status);
-        cudaFree(ctx->d_counter);
+        cudaFree(ctx->d_sync);
         delete ctx;
         return UE_ERR_CUDA;
     }
@@ -135,7 +135,7 @@ ue_status ue_destroy(ue_ctx* ctx)
     if (st == UE_OK && cudaDeviceSynchronize() != cudaSuccess) st = UE_ERR_CUDA;
     cudaFree(ctx->d_err);
     cudaFree(ctx->d_status);
-    cudaFree(ctx->d_counter);
+    cudaFree(ctx->d_sync);
     ctx->magic = 0;
     delete ctx;
     return st;
@@ -190,7 +190,7 @@ ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
         return UE_ERR_INVALID_ARG;
     if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
     return from_cuda(ue::launch_reroute(ctx->z, idx, *plan, phys_slot, dest_row, ctx->d_status,
-                                        ctx->d_counter, ctx->spin_limit, ctx->drop_first,
+                                        ctx->d_sync, ctx->spin_limit, ctx->drop_first,
                                         ctx->d_err, as_stream(stream)));
 }
 

@@ -24,11 +24,13 @@ constexpr int kWarp = 32;
 constexpr unsigned kFull = 0xffffffffu;
 
 // Reroute tiling: pairs per tile and threads per tile.
-constexpr int kRerouteTile = 4096;
-constexpr int kRerouteThreads = 256;
+constexpr int kRerouteTile = 8192;
+constexpr int kRerouteThreads = 512;
 constexpr int kRerouteWarps = kRerouteThreads / kWarp;
 
-// Look-back status word: [31:30] flag, [29:0] count.
+// Look-back status word (64-bit): [63:32] launch tag, [31:30] flag,
+// [29:0] count. A word whose tag is not the current launch's reads as
+// "not yet published", so the words never need clearing between launches.
 constexpr uint32_t kFlagInvalid = 0u;
 constexpr uint32_t kFlagAggregate = 1u;
 constexpr uint32_t kFlagPrefix = 2u;
@@ -69,10 +71,14 @@ cudaError_t launch_count(const Sizes& z, const int32_t* idx, int32_t* load_re,
                          int32_t* load_e, int* err, cudaStream_t st);
 cudaError_t launch_plan(const Sizes& z, const int32_t* load_e,
                         const ue_placement& out, int* err, cudaStream_t st);
+// Reroute scratch: tiles*E 64-bit status words and sync[0..2] = {tile
+// ticket, finished CTAs, launch epoch}, zeroed once; each launch leaves them
+// ready for the next one (the last CTA resets the ticket and the counter and
+// advances the epoch).
 cudaError_t launch_reroute(const Sizes& z, const int32_t* idx,
                            const ue_placement& plan, int32_t* phys_slot,
-                           int32_t* dest_row, uint32_t* status,
-                           uint32_t* tile_counter, int64_t spin_limit,
+                           int32_t* dest_row, unsigned long long* status,
+                           uint32_t* sync, int64_t spin_limit,
                            int drop_first, int* err, cudaStream_t st);
 // Launch shapes of the row kernels, fixed once per context (ue_init) so that
 // a call only enqueues work (nothing else touches the runtime, which keeps

@@ -7,9 +7,12 @@
 // outside allocations, in a process whose device memory is reserved up front
 // by another runtime) or code that has no place to keep a context. This entry
 // point needs no context and allocates nothing. Its scratch (the look-back
-// status words and the tile ticket) is a file-scope __device__ array of fixed
-// size, which every GPU that loads this library holds until the process
-// exits.
+// status words, the tile ticket, the finished-CTA counter and the launch
+// epoch) is a file-scope __device__ array of fixed size, which every GPU that
+// loads this library holds until the process exits. The array starts zeroed
+// and is never cleared: status words carry their launch's epoch, so words
+// left by an earlier call read as unpublished, and the last CTA of every
+// call resets the ticket and the counter.
 //
 // The array's name, used in host code, is only a host-side stand-in for the
 // symbol, not a device address. The device address is fetched once per
@@ -21,19 +24,19 @@
 
 namespace {
 
-constexpr size_t kStatusWords = size_t(1) << 19;  // 2 MiB of look-back words
-constexpr size_t kCounterWord = kStatusWords;     // tile ticket
-constexpr size_t kErrWord = kStatusWords + 32;    // error word when none is given
-constexpr size_t kScratchWords = kStatusWords + 64;
+constexpr size_t kStatusWords = size_t(1) << 18;  // 2 MiB of 64-bit look-back words
+constexpr size_t kSyncWord = kStatusWords;        // ticket, counter, epoch (as 32-bit)
+constexpr size_t kErrWord = kStatusWords + 16;    // error word when none is given
+constexpr size_t kScratchWords = kStatusWords + 32;
 constexpr int kMaxDevices = 64;
 
-static __device__ __align__(256) uint32_t g_reroute_scratch[kScratchWords];
+static __device__ __align__(256) unsigned long long g_reroute_scratch[kScratchWords];
 
 std::mutex g_mutex;
-uint32_t* g_scratch_addr[kMaxDevices] = {};
+unsigned long long* g_scratch_addr[kMaxDevices] = {};
 
 // device address of g_reroute_scratch on the current device, looked up once
-ue_status scratch_address(uint32_t** out)
+ue_status scratch_address(unsigned long long** out)
 {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return UE_ERR_CUDA;
@@ -46,7 +49,7 @@ ue_status scratch_address(uint32_t** out)
             cudaGetLastError();
             return UE_ERR_CUDA;
         }
-        g_scratch_addr[dev] = static_cast<uint32_t*>(p);
+        g_scratch_addr[dev] = static_cast<unsigned long long*>(p);
     }
     *out = g_scratch_addr[dev];
     return UE_OK;
@@ -77,14 +80,14 @@ extern "C" ue_status ue_reroute_noalloc(const ue_config* cfg, const int32_t* idx
     const int64_t tiles = (z.Q + ue::kRerouteTile - 1) / ue::kRerouteTile;
     if ((size_t)tiles * (size_t)z.E > kStatusWords) return UE_ERR_UNSUPPORTED;
 
-    uint32_t* base = nullptr;
+    unsigned long long* base = nullptr;
     const ue_status st = scratch_address(&base);
     if (st != UE_OK) return st;
     int* err = error != nullptr ? reinterpret_cast<int*>(error)
                                 : reinterpret_cast<int*>(base + kErrWord);
-    // the launch clears the status words and the ticket it uses on the stream
-    const cudaError_t ce = ue::launch_reroute(z, idx, *plan, phys_slot, dest_row, base,
-                                              base + kCounterWord, int64_t(1) << 22, 0, err,
+    uint32_t* sync = reinterpret_cast<uint32_t*>(base + kSyncWord);
+    const cudaError_t ce = ue::launch_reroute(z, idx, *plan, phys_slot, dest_row, base, sync,
+                                              int64_t(1) << 22, 0, err,
                                               reinterpret_cast<cudaStream_t>(stream));
     return ce == cudaSuccess ? UE_OK : UE_ERR_CUDA;
 }
