@@ -266,6 +266,81 @@ def workload_config(w):
             "experts": "identity (combine reads the dispatch buffer)"}
 
 
+# ----------------------------------------------------------------- sweep ----
+def run_sweep(args):
+    """All 48 x 8 instances of the non-stationary sweep through one CUDA graph
+    of the whole path. Each instance's logits are staged into the input
+    buffer outside the timed region; each replay is timed with CUDA events.
+    Reports the distribution of us per layer and of the imbalance."""
+    import numpy as np
+    import torch
+
+    import synth
+    import token_rerouting_b200 as ue
+    from token_rerouting_b200 import build as ue_build
+
+    ue_build.build()
+    w = synth.WORKLOADS["sweep_48x8_r64_e128"]
+    dev = torch.device("cuda", 0)
+    L = ue.Layer(w.R, w.T, w.E, w.K, w.S, w.d, device=0)
+    L.hidden.copy_(torch.from_numpy(synth.hidden(w).view(np.int16)).to(dev).view(torch.bfloat16))
+    L.logits.copy_(torch.from_numpy(synth.logits(w, 0, 0)))
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        for _ in range(max(3, args.warmup)):
+            L.run(stream=s)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        L.run(stream=s)
+    torch.cuda.synchronize(dev)
+    stage = torch.empty(L.logits.shape, dtype=torch.float32).pin_memory()
+    times, before, after, copies = [], [], [], []
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(0)
+    clocks.start()
+    for layer in range(w.layers):
+        for mb in range(w.microbatches):
+            stage.copy_(torch.from_numpy(synth.logits(w, layer, mb)))
+            L.logits.copy_(stage, non_blocking=True)
+            torch.cuda.synchronize(dev)
+            a.record()
+            graph.replay()
+            b.record()
+            torch.cuda.synchronize(dev)
+            times.append(a.elapsed_time(b) * 1e3)
+            st = L.stats.cpu().numpy()
+            before.append(float(st[1]) / (w.Q / w.R))
+            after.append(float(st[2]) / (w.Q / w.R))
+            copies.append(int(st[0]))
+    clk = clocks.stop()
+    rc = L.error()
+    L.close()
+    if rc != 0:
+        raise SystemExit(f"device error in the sweep: {ue.STATUS.get(rc, rc)}")
+
+    def dist(x):
+        x = np.asarray(x, dtype=np.float64)
+        return {"min": float(x.min()), "median": float(np.median(x)), "max": float(x.max())}
+
+    total_s = sum(times) / 1e6
+    line = {
+        "metric": METRIC, "value": len(times) * w.Q / total_s, "unit": UNIT, "n_gpus": 1,
+        "steps": len(times), "warmup": max(3, args.warmup),
+        "ms_per_step": 1e3 * total_s / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "R": w.R, "T": w.T, "E": w.E, "K": w.K, "S": w.S,
+                   "d": w.d, "instances": len(times), "pairs_per_instance": w.Q,
+                   "graph": "whole path captured once, replayed per instance",
+                   "l2": "inputs larger than L2"},
+        "us_per_layer": dist(times), "max_over_mean_before": dist(before),
+        "max_over_mean_after": dist(after), "copies": dist(copies), "clocks": clk,
+        "gpu_launches": len(KERNELS) * len(times),
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ main ----
 def main():
     ap = argparse.ArgumentParser()
@@ -279,6 +354,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="the 48 x 8 non-stationary sweep, CUDA-graph captured")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -290,6 +367,9 @@ def main():
         w = dataclasses.replace(w, T=args.tokens_per_rank, name=f"{w.name}_t{args.tokens_per_rank}")
     if args.impl == "reference":
         run_reference(args, w)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
 
     world, rank, local = dist_setup(args.gpus)

@@ -54,8 +54,13 @@ def _bind(lib):
     lib.or_permute.argtypes = [p, i64, i32, i32, p, p]
     lib.or_permute_rows.argtypes = [p, i64, i32, i32, p, p, i64, p]
     lib.or_combine.argtypes = [p, i64, i32, i32, p, p, p, i64, p]
+    lib.or_combine_backward.argtypes = [p, p, i64, i32, i32, p, p, p, i64, p, p]
+    lib.or_permute_backward.argtypes = [p, i64, i32, i32, p, p, i64, p]
+    lib.or_weight_sync.argtypes = [i32, p, i32, p, p, i64]
+    lib.or_grad_reduce.argtypes = [i32, p, i32, p, p, i64, p]
     for f in ("or_gate_topk", "or_count", "or_plan", "or_reroute",
-              "or_permute", "or_permute_rows", "or_combine"):
+              "or_permute", "or_permute_rows", "or_combine", "or_combine_backward",
+              "or_permute_backward", "or_weight_sync", "or_grad_reduce"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -196,6 +201,73 @@ def combine(y_u16: np.ndarray, N: int, K: int, dest_row: np.ndarray,
         nt = 0
     _check(_load().or_combine(_ptr(y_u16), N, d, K, _ptr(dest_row), _ptr(w),
                               _ptr(tokens), nt, _ptr(out)), "combine")
+    return out
+
+
+def combine_backward(dout: np.ndarray, y_u16: np.ndarray, K: int, dest_row: np.ndarray,
+                     w: np.ndarray, tokens: np.ndarray | None = None):
+    """fp64 (dy rows per (token, k), dw [tokens][K]) of the combine's backward.
+    dout fp32 [N][d], y bf16 [Q][d], w fp32 [N][K]."""
+    dout = np.ascontiguousarray(dout, dtype=np.float32)
+    N, d = dout.shape
+    y_u16 = np.ascontiguousarray(y_u16, dtype=np.uint16)
+    dest_row = np.ascontiguousarray(dest_row, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    if tokens is not None:
+        tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+        cnt = tokens.size
+    else:
+        cnt = N
+    dy = np.empty((cnt * K, d), dtype=np.float64)
+    dw = np.empty((cnt, K), dtype=np.float64)
+    _check(_load().or_combine_backward(_ptr(dout), _ptr(y_u16), N, d, K, _ptr(dest_row),
+                                       _ptr(w), _ptr(tokens), cnt if tokens is not None else 0,
+                                       _ptr(dy), _ptr(dw)), "combine_backward")
+    return dy, dw
+
+
+def permute_backward(ddispatch_u16: np.ndarray, N: int, K: int, dest_row: np.ndarray,
+                     tokens: np.ndarray | None = None):
+    """fp64 dhidden[n] = sum_k ddispatch[dest_row[n, k]] (all or listed tokens)."""
+    ddispatch_u16 = np.ascontiguousarray(ddispatch_u16, dtype=np.uint16)
+    d = ddispatch_u16.shape[1]
+    dest_row = np.ascontiguousarray(dest_row, dtype=np.int32)
+    if tokens is not None:
+        tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+        cnt = tokens.size
+    else:
+        cnt = N
+    out = np.empty((cnt, d), dtype=np.float64)
+    _check(_load().or_permute_backward(_ptr(ddispatch_u16), N, d, K, _ptr(dest_row),
+                                       _ptr(tokens), cnt if tokens is not None else 0,
+                                       _ptr(out)), "permute_backward")
+    return out
+
+
+def weight_sync(slot_expert: np.ndarray, master: np.ndarray, replicas: np.ndarray):
+    """replicas[g] = master[slot_expert[g]] for every used slot (in place on a
+    copy of `replicas`); rows are raw bytes [E][B] and [G][B]."""
+    master = np.ascontiguousarray(master, dtype=np.uint8)
+    out = np.array(replicas, dtype=np.uint8, copy=True, order="C")
+    se = np.ascontiguousarray(slot_expert, dtype=np.int32)
+    G = se.size
+    E, B = master.shape
+    _check(_load().or_weight_sync(G, _ptr(se) if G else None, E, _ptr(master),
+                                  _ptr(out) if G else None, B), "weight_sync")
+    return out
+
+
+def grad_reduce(slot_expert: np.ndarray, replicas: np.ndarray, master: np.ndarray):
+    """fp64 master[e] + sum of e's replica gradients (ascending slot)."""
+    master = np.ascontiguousarray(master, dtype=np.float32)
+    E, W = master.shape
+    se = np.ascontiguousarray(slot_expert, dtype=np.int32)
+    G = se.size
+    replicas = np.ascontiguousarray(replicas, dtype=np.float32)
+    out = np.empty((E, W), dtype=np.float64)
+    _check(_load().or_grad_reduce(G, _ptr(se) if G else None, E,
+                                  _ptr(replicas) if G else None, _ptr(master), W, _ptr(out)),
+           "grad_reduce")
     return out
 
 

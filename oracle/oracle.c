@@ -3,7 +3,9 @@
  * expert rebalancing hot path of UltraEP:
  *
  *   gate top-k -> exact per-expert histogram -> quota-driven replication
- *   plan -> token-to-replica reroute -> permute -> gate-weighted combine.
+ *   plan -> token-to-replica reroute -> permute -> gate-weighted combine,
+ *   and beside it the backward of the permute and the combine, the weight
+ *   sync to replica slots and the gradient reduction to master experts.
  *
  * TEST INFRASTRUCTURE. Nothing in the product path links or calls this file.
  * Only the test suite, the package smoke check and the benchmark's
@@ -451,6 +453,123 @@ int or_combine(const uint16_t* y, int64_t N, int32_t d, int32_t K,
             for (int32_t c = 0; c < d; ++c)
                 out[j * d + c] += wk * or_bf16_to_double(y[row * d + c]);
         }
+    }
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* backward of permute and combine; weight sync; gradient reduction         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Backward of the gate-weighted combine ([P3] "Interface / 2. Forward and
+ * backward": reroute gathers gradients back to logical experts in backward;
+ * the combine is out[n] = sum_k w[n][k] * y[dest_row[n*K+k]]):
+ *     dy[dest_row[n*K+k]] = w[n][k] * dout[n]             (expert outputs)
+ *     dw[n][k]            = sum_c dout[n][c] * y[dest_row[n*K+k]][c]   (gates)
+ * in fp64. dout fp32 [N][d], y bf16 [Q][d], w fp32 [N][K]. Evaluated for the
+ * listed tokens (all when tokens == NULL): dy_rows gets one row per (token, k)
+ * in that order ([count*K][d]), dw one row per token ([count][K]).
+ */
+int or_combine_backward(const float* dout, const uint16_t* y, int64_t N, int32_t d,
+                        int32_t K, const int32_t* dest_row, const float* w,
+                        const int64_t* tokens, int64_t ntok, double* dy_rows, double* dw)
+{
+    if (!dout || !y || !dest_row || !w || !dy_rows || !dw || N < 0 || d < 1 || K < 1)
+        return OR_EINVAL;
+    int64_t Q = N * K;
+    int64_t count = tokens ? ntok : N;
+    for (int64_t j = 0; j < count; ++j) {
+        int64_t n = tokens ? tokens[j] : j;
+        if (n < 0 || n >= N) return OR_EDATA;
+        for (int32_t k = 0; k < K; ++k) {
+            int64_t row = dest_row[n * K + k];
+            if (row < 0 || row >= Q) return OR_EDATA;
+            double wk = (double)w[n * K + k];
+            double dot = 0.0;
+            for (int32_t c = 0; c < d; ++c) {
+                double g = (double)dout[n * d + c];
+                dy_rows[(j * K + k) * d + c] = wk * g;
+                dot += g * or_bf16_to_double(y[row * d + c]);
+            }
+            dw[j * K + k] = dot;
+        }
+    }
+    return OR_OK;
+}
+
+/*
+ * Backward of the permute (dispatch[dest_row[n*K+k]] = hidden[n]): every
+ * token's gradient is the sum of its K dispatched rows' gradients,
+ *     dhidden[n] = sum_k ddispatch[dest_row[n*K+k]]
+ * in fp64, for the listed tokens (all when tokens == NULL).
+ */
+int or_permute_backward(const uint16_t* ddispatch, int64_t N, int32_t d, int32_t K,
+                        const int32_t* dest_row, const int64_t* tokens, int64_t ntok,
+                        double* dhidden)
+{
+    if (!ddispatch || !dest_row || !dhidden || N < 0 || d < 1 || K < 1) return OR_EINVAL;
+    int64_t Q = N * K;
+    int64_t count = tokens ? ntok : N;
+    for (int64_t j = 0; j < count; ++j) {
+        int64_t n = tokens ? tokens[j] : j;
+        if (n < 0 || n >= N) return OR_EDATA;
+        for (int32_t c = 0; c < d; ++c) dhidden[j * d + c] = 0.0;
+        for (int32_t k = 0; k < K; ++k) {
+            int64_t row = dest_row[n * K + k];
+            if (row < 0 || row >= Q) return OR_EDATA;
+            for (int32_t c = 0; c < d; ++c)
+                dhidden[j * d + c] += or_bf16_to_double(ddispatch[row * d + c]);
+        }
+    }
+    return OR_OK;
+}
+
+/*
+ * Weight sync on one GPU ([P3] "Interface / 2. Forward and backward":
+ * weight_sync materializes the plan by distributing master weights to replica
+ * slots): every redundant slot g holding expert e receives a copy of e's
+ * weights, replicas[g] = master[e], bytes_per_expert bytes each; empty slots
+ * are left as they are.
+ */
+int or_weight_sync(int32_t G, const int32_t* slot_expert, int32_t E,
+                   const uint8_t* master, uint8_t* replicas, int64_t bytes_per_expert)
+{
+    if (G < 0 || (G > 0 && (!slot_expert || !replicas)) || !master || E < 1 ||
+        bytes_per_expert < 0)
+        return OR_EINVAL;
+    for (int32_t g = 0; g < G; ++g) {
+        int32_t e = slot_expert[g];
+        if (e < 0) continue;
+        if (e >= E) return OR_EDATA;
+        memcpy(replicas + (int64_t)g * bytes_per_expert, master + (int64_t)e * bytes_per_expert,
+               (size_t)bytes_per_expert);
+    }
+    return OR_OK;
+}
+
+/*
+ * Gradient reduction on one GPU ([P3] "Interface / 2. Forward and backward":
+ * grad_reduce reduces replica Wgrad into master-expert gradients; "Performance
+ * Tuning / Expert communication": a deterministic, non-atomic reduction):
+ *     master[e] + sum over the redundant slots g holding e, ascending g,
+ *     of replicas[g]
+ * in fp64 (fp32 inputs), written to out [E][numel].
+ */
+int or_grad_reduce(int32_t G, const int32_t* slot_expert, int32_t E, const float* replicas,
+                   const float* master, int64_t numel, double* out)
+{
+    if (G < 0 || (G > 0 && (!slot_expert || !replicas)) || !master || !out || E < 1 ||
+        numel < 0)
+        return OR_EINVAL;
+    for (int32_t e = 0; e < E; ++e)
+        for (int64_t i = 0; i < numel; ++i) out[(int64_t)e * numel + i] = (double)master[(int64_t)e * numel + i];
+    for (int32_t g = 0; g < G; ++g) {
+        int32_t e = slot_expert[g];
+        if (e < 0) continue;
+        if (e >= E) return OR_EDATA;
+        for (int64_t i = 0; i < numel; ++i)
+            out[(int64_t)e * numel + i] += (double)replicas[(int64_t)g * numel + i];
     }
     return OR_OK;
 }

@@ -15,6 +15,7 @@ import pytest
 import oracle
 from tests import test_oracle_gate as tg
 from tests import test_oracle_plan as tp
+from tests import test_oracle_backward as tb
 from tests import test_oracle_rows as tr
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
@@ -46,6 +47,16 @@ MUTANTS = {
     "permute_wrong_token": ("memcpy(dispatch + row * d, hidden + (i / K) * d,",
                             "memcpy(dispatch + row * d, hidden + (i % K) * d,"),
     "combine_first_weight_only": ("double wk = w[n * K + k];", "double wk = w[n * K];"),
+    "backward_dy_without_weight": ("dy_rows[(j * K + k) * d + c] = wk * g;",
+                                   "dy_rows[(j * K + k) * d + c] = g;"),
+    "backward_dw_wrong_row": ("dot += g * or_bf16_to_double(y[row * d + c]);",
+                              "dot += g * or_bf16_to_double(y[(n * K) * d + c]);"),
+    "permute_backward_drops_last_k": ("        for (int32_t k = 0; k < K; ++k) {\n            int64_t row = dest_row[n * K + k];\n            if (row < 0 || row >= Q) return OR_EDATA;\n            for (int32_t c = 0; c < d; ++c)\n                dhidden",
+                                      "        for (int32_t k = 0; k + 1 < K; ++k) {\n            int64_t row = dest_row[n * K + k];\n            if (row < 0 || row >= Q) return OR_EDATA;\n            for (int32_t c = 0; c < d; ++c)\n                dhidden"),
+    "weight_sync_wrong_source": ("memcpy(replicas + (int64_t)g * bytes_per_expert, master + (int64_t)e * bytes_per_expert,",
+                                 "memcpy(replicas + (int64_t)g * bytes_per_expert, master + (int64_t)g % E * bytes_per_expert,"),
+    "grad_reduce_skips_master": ("out[(int64_t)e * numel + i] = (double)master[(int64_t)e * numel + i];",
+                                 "out[(int64_t)e * numel + i] = 0.0;"),
 }
 
 
@@ -67,6 +78,13 @@ def run_pins(golden_dir):
         ("permute", tr.test_permute_definition_small),
         ("combine_exact", tr.test_combine_exact_dyadic_case),
         ("combine_identity", tr.test_combine_identity_experts_reproduce_hidden),
+        ("bwd_hand", tb.test_combine_backward_hand_case),
+        ("bwd_adjoint", tb.test_combine_backward_adjoint_identities),
+        ("pbwd_adjoint", tb.test_permute_backward_adjoint_identity),
+        ("pbwd_hand", tb.test_permute_backward_sums_k_rows),
+        ("wsync", tb.test_weight_sync_definition),
+        ("greduce_hand", tb.test_grad_reduce_dyadic_hand_case),
+        ("greduce_np", tb.test_grad_reduce_matches_numpy_add_at),
     ]
     failed = []
     for name, fn in pins:
