@@ -341,6 +341,97 @@ def run_sweep(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------- rows ----
+EXPERT_NUMEL = 2 * 4096 * 1536 + 4096 * 1536  # Qwen3-235B expert: fc1 2hf + fc2 hf
+
+
+def run_row(args, w):
+    """Backward of combine / permute, weight sync or gradient reduction on the
+    Qwen3-shaped layer (expert tensors of Qwen3-235B size), device-timed."""
+    import numpy as np
+    import torch
+
+    import token_rerouting_b200 as ue
+    from token_rerouting_b200 import build as ue_build
+
+    ue_build.build()
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev).manual_seed(0)
+    L = ue.Layer(w.R, w.T, w.E, w.K, w.S, w.d if args.row == "backward" else 8, device=0,
+                 with_rows=False)
+    L.logits.copy_(torch.from_numpy(synth_logits(w)))
+    L.run_routing()
+    torch.cuda.synchronize(dev)
+    peak, peak_kind = load_peaks()
+    st = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(args.steps):
+            fn()
+        b.record(st)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / args.steps / 1e3
+
+    kernels = {}
+    if args.row == "backward":
+        N, K, d, Q = w.N, w.K, w.d, w.Q
+        dout = torch.randn((N, d), dtype=torch.float32, device=dev, generator=gen)
+        y = torch.randn((Q, d), dtype=torch.float32, device=dev, generator=gen).to(torch.bfloat16)
+        dy = torch.empty_like(y)
+        dw = torch.empty((N, K), dtype=torch.float32, device=dev)
+        dh = torch.empty((N, d), dtype=torch.float32, device=dev)
+        t1 = timed(lambda: ue.ue_combine_backward(L.ctx, dout, y, L.dest_row, L.w, dy, dw, st))
+        t2 = timed(lambda: ue.ue_permute_backward(L.ctx, y, L.dest_row, dh, st))
+        kernels["combine_backward"] = (t1, 4 * N * d + 2 * Q * d + 8 * Q + 2 * Q * d + 4 * Q)
+        kernels["permute_backward"] = (t2, 2 * Q * d + 4 * Q + 4 * N * d)
+        workload = dict(workload=w.name, N=N, K=K, d=d, pairs=Q)
+    else:
+        plan = L.plan_arrays()
+        se = plan["slot_expert"]
+        used = int((se >= 0).sum())
+        cnt = np.bincount(se[se >= 0], minlength=w.E)
+        if args.row == "weight_sync":
+            bpe = EXPERT_NUMEL * 2
+            master = torch.randint(-30000, 30000, (w.E, EXPERT_NUMEL), dtype=torch.int16,
+                                   device=dev, generator=gen)
+            reps = torch.empty((w.G, EXPERT_NUMEL), dtype=torch.int16, device=dev)
+            t = timed(lambda: ue.ue_weight_sync(L.ctx, L.plan, master, reps, bpe, st))
+            kernels["weight_sync"] = (t, 2 * used * bpe)
+        else:
+            master = torch.randn((w.E, EXPERT_NUMEL), dtype=torch.float32, device=dev, generator=gen)
+            reps = torch.randn((w.G, EXPERT_NUMEL), dtype=torch.float32, device=dev, generator=gen)
+            t = timed(lambda: ue.ue_grad_reduce(L.ctx, L.plan, reps, master, EXPERT_NUMEL, st))
+            nrep = int((cnt > 0).sum())
+            kernels["grad_reduce"] = (t, 4 * EXPERT_NUMEL * (2 * nrep + used))
+        workload = dict(workload=w.name, expert_numel=EXPERT_NUMEL, replicas=used,
+                        replicated_experts=int((cnt > 0).sum()),
+                        expert_shape="Qwen3-235B expert: fc1 2*4096*1536 + fc2 4096*1536")
+    rc = L.error()
+    L.close()
+    if rc != 0:
+        raise SystemExit(f"device error: {rc}")
+    out = {}
+    for k, (t, by) in kernels.items():
+        gbs = by / t / 1e9
+        out[k] = {"us": t * 1e6, "algorithmic_bytes": by, "gbs": gbs, "frac_of_peak": gbs / peak}
+    dom = max(out, key=lambda k: out[k]["us"])
+    line = {"row": args.row, "config": workload, "steps": args.steps, "kernels": out,
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": out[dom]["gbs"], "peak": peak,
+                         "unit": "GB/s", "frac": out[dom]["frac_of_peak"],
+                         "peak_kind": f"of {peak_kind}"}}
+    print(json.dumps(line), flush=True)
+
+
+def synth_logits(w):
+    import synth
+    return synth.logits(w)
+
+
 # ------------------------------------------------------------------ main ----
 def main():
     ap = argparse.ArgumentParser()
@@ -356,6 +447,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="the 48 x 8 non-stationary sweep, CUDA-graph captured")
+    ap.add_argument("--row", choices=("backward", "weight_sync", "grad_reduce"), default=None,
+                    help="measure one of the rows beside the forward path")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -370,6 +463,9 @@ def main():
         return
     if args.sweep:
         run_sweep(args)
+        return
+    if args.row:
+        run_row(args, w)
         return
 
     world, rank, local = dist_setup(args.gpus)

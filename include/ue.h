@@ -192,6 +192,55 @@ ue_status ue_permute(ue_ctx* ctx, const uint16_t* hidden,
 ue_status ue_combine(ue_ctx* ctx, const uint16_t* y, const int32_t* dest_row,
                      const float* w, float* out, void* stream);
 
+/* Backward of the combine ("Interface / 2. Forward and backward": reroute
+ * gathers gradients back to logical experts in the backward; with the
+ * compact [N][K] routing each pair has one physical row, so the gradients
+ * are those of the combine):
+ *   dout     fp32 [N][d], 16-byte aligned: gradient of `out`.
+ *   y        bf16 [Q][d]: the expert outputs the forward combined.
+ *   dest_row int32 [N][K], w fp32 [N][K]: as in the forward.
+ *   dy       bf16 [Q][d], 16-byte aligned: dy[dest_row[n*K+k]] =
+ *            w[n][k] * dout[n], product in fp32 rounded once to bf16.
+ *   dw       fp32 [N][K]: dw[n][k] = <dout[n], y[dest_row[n*K+k]]>,
+ *            accumulated in fp32 in a fixed order (the same on every run).
+ * Rows outside [0, Q) are skipped and set UE_ERR_DEVICE_BOUNDS. */
+ue_status ue_combine_backward(ue_ctx* ctx, const float* dout, const uint16_t* y,
+                              const int32_t* dest_row, const float* w, uint16_t* dy,
+                              float* dw, void* stream);
+
+/* Backward of the permute: dhidden[n] = sum_k ddispatch[dest_row[n*K+k]],
+ * fp32 [N][d] (16-byte aligned), k ascending from 0; ddispatch bf16 [Q][d].
+ * Rows outside [0, Q) are skipped and set UE_ERR_DEVICE_BOUNDS. */
+ue_status ue_permute_backward(ue_ctx* ctx, const uint16_t* ddispatch,
+                              const int32_t* dest_row, float* dhidden, void* stream);
+
+/* Weight sync on one GPU ("Interface / 2. Forward and backward":
+ * weight_sync distributes master-expert weights to the replica slots;
+ * "Interface / 1. Initialization": replica buffers reused across layers).
+ *   plan             a placement from ue_plan (slot_expert is read).
+ *   master           [E][bytes_per_expert] bytes, 16-byte aligned.
+ *   replicas         [G][bytes_per_expert] bytes, 16-byte aligned:
+ *                    replicas[g] = master[slot_expert[g]] for every used
+ *                    slot; empty slots are left unchanged.
+ *   bytes_per_expert > 0 and a multiple of 16 (e.g. bf16 fc1 + fc2 weights:
+ *                    2 * (2*h*f + h*f) bytes).
+ * A slot_expert entry >= E sets UE_ERR_DEVICE_BOUNDS. */
+ue_status ue_weight_sync(ue_ctx* ctx, const ue_placement* plan, const void* master,
+                         void* replicas, int64_t bytes_per_expert, void* stream);
+
+/* Gradient reduction on one GPU ("Interface / 2. Forward and backward":
+ * grad_reduce reduces replica Wgrad into master-expert gradients;
+ * "Performance Tuning / Expert communication": deterministic, non-atomic).
+ *   plan             a placement from ue_plan (slot_expert is read).
+ *   replica_grads    fp32 [G][numel_per_expert], 16-byte aligned.
+ *   master_grads     fp32 [E][numel_per_expert], 16-byte aligned, updated in
+ *                    place: master[e] = master[e] + replicas[g1] + ... over
+ *                    e's replica slots in ascending g, added in that order,
+ *                    so the result is the same on every run.
+ *   numel_per_expert > 0 and a multiple of 4. */
+ue_status ue_grad_reduce(ue_ctx* ctx, const ue_placement* plan, const float* replica_grads,
+                         float* master_grads, int64_t numel_per_expert, void* stream);
+
 /* ue_reroute, without a context and without allocating anything (the
  * pages have no counterpart to this call). For callers that cannot call
  * cudaMalloc: code running inside an allocator's hooks or under a memory

@@ -32,7 +32,8 @@ UE_ERR_DEVICE_BOUNDS, UE_ERR_TIMEOUT, UE_ERR_UNSUPPORTED = 4, 5, 6
 
 # every symbol include/ue.h declares
 EXPORTS = ("ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count",
-           "ue_plan", "ue_reroute", "ue_permute", "ue_combine", "ue_reroute_noalloc",
+           "ue_plan", "ue_reroute", "ue_permute", "ue_combine", "ue_combine_backward",
+           "ue_permute_backward", "ue_weight_sync", "ue_grad_reduce", "ue_reroute_noalloc",
            "ue_debug_set_lookback_limit", "ue_debug_drop_first_publish")
 
 
@@ -76,6 +77,10 @@ def load_library(path: str | None = None):
     lib.ue_reroute.argtypes = [vp, vp, ctypes.POINTER(ue_placement), vp, vp, vp]
     lib.ue_permute.argtypes = [vp, vp, vp, vp, vp]
     lib.ue_combine.argtypes = [vp, vp, vp, vp, vp, vp]
+    lib.ue_combine_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.ue_permute_backward.argtypes = [vp, vp, vp, vp, vp]
+    lib.ue_weight_sync.argtypes = [vp, ctypes.POINTER(ue_placement), vp, vp, i64, vp]
+    lib.ue_grad_reduce.argtypes = [vp, ctypes.POINTER(ue_placement), vp, vp, i64, vp]
     lib.ue_reroute_noalloc.argtypes = [ctypes.POINTER(ue_config), vp,
                                        ctypes.POINTER(ue_placement), vp, vp, vp, vp]
     lib.ue_debug_set_lookback_limit.argtypes = [vp, i64]
@@ -168,6 +173,32 @@ def ue_combine(ctx, y, dest_row, w, out, stream=None):
                                                 _ptr(out), _stream(stream)))
 
 
+def ue_combine_backward(ctx, dout, y, dest_row, w, dy, dw, stream=None):
+    _ok("ue_combine_backward",
+        load_library().ue_combine_backward(ctx, _ptr(dout), _ptr(y), _ptr(dest_row), _ptr(w),
+                                           _ptr(dy), _ptr(dw), _stream(stream)))
+
+
+def ue_permute_backward(ctx, ddispatch, dest_row, dhidden, stream=None):
+    _ok("ue_permute_backward",
+        load_library().ue_permute_backward(ctx, _ptr(ddispatch), _ptr(dest_row), _ptr(dhidden),
+                                           _stream(stream)))
+
+
+def ue_weight_sync(ctx, plan: ue_placement, master, replicas, bytes_per_expert: int,
+                   stream=None):
+    _ok("ue_weight_sync",
+        load_library().ue_weight_sync(ctx, ctypes.byref(plan), _ptr(master), _ptr(replicas),
+                                      bytes_per_expert, _stream(stream)))
+
+
+def ue_grad_reduce(ctx, plan: ue_placement, replica_grads, master_grads, numel_per_expert: int,
+                   stream=None):
+    _ok("ue_grad_reduce",
+        load_library().ue_grad_reduce(ctx, ctypes.byref(plan), _ptr(replica_grads),
+                                      _ptr(master_grads), numel_per_expert, _stream(stream)))
+
+
 def ue_reroute_noalloc(cfg: ue_config, idx, plan: ue_placement, phys_slot, dest_row,
                        error=None, stream=None):
     """ue_reroute without a context; allocates nothing (see include/ue.h)."""
@@ -190,7 +221,8 @@ def ue_debug_drop_first_publish(ctx, enable: bool):
 from .layer import Layer  # noqa: E402  (buffers + one call per step)
 
 __all__ = ["ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count", "ue_plan",
-           "ue_reroute", "ue_permute", "ue_combine", "ue_reroute_noalloc",
+           "ue_reroute", "ue_permute", "ue_combine", "ue_combine_backward",
+           "ue_permute_backward", "ue_weight_sync", "ue_grad_reduce", "ue_reroute_noalloc",
            "ue_debug_set_lookback_limit",
            "ue_debug_drop_first_publish", "ue_config", "ue_placement", "make_config",
            "placement", "load_library", "Layer", "UEError", "STATUS", "EXPORTS"]

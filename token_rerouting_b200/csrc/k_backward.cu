@@ -1,0 +1,155 @@
+// k_backward.cu -- backward of the gate-weighted combine.
+//
+// "UltraEP" README, "Interface / 2. Forward and backward": reroute expands
+// logical routing to physical replicas in the forward and gathers gradients
+// back to logical experts in the backward. With the compact [N][K] routing
+// each pair maps to one physical row, so the gradient that reaches the
+// router's gates and the one that reaches the expert outputs are those of
+// the combine out[n] = sum_k w[n][k] * y[dest_row[n*K+k]]:
+//     dy[dest_row[n*K+k]] = w[n][k] * dout[n]      (bf16, rounded once)
+//     dw[n][k]            = <dout[n], y[dest_row[n*K+k]]>   (fp32)
+// (The permute's backward, dhidden[n] = sum_k ddispatch[dest_row[n*K+k]], is
+// the combine with unit weights and runs in k_combine.cu.)
+//
+// Design (B200): HBM-bound (per pair: 2d bytes of y read, 2d bytes of dy
+// written; per token 4d bytes of dout read once). A group of threads owns a
+// token; each thread owns 16-byte chunks of the row (8 elements), reads the
+// token's fp32 gradient chunk once, then for each k reads the y chunk,
+// accumulates the dot product in fp32 (fixed order) and writes w*dout as
+// bf16. The per-thread partial dots are summed by a fixed tree (warp
+// shuffles, then a shared-memory pass across the token's warps), so dw is
+// deterministic.
+#include <cuda_bf16.h>
+
+#include "ue_internal.cuh"
+
+namespace ue {
+namespace {
+
+constexpr int kBwdThreads = 256;
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+    const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    return a | (b << 16);
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(kBwdThreads)
+combine_bwd_kernel(const float* __restrict__ dout, const uint16_t* __restrict__ y,
+                   const int32_t* __restrict__ dest_row, const float* __restrict__ w,
+                   uint16_t* __restrict__ dy, float* __restrict__ dw, int64_t N, int K, int d,
+                   int tpt, int64_t Q, int* err)
+{
+    __shared__ float s_part[kBwdThreads / 32][KMAX];
+    const int C = d >> 3;
+    const int tpb = blockDim.x / tpt;
+    const int sub = threadIdx.x / tpt;
+    const int lt = threadIdx.x - sub * tpt;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int wpt = (tpt + 31) / 32;  // warps per token (tpt >= 32)
+    // token groups never straddle a warp (tpt is a multiple of 32)
+    for (int64_t n0 = (int64_t)blockIdx.x * tpb; n0 < N; n0 += (int64_t)gridDim.x * tpb) {
+        const int64_t n = n0 + sub;
+        const bool live = sub < tpb && n < N;
+        int rows[KMAX];
+        float wk[KMAX], part[KMAX];
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            rows[k] = -1;
+            wk[k] = 0.0f;
+            part[k] = 0.0f;
+            if (live && k < K) {
+                const int r = __ldg(dest_row + n * K + k);
+                if (r >= 0 && (int64_t)r < Q) {
+                    rows[k] = r;
+                    wk[k] = __ldg(w + n * K + k);
+                } else if (lt == 0) {
+                    raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(n * K + k, (int64_t)INT_MAX));
+                }
+            }
+        }
+        for (int c = lt; live && c < C; c += tpt) {
+            const float4 g0 = __ldcs(reinterpret_cast<const float4*>(dout + n * d) + 2 * c);
+            const float4 g1 = __ldcs(reinterpret_cast<const float4*>(dout + n * d) + 2 * c + 1);
+            const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            uint4 v[KMAX];
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k)
+                v[k] = rows[k] >= 0 ? __ldcs(reinterpret_cast<const uint4*>(y + (int64_t)rows[k] * d) + c)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k) {
+                if (rows[k] < 0) continue;
+                const uint32_t u[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    part[k] = fmaf(g[2 * q], __uint_as_float(u[q] << 16), part[k]);
+                    part[k] = fmaf(g[2 * q + 1], __uint_as_float(u[q] & 0xffff0000u), part[k]);
+                }
+                uint4 o;
+                o.x = pack_bf16x2(wk[k] * g[0], wk[k] * g[1]);
+                o.y = pack_bf16x2(wk[k] * g[2], wk[k] * g[3]);
+                o.z = pack_bf16x2(wk[k] * g[4], wk[k] * g[5]);
+                o.w = pack_bf16x2(wk[k] * g[6], wk[k] * g[7]);
+                __stcs(reinterpret_cast<uint4*>(dy + (int64_t)rows[k] * d) + c, o);
+            }
+        }
+        // dw: fixed-order tree over the token's threads
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            float p = part[k];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(kFull, p, off);
+            if (lane == 0) s_part[warp][k] = p;
+        }
+        __syncthreads();
+        if (live && lt == 0) {
+            const int w0 = warp;  // the token's first warp
+            for (int k = 0; k < K && k < KMAX; ++k) {
+                float acc = 0.0f;
+                for (int ww = 0; ww < wpt; ++ww) acc += s_part[w0 + ww][k];
+                if (rows[k] >= 0) dw[n * K + k] = acc;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+template <int KMAX>
+cudaError_t launch_k(const Sizes& z, const float* dout, const uint16_t* y, const int32_t* dest_row,
+                     const float* w, uint16_t* dy, float* dw, int num_sms, int* err,
+                     cudaStream_t st)
+{
+    const int C = z.d / 8;
+    int tpt = 32;
+    while (tpt < C && tpt < kBwdThreads) tpt <<= 1;
+    const int tpb = kBwdThreads / tpt;
+    int per_sm = 0;
+    cudaError_t ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_bwd_kernel<KMAX>,
+                                                                   kBwdThreads, 0);
+    if (ce != cudaSuccess) return ce;
+    per_sm = std::max(per_sm, 1);
+    const int64_t need = std::max<int64_t>(1, (z.N + tpb - 1) / tpb);
+    const int grid = (int)std::min<int64_t>(need, (int64_t)num_sms * per_sm);
+    combine_bwd_kernel<KMAX><<<grid, kBwdThreads, 0, st>>>(dout, y, dest_row, w, dy, dw, z.N, z.K,
+                                                           z.d, tpt, z.Q, err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_combine_backward(const Sizes& z, const float* dout, const uint16_t* y,
+                                    const int32_t* dest_row, const float* w, uint16_t* dy,
+                                    float* dw, int num_sms, int* err, cudaStream_t st)
+{
+    if (z.N == 0) return cudaSuccess;
+    if (z.K <= 4) return launch_k<4>(z, dout, y, dest_row, w, dy, dw, num_sms, err, st);
+    if (z.K <= 8) return launch_k<8>(z, dout, y, dest_row, w, dy, dw, num_sms, err, st);
+    if (z.K <= 16) return launch_k<16>(z, dout, y, dest_row, w, dy, dw, num_sms, err, st);
+    return launch_k<32>(z, dout, y, dest_row, w, dy, dw, num_sms, err, st);
+}
+
+}  // namespace ue

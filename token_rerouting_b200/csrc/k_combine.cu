@@ -17,7 +17,9 @@ namespace {
 
 constexpr int kCombineThreads = 256;
 
-template <int KMAX>
+// UNIT: every weight is 1 (the backward of the permute: the sum of a token's
+// K dispatched rows); w is not read.
+template <int KMAX, bool UNIT>
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ dest_row,
                const float* __restrict__ w, float* __restrict__ out, int64_t N, int K,
@@ -39,7 +41,7 @@ combine_kernel(const uint16_t* __restrict__ y, const int32_t* __restrict__ dest_
                 const int r = __ldg(dest_row + n * K + k);
                 if (r >= 0 && (int64_t)r < Q) {
                     rows[k] = r;
-                    wk[k] = __ldg(w + n * K + k);
+                    wk[k] = UNIT ? 1.0f : __ldg(w + n * K + k);
                 } else if (lt == 0) {
                     raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(n * K + k, (int64_t)INT_MAX));
                 }
@@ -83,7 +85,7 @@ cudaError_t shape_k(const Sizes& z, int num_sms, CombineShape* out)
     while (tpt < C && tpt < kCombineThreads) tpt <<= 1;
     const int tpb = kCombineThreads / tpt;
     int per_sm = 0;
-    cudaError_t ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_kernel<KMAX>,
+    cudaError_t ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_kernel<KMAX, false>,
                                                                    kCombineThreads, 0);
     if (ce != cudaSuccess) return ce;
     per_sm = std::max(per_sm, 1);
@@ -108,9 +110,16 @@ cudaError_t launch_combine(const Sizes& z, const CombineShape& sh, const uint16_
                            cudaStream_t st)
 {
     if (z.N == 0) return cudaSuccess;
-#define UE_COMBINE(KM)                                                                          \
-    combine_kernel<KM><<<sh.grid, kCombineThreads, 0, st>>>(y, dest_row, w, out, z.N, z.K, z.d, \
-                                                             sh.tpt, z.Q, err)
+    const bool unit = (w == nullptr);
+#define UE_COMBINE(KM)                                                                         \
+    do {                                                                                       \
+        if (unit)                                                                              \
+            combine_kernel<KM, true><<<sh.grid, kCombineThreads, 0, st>>>(                     \
+                y, dest_row, w, out, z.N, z.K, z.d, sh.tpt, z.Q, err);                         \
+        else                                                                                   \
+            combine_kernel<KM, false><<<sh.grid, kCombineThreads, 0, st>>>(                    \
+                y, dest_row, w, out, z.N, z.K, z.d, sh.tpt, z.Q, err);                         \
+    } while (0)
     if (z.K <= 4) UE_COMBINE(4);
     else if (z.K <= 8) UE_COMBINE(8);
     else if (z.K <= 16) UE_COMBINE(16);

@@ -218,6 +218,58 @@ ue_status ue_combine(ue_ctx* ctx, const uint16_t* y, const int32_t* dest_row, co
                                         as_stream(stream)));
 }
 
+ue_status ue_combine_backward(ue_ctx* ctx, const float* dout, const uint16_t* y,
+                              const int32_t* dest_row, const float* w, uint16_t* dy, float* dw,
+                              void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(dout, 16) || !aligned(y, 16) || !aligned(dest_row, 4) ||
+        !aligned(w, 4) || !aligned(dy, 16) || !aligned(dw, 4))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_combine_backward(ctx->z, dout, y, dest_row, w, dy, dw,
+                                                 ctx->num_sms, ctx->d_err, as_stream(stream)));
+}
+
+ue_status ue_permute_backward(ue_ctx* ctx, const uint16_t* ddispatch, const int32_t* dest_row,
+                              float* dhidden, void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(ddispatch, 16) || !aligned(dest_row, 4) ||
+        !aligned(dhidden, 16))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    // the combine with every weight equal to 1
+    return from_cuda(ue::launch_combine(ctx->z, ctx->comb, ddispatch, dest_row, nullptr, dhidden,
+                                        ctx->d_err, as_stream(stream)));
+}
+
+ue_status ue_weight_sync(ue_ctx* ctx, const ue_placement* plan, const void* master,
+                         void* replicas, int64_t bytes_per_expert, void* stream)
+{
+    if (!ctx_ok(ctx) || plan == nullptr || !aligned(master, 16) || bytes_per_expert <= 0 ||
+        bytes_per_expert % 16 != 0)
+        return UE_ERR_INVALID_ARG;
+    if (ctx->z.G > 0 && (!aligned(plan->slot_expert, 4) || !aligned(replicas, 16)))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_weight_sync(ctx->z, plan->slot_expert, master, replicas,
+                                            bytes_per_expert, ctx->num_sms, ctx->d_err,
+                                            as_stream(stream)));
+}
+
+ue_status ue_grad_reduce(ue_ctx* ctx, const ue_placement* plan, const float* replica_grads,
+                         float* master_grads, int64_t numel_per_expert, void* stream)
+{
+    if (!ctx_ok(ctx) || plan == nullptr || !aligned(master_grads, 16) ||
+        numel_per_expert <= 0 || numel_per_expert % 4 != 0)
+        return UE_ERR_INVALID_ARG;
+    if (ctx->z.G > 0 && (!aligned(plan->slot_expert, 4) || !aligned(replica_grads, 16)))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_grad_reduce(ctx->z, plan->slot_expert, replica_grads,
+                                            master_grads, numel_per_expert, ctx->num_sms,
+                                            ctx->d_err, as_stream(stream)));
+}
+
 ue_status ue_debug_set_lookback_limit(ue_ctx* ctx, int64_t polls)
 {
     if (!ctx_ok(ctx) || polls < 0) return UE_ERR_INVALID_ARG;

@@ -101,4 +101,16 @@ cudaError_t launch_combine(const Sizes& z, const CombineShape& sh, const uint16_
 
 int gate_topk_grid(const Sizes& z, int num_sms);
 
+// Beside the forward path: backward of the combine (the permute's backward
+// is launch_combine with w == nullptr), weight sync and gradient reduction.
+cudaError_t launch_combine_backward(const Sizes& z, const float* dout, const uint16_t* y,
+                                    const int32_t* dest_row, const float* w, uint16_t* dy,
+                                    float* dw, int num_sms, int* err, cudaStream_t st);
+cudaError_t launch_weight_sync(const Sizes& z, const int32_t* slot_expert, const void* master,
+                               void* replicas, int64_t bytes_per_expert, int num_sms, int* err,
+                               cudaStream_t st);
+cudaError_t launch_grad_reduce(const Sizes& z, const int32_t* slot_expert, const float* replicas,
+                               float* master, int64_t numel_per_expert, int num_sms, int* err,
+                               cudaStream_t st);
+
 }  // namespace ue
