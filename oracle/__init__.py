@@ -49,8 +49,12 @@ def _bind(lib):
     p = ctypes.c_void_p
     lib.or_gate_topk.argtypes = [p, i64, i32, i32, p, p]
     lib.or_count.argtypes = [p, i32, i32, i32, i32, p, p]
-    lib.or_plan.argtypes = [i32, i32, i32, p, p, p, p, p, p, p, p, p]
+    lib.or_plan.argtypes = [i32, i32, i32, p, i32, p, p, p, p, p, p, p, p]
+    lib.or_plan_bisect.argtypes = [i32, i32, i32, p, i32, i32, i32, i32, p, p, p, p, p, p]
     lib.or_reroute.argtypes = [p, i64, i32, i32, i32, p, p, p, p, p]
+    lib.or_reroute_interleave.argtypes = [p, i32, i32, i32, i32, i32, p, p, p, p, p]
+    lib.or_locality_split.argtypes = [i32, i32, i32, p, p, p, p, p, p]
+    lib.or_reroute_local.argtypes = [p, i32, i32, i32, i32, i32, p, p, p, p, p]
     lib.or_permute.argtypes = [p, i64, i32, i32, p, p]
     lib.or_permute_rows.argtypes = [p, i64, i32, i32, p, p, i64, p]
     lib.or_combine.argtypes = [p, i64, i32, i32, p, p, p, i64, p]
@@ -58,7 +62,8 @@ def _bind(lib):
     lib.or_permute_backward.argtypes = [p, i64, i32, i32, p, p, i64, p]
     lib.or_weight_sync.argtypes = [i32, p, i32, p, p, i64]
     lib.or_grad_reduce.argtypes = [i32, p, i32, p, p, i64, p]
-    for f in ("or_gate_topk", "or_count", "or_plan", "or_reroute",
+    for f in ("or_gate_topk", "or_count", "or_plan", "or_plan_bisect", "or_reroute",
+              "or_reroute_interleave", "or_locality_split", "or_reroute_local",
               "or_permute", "or_permute_rows", "or_combine", "or_combine_backward",
               "or_permute_backward", "or_weight_sync", "or_grad_reduce"):
         getattr(lib, f).restype = ctypes.c_int
@@ -120,8 +125,10 @@ class Plan:
     trace_r: np.ndarray      # [iterations] chosen rank per iteration
 
 
-def plan(load_e: np.ndarray, R: int, S: int) -> Plan:
-    """Greedy quota-driven replication plan from the exact per-expert load."""
+def plan(load_e: np.ndarray, R: int, S: int, min_tokens: int = 0) -> Plan:
+    """Greedy quota-driven replication plan from the exact per-expert load
+    (min_tokens > 0: an expert takes another copy only if each of its copies
+    keeps at least min_tokens pairs)."""
     load_e = np.ascontiguousarray(load_e, dtype=np.int32)
     E = load_e.shape[0]
     M = E // R
@@ -134,13 +141,87 @@ def plan(load_e: np.ndarray, R: int, S: int) -> Plan:
     stats = np.empty(4, dtype=np.int32)
     te = np.full(max(G, 1), -1, dtype=np.int32)
     tr = np.full(max(G, 1), -1, dtype=np.int32)
-    _check(_load().or_plan(R, E, S, _ptr(load_e), _ptr(slot_expert),
+    _check(_load().or_plan(R, E, S, _ptr(load_e), min_tokens, _ptr(slot_expert),
                            _ptr(n_copies), _ptr(slot_quota), _ptr(slot_offset),
                            _ptr(rank_load), _ptr(stats), _ptr(te), _ptr(tr)),
            "plan")
     it = int(stats[0])
     return Plan(slot_expert[:G].copy(), n_copies, slot_quota, slot_offset,
                 rank_load, stats, te[:it].copy(), tr[:it].copy())
+
+
+def plan_bisect(load_e: np.ndarray, R: int, S: int, eps_inv: int = 100,
+                threshold: int | None = None, min_tokens: int = 1024,
+                allow_zero_master: bool = False) -> Plan:
+    """Capacity planner: bisection on max/mean over the grid k/eps_inv with a
+    quota oracle per probe. threshold is the early-stop ratio in units of
+    1/eps_inv (default eps_inv, i.e. 1.0). stats = {probes, max before, max
+    after, final k}; trace_e / trace_r are empty."""
+    load_e = np.ascontiguousarray(load_e, dtype=np.int32)
+    E = load_e.shape[0]
+    M = E // R
+    G, P = R * S, R * (M + S)
+    thr = eps_inv if threshold is None else threshold
+    slot_expert = np.empty(max(G, 1), dtype=np.int32)
+    n_copies = np.empty(E, dtype=np.int32)
+    slot_quota = np.empty(P, dtype=np.int32)
+    slot_offset = np.empty(P + 1, dtype=np.int32)
+    rank_load = np.empty(R, dtype=np.int32)
+    stats = np.empty(4, dtype=np.int32)
+    _check(_load().or_plan_bisect(R, E, S, _ptr(load_e), eps_inv, thr, min_tokens,
+                                  int(bool(allow_zero_master)), _ptr(slot_expert),
+                                  _ptr(n_copies), _ptr(slot_quota), _ptr(slot_offset),
+                                  _ptr(rank_load), _ptr(stats)), "plan_bisect")
+    empty = np.empty(0, dtype=np.int32)
+    return Plan(slot_expert[:G].copy(), n_copies, slot_quota, slot_offset, rank_load,
+                stats, empty, empty)
+
+
+def _slot_expert_arg(pl: Plan):
+    se = np.ascontiguousarray(pl.slot_expert, dtype=np.int32)
+    return se if se.size else np.full(1, -1, dtype=np.int32)
+
+
+def reroute_interleave(idx: np.ndarray, R: int, T: int, E: int, S: int, pl: Plan):
+    """Prefix-fill reroute with the pairs taken in (token, rank, k) order."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    K = idx.size // (R * T) if R * T else 1
+    phys = np.empty(idx.shape, dtype=np.int32)
+    dest = np.empty(idx.shape, dtype=np.int32)
+    _check(_load().or_reroute_interleave(_ptr(idx), R, T, K, E, S, _ptr(_slot_expert_arg(pl)),
+                                         _ptr(np.ascontiguousarray(pl.slot_quota)),
+                                         _ptr(np.ascontiguousarray(pl.slot_offset)),
+                                         _ptr(phys), _ptr(dest)), "reroute_interleave")
+    return phys, dest
+
+
+def locality_split(load_re: np.ndarray, S: int, pl: Plan):
+    """Per-source-rank split of every copy's quota, own rank first:
+    (src_quota [R][P], src_offset [R][P])."""
+    load_re = np.ascontiguousarray(load_re, dtype=np.int32)
+    R, E = load_re.shape
+    P = pl.slot_quota.size
+    src_quota = np.empty((R, P), dtype=np.int32)
+    src_offset = np.empty((R, P), dtype=np.int32)
+    _check(_load().or_locality_split(R, E, S, _ptr(load_re), _ptr(_slot_expert_arg(pl)),
+                                     _ptr(np.ascontiguousarray(pl.slot_quota)),
+                                     _ptr(np.ascontiguousarray(pl.slot_offset)),
+                                     _ptr(src_quota), _ptr(src_offset)), "locality_split")
+    return src_quota, src_offset
+
+
+def reroute_local(idx: np.ndarray, R: int, T: int, E: int, S: int, pl: Plan,
+                  src_quota: np.ndarray, src_offset: np.ndarray):
+    """Reroute under the locality-aware split."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    K = idx.size // (R * T) if R * T else 1
+    phys = np.empty(idx.shape, dtype=np.int32)
+    dest = np.empty(idx.shape, dtype=np.int32)
+    _check(_load().or_reroute_local(_ptr(idx), R, T, K, E, S, _ptr(_slot_expert_arg(pl)),
+                                    _ptr(np.ascontiguousarray(src_quota, dtype=np.int32)),
+                                    _ptr(np.ascontiguousarray(src_offset, dtype=np.int32)),
+                                    _ptr(phys), _ptr(dest)), "reroute_local")
+    return phys, dest
 
 
 def reroute(idx: np.ndarray, R: int, E: int, S: int, pl: Plan):

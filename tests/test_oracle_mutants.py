@@ -17,6 +17,7 @@ from tests import test_oracle_gate as tg
 from tests import test_oracle_plan as tp
 from tests import test_oracle_backward as tb
 from tests import test_oracle_rows as tr
+from tests import test_oracle_variants as tv
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 
@@ -55,6 +56,28 @@ MUTANTS = {
                                       "        for (int32_t k = 0; k + 1 < K; ++k) {\n            int64_t row = dest_row[n * K + k];\n            if (row < 0 || row >= Q) return OR_EDATA;\n            for (int32_t c = 0; c < d; ++c)\n                dhidden"),
     "weight_sync_wrong_source": ("memcpy(replicas + (int64_t)g * bytes_per_expert, master + (int64_t)e * bytes_per_expert,",
                                  "memcpy(replicas + (int64_t)g * bytes_per_expert, master + (int64_t)g % E * bytes_per_expert,"),
+    "greedy_minimum_without_new_copy": ("if ((int64_t)load_e[e] < (int64_t)min_tokens * (n_copies[e] + 1)) continue;",
+                                        "if ((int64_t)load_e[e] < (int64_t)min_tokens * n_copies[e]) continue;"),
+    "bisect_shed_smallest_master_first": ("if (!done[e] && (best < 0 || L[e] > L[best])) best = e;",
+                                          "if (!done[e] && (best < 0 || L[e] < L[best])) best = e;"),
+    "bisect_no_raise_to_minimum": ("if (s < m) s = m;", ";"),
+    "bisect_no_cut_rule": ("if (rem - piece > 0 && rem - piece < m) piece = rem - m;", ";"),
+    "bisect_receiver_tie_to_higher_r": ("if (rs < 0 || spare[r] > spare[rs]) rs = r;",
+                                        "if (rs < 0 || spare[r] >= spare[rs]) rs = r;"),
+    "bisect_smallest_demand_first": ("if (!done[f] && shed[f] > 0 && (e < 0 || shed[f] > shed[e])) e = f;",
+                                     "if (!done[f] && shed[f] > 0 && (e < 0 || shed[f] < shed[e])) e = f;"),
+    "bisect_mid_rounds_up": ("int64_t mid = lo + (hi - lo) / 2;", "int64_t mid = lo + (hi - lo + 1) / 2;"),
+    "bisect_capacity_rounds_up": ("int rc = or_quota_oracle(R, E, S, load_e, k * Q / DR,",
+                                  "int rc = or_quota_oracle(R, E, S, load_e, (k * Q + DR - 1) / DR,"),
+    "bisect_master_may_always_empty": ("int64_t keep = (allow_zero || L[best] == 0) ? 0 : 1;",
+                                       "int64_t keep = 0;"),
+    "split_without_local_pass": ("int64_t a = s[h] < q[j] ? s[h] : q[j];", "int64_t a = 0;"),
+    "split_remote_descending": ("for (int32_t r = 0; r < R && q[j] > 0; ++r) {",
+                                "for (int32_t r = R - 1; r >= 0 && q[j] > 0; --r) {"),
+    "interleave_rank_major": ("    for (int32_t t = 0; t < T; ++t) {\n        for (int32_t r = 0; r < R; ++r) {",
+                              "    for (int32_t r = 0; r < R; ++r) {\n        for (int32_t t = 0; t < T; ++t) {"),
+    "local_row_without_source_offset": ("dest_row[i] = src_offset[(int64_t)r * P + found] + (int32_t)(o - start);",
+                                        "dest_row[i] = src_offset[found] + (int32_t)(o - start);"),
     "grad_reduce_skips_master": ("out[(int64_t)e * numel + i] = (double)master[(int64_t)e * numel + i];",
                                  "out[(int64_t)e * numel + i] = 0.0;"),
 }
@@ -85,6 +108,15 @@ def run_pins(golden_dir):
         ("wsync", tb.test_weight_sync_definition),
         ("greduce_hand", tb.test_grad_reduce_dyadic_hand_case),
         ("greduce_np", tb.test_grad_reduce_matches_numpy_add_at),
+        ("bisect_hand", lambda: tv.test_bisect_hand_cases(golden_dir)),
+        ("greedy_min_hand", lambda: tv.test_greedy_min_tokens_hand_cases(golden_dir)),
+        ("split_hand", lambda: tv.test_locality_split_hand_cases(golden_dir)),
+        ("bisect_invariants", lambda: tv.test_bisect_invariants_random(8, 64, 2, 1.2, 16)),
+        ("bisect_opt", lambda: tv.test_bisect_bounded_by_exhaustive_opt(2, 4, 1)),
+        ("greedy_min_invariants", lambda: tv.test_greedy_min_tokens_invariants(8, 64, 2, 1.2, 64)),
+        ("split_invariants", lambda: tv.test_locality_split_invariants(8, 128, 64, 4, 2, True, "greedy")),
+        ("split_remote", lambda: tv.test_locality_cuts_remote_pairs_of_a_hot_expert(golden_dir)),
+        ("interleave", lambda: tv.test_interleave_is_prefix_fill_in_token_major_order(8, 128, 64, 4, 2, "greedy")),
     ]
     failed = []
     for name, fn in pins:
