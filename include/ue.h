@@ -81,7 +81,8 @@ typedef struct {
  *   rank_load   [R]   pairs each rank processes under the plan
  *   stats       [4]   {iterations, max rank load before (masters only),
  *                      max rank load after, copies placed on a rank that
- *                      already held a copy of the same expert}
+ *                      already held a copy of the same expert} (ue_plan;
+ *                      ue_plan_ex's capacity planner writes other stats)
  * slot_expert may be NULL when S == 0. */
 typedef struct {
     int32_t* slot_expert;
@@ -95,10 +96,11 @@ typedef struct {
 typedef struct ue_ctx ue_ctx; /* opaque */
 
 /* Create a context for `cfg` on CUDA device `device` (made current) and
- * allocate its scratch once: the error word and the reroute's look-back
- * status words (ceil(Q/8192)*E 64-bit words plus a ticket, a counter and an
- * epoch). Nothing is allocated after this call ("Interface / 1. Initialization": buffers
- * reserved up front, no dynamic allocation at runtime).
+ * allocate its scratch once: the error word, the reroute's look-back status
+ * words (ceil(Q/8192)*E 64-bit words plus a ticket, a counter and an epoch)
+ * and the locality order's two int32 [R][P] tables. Nothing is allocated
+ * after this call ("Interface / 1. Initialization": buffers reserved up
+ * front, no dynamic allocation at runtime).
  * Returns UE_ERR_INVALID_ARG for a null `out` or a config outside the
  * limits (checked before any CUDA call), UE_ERR_UNSUPPORTED if the device
  * is not compute capability 10.x, UE_ERR_CUDA / UE_ERR_NOMEM on failure.
@@ -152,6 +154,56 @@ ue_status ue_count(ue_ctx* ctx, const int32_t* idx, int32_t* load_re,
 ue_status ue_plan(ue_ctx* ctx, const int32_t* load_e, const ue_placement* out,
                   void* stream);
 
+/* Planner choice for ue_plan_ex. "UltraEP" README, "Performance Tuning /
+ * Replication planning" names the knobs followed here (balancing binary
+ * search, its early-stop target and ratio tolerance eps, minimal load per
+ * replica, zero-load masters); the pages give no algorithm, and the rules
+ * below are this library's reading of them. */
+typedef struct {
+    int32_t solver;            /* UE_SOLVER_GREEDY or UE_SOLVER_BISECT          */
+    int32_t min_tokens;        /* minimal pairs per replica: >= 0 for the greedy
+                                  (0: no minimum), >= 1 for the bisection
+                                  (the pages' default is 1024)                  */
+    int32_t eps_inv;           /* bisection: max/mean runs on the grid
+                                  k / eps_inv, 1 <= eps_inv <= 10000 (the pages'
+                                  default eps = 0.01 is eps_inv = 100)          */
+    int32_t threshold;         /* bisection: early-stop ratio in units of
+                                  1/eps_inv, >= 0 (the pages' default 1.0 is
+                                  threshold = eps_inv)                          */
+    int32_t allow_zero_master; /* bisection: 1 lets a master shed all its
+                                  pairs (the pages' default is 0)               */
+} ue_plan_opts;
+
+enum { UE_SOLVER_GREEDY = 0, UE_SOLVER_BISECT = 1 };
+
+/* Replication plan with a choice of planner. Arguments as for ue_plan.
+ *   UE_SOLVER_GREEDY: the ue_plan rule, where only experts with
+ *     L_e >= min_tokens * (c_e + 1) may take a copy (each copy keeps at
+ *     least min_tokens pairs); the greedy also stops when no expert may.
+ *     stats as for ue_plan. min_tokens = 0 gives exactly ue_plan.
+ *   UE_SOLVER_BISECT: a capacity planner. The ratio max/mean runs on the
+ *     grid k/D (D = eps_inv), capacity C(k) = floor(k*Q / (D*R)); H_r is the
+ *     load of rank r's masters. A quota oracle tests C: every rank with
+ *     H_r > C sheds H_r - C pairs from its masters, largest load first (ties
+ *     to the lower e), each giving max(min(left, L_e - keep), m) if
+ *     L_e - keep >= m (keep = 1, or 0 with allow_zero_master or L_e = 0);
+ *     the shed amounts, largest first (ties to the lower e), go in pieces
+ *     to the rank with a free slot and the most spare capacity
+ *     max(0, C - H_r) (ties to the lower r), piece = min(rem, spare), cut to
+ *     rem - m if it would leave 0 < rem - piece < m; a piece below m, no
+ *     receiver or uncovered excess fails C; a replica takes its rank's
+ *     lowest free slot and the piece as quota; the master keeps the rest.
+ *     The search probes k = threshold first and stops if it passes; else it
+ *     bisects between lo = threshold and the smallest k with C(k) >= max H
+ *     while hi - lo > 1 (success moves hi), and the plan is the oracle's
+ *     result at hi. Quotas are then arbitrary per copy (ue_reroute handles
+ *     them). stats = {probes, max rank load before, max rank load after,
+ *     final grid point k}. Runs as a single CTA of 1024 threads that settles
+ *     five levels of the bisection per round.
+ * Invalid options return UE_ERR_INVALID_ARG. */
+ue_status ue_plan_ex(ue_ctx* ctx, const int32_t* load_e, const ue_plan_opts* opts,
+                     const ue_placement* out, void* stream);
+
 /* Logical -> physical routing ("Interface / 2. Forward and backward":
  * reroute expands logical routing to physical replicas).
  *   idx       int32 [N][K] expert ids.
@@ -167,6 +219,55 @@ ue_status ue_plan(ue_ctx* ctx, const int32_t* load_e, const ue_placement* out,
  * UE_ERR_DEVICE_BOUNDS. */
 ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
                      int32_t* phys_slot, int32_t* dest_row, void* stream);
+
+enum { UE_ORDER_PREFIX = 0, UE_ORDER_INTERLEAVE = 1 };
+
+/* ue_reroute with a choice of pair order ("UltraEP" README, "Performance
+ * Tuning / Replication planning": interleave the token order so that the
+ * dispatch that follows does not congest; the reading here is a token-major
+ * order across the source ranks).
+ *   order UE_ORDER_PREFIX:     exactly ue_reroute (global order (r, t, k)).
+ *   order UE_ORDER_INTERLEAVE: the copies are filled by prefix sum with the
+ *     pairs taken in the order (t, r, k): token 0 of every rank, then token
+ *     1 of every rank, ...; each copy then receives a range of token
+ *     positions from every source rank. Rows of a slot hold its pairs in
+ *     that order. phys_slot and dest_row are still indexed by pair i.
+ * Other arguments and errors as for ue_reroute. */
+ue_status ue_reroute_ex(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
+                        int32_t order, int32_t* phys_slot, int32_t* dest_row,
+                        void* stream);
+
+/* Locality-aware split of every copy's quota over the source ranks
+ * ("UltraEP" README, "Performance Tuning / Replication planning": a
+ * per-rank quota decomposition that cuts remote traffic; the reading here
+ * is own-rank first). For expert e with copies j in copy order (master, then
+ * replicas by ascending g) on host ranks h_j with quotas q_j, and the source
+ * loads s_r = load_re[r][e]:
+ *   local pass:  every copy j, in copy order, first takes min(s_{h_j}, q_j)
+ *                pairs from its own host rank;
+ *   remote pass: every copy j, in copy order, fills the rest of its quota
+ *                from the source ranks in ascending r.
+ *   load_re    int32 [R][E] from ue_count for the same idx as the plan.
+ *   plan       a placement (slot_expert, slot_quota, slot_offset are read).
+ *   src_quota  int32 [R][P]: pairs of source rank r assigned to slot p.
+ *   src_offset int32 [R][P]: dispatch row of the first of them (a slot
+ *              holds its pairs by source rank, then in the source's order).
+ * An expert whose source loads do not sum to its quotas, or a slot_expert
+ * entry >= E, sets UE_ERR_DEVICE_BOUNDS. */
+ue_status ue_locality_split(ue_ctx* ctx, const int32_t* load_re, const ue_placement* plan,
+                            int32_t* src_quota, int32_t* src_offset, void* stream);
+
+/* Reroute under the locality-aware split: source rank r hands its pairs of
+ * expert e, in its own order (t, k), to e's copies in copy order,
+ * src_quota[r][p] pairs each, at rows src_offset[r][p], src_offset[r][p]+1,
+ * ... The arrays are those ue_locality_split wrote for this plan and load_re
+ * (and load_re is ue_count's for idx). Uses the context's [R][P] tables,
+ * rebuilt on every call. Other arguments and errors as for ue_reroute; a
+ * pair outside its source rank's split sets UE_ERR_DEVICE_BOUNDS. */
+ue_status ue_reroute_local(ue_ctx* ctx, const int32_t* idx, const int32_t* load_re,
+                           const ue_placement* plan, const int32_t* src_quota,
+                           const int32_t* src_offset, int32_t* phys_slot,
+                           int32_t* dest_row, void* stream);
 
 /* Token dispatch into per-slot contiguous buffers ("Interface / 2. Forward
  * and backward": dispatch(hidden, probs, routing_map), here a single-GPU

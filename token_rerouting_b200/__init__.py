@@ -8,7 +8,9 @@ streams; tensors are passed by ``data_ptr()``. There is no CPU fallback: if
 
 The functions carry the C names: ``ue_init``, ``ue_gate_topk``, ``ue_count``,
 ``ue_plan``, ``ue_reroute``, ``ue_permute``, ``ue_combine``, ``ue_get_error``,
-``ue_destroy`` (see include/ue.h for the contract of each).
+``ue_destroy``, the planner variants ``ue_plan_ex``, ``ue_reroute_ex``,
+``ue_locality_split``, ``ue_reroute_local``, and the rows beside the forward
+path (see include/ue.h for the contract of each).
 """
 from __future__ import annotations
 
@@ -32,7 +34,8 @@ UE_ERR_DEVICE_BOUNDS, UE_ERR_TIMEOUT, UE_ERR_UNSUPPORTED = 4, 5, 6
 
 # every symbol include/ue.h declares
 EXPORTS = ("ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count",
-           "ue_plan", "ue_reroute", "ue_permute", "ue_combine", "ue_combine_backward",
+           "ue_plan", "ue_plan_ex", "ue_reroute", "ue_reroute_ex", "ue_locality_split",
+           "ue_reroute_local", "ue_permute", "ue_combine", "ue_combine_backward",
            "ue_permute_backward", "ue_weight_sync", "ue_grad_reduce", "ue_reroute_noalloc",
            "ue_debug_set_lookback_limit", "ue_debug_drop_first_publish")
 
@@ -52,6 +55,27 @@ class ue_placement(ctypes.Structure):
     _fields_ = [("slot_expert", ctypes.c_void_p), ("n_copies", ctypes.c_void_p),
                 ("slot_quota", ctypes.c_void_p), ("slot_offset", ctypes.c_void_p),
                 ("rank_load", ctypes.c_void_p), ("stats", ctypes.c_void_p)]
+
+
+UE_SOLVER_GREEDY, UE_SOLVER_BISECT = 0, 1
+UE_ORDER_PREFIX, UE_ORDER_INTERLEAVE = 0, 1
+
+
+class ue_plan_opts(ctypes.Structure):
+    _fields_ = [("solver", ctypes.c_int32), ("min_tokens", ctypes.c_int32),
+                ("eps_inv", ctypes.c_int32), ("threshold", ctypes.c_int32),
+                ("allow_zero_master", ctypes.c_int32)]
+
+
+def plan_opts(solver: int = UE_SOLVER_GREEDY, min_tokens: int | None = None, eps_inv: int = 100,
+              threshold: int | None = None, allow_zero_master: bool = False) -> ue_plan_opts:
+    """Planner options; the defaults are the pages' (minimum 1024 pairs per
+    replica and eps 0.01, early stop at 1.0, for the bisection; no minimum for
+    the greedy)."""
+    if min_tokens is None:
+        min_tokens = 1024 if solver == UE_SOLVER_BISECT else 0
+    return ue_plan_opts(solver, min_tokens, eps_inv,
+                        eps_inv if threshold is None else threshold, int(bool(allow_zero_master)))
 
 
 _lib = None
@@ -74,7 +98,13 @@ def load_library(path: str | None = None):
     lib.ue_gate_topk.argtypes = [vp, vp, vp, vp, vp]
     lib.ue_count.argtypes = [vp, vp, vp, vp, vp]
     lib.ue_plan.argtypes = [vp, vp, ctypes.POINTER(ue_placement), vp]
+    lib.ue_plan_ex.argtypes = [vp, vp, ctypes.POINTER(ue_plan_opts), ctypes.POINTER(ue_placement),
+                               vp]
     lib.ue_reroute.argtypes = [vp, vp, ctypes.POINTER(ue_placement), vp, vp, vp]
+    lib.ue_reroute_ex.argtypes = [vp, vp, ctypes.POINTER(ue_placement), i32, vp, vp, vp]
+    lib.ue_locality_split.argtypes = [vp, vp, ctypes.POINTER(ue_placement), vp, vp, vp]
+    lib.ue_reroute_local.argtypes = [vp, vp, vp, ctypes.POINTER(ue_placement), vp, vp, vp, vp,
+                                     vp]
     lib.ue_permute.argtypes = [vp, vp, vp, vp, vp]
     lib.ue_combine.argtypes = [vp, vp, vp, vp, vp, vp]
     lib.ue_combine_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
@@ -157,6 +187,31 @@ def ue_plan(ctx, load_e, plan: ue_placement, stream=None):
                                           _stream(stream)))
 
 
+def ue_plan_ex(ctx, load_e, opts: ue_plan_opts, plan: ue_placement, stream=None):
+    _ok("ue_plan_ex", load_library().ue_plan_ex(ctx, _ptr(load_e), ctypes.byref(opts),
+                                                ctypes.byref(plan), _stream(stream)))
+
+
+def ue_reroute_ex(ctx, idx, plan: ue_placement, order: int, phys_slot, dest_row, stream=None):
+    _ok("ue_reroute_ex", load_library().ue_reroute_ex(ctx, _ptr(idx), ctypes.byref(plan), order,
+                                                      _ptr(phys_slot), _ptr(dest_row),
+                                                      _stream(stream)))
+
+
+def ue_locality_split(ctx, load_re, plan: ue_placement, src_quota, src_offset, stream=None):
+    _ok("ue_locality_split",
+        load_library().ue_locality_split(ctx, _ptr(load_re), ctypes.byref(plan), _ptr(src_quota),
+                                         _ptr(src_offset), _stream(stream)))
+
+
+def ue_reroute_local(ctx, idx, load_re, plan: ue_placement, src_quota, src_offset, phys_slot,
+                     dest_row, stream=None):
+    _ok("ue_reroute_local",
+        load_library().ue_reroute_local(ctx, _ptr(idx), _ptr(load_re), ctypes.byref(plan),
+                                        _ptr(src_quota), _ptr(src_offset), _ptr(phys_slot),
+                                        _ptr(dest_row), _stream(stream)))
+
+
 def ue_reroute(ctx, idx, plan: ue_placement, phys_slot, dest_row, stream=None):
     _ok("ue_reroute", load_library().ue_reroute(ctx, _ptr(idx), ctypes.byref(plan),
                                                 _ptr(phys_slot), _ptr(dest_row),
@@ -221,6 +276,9 @@ def ue_debug_drop_first_publish(ctx, enable: bool):
 from .layer import Layer  # noqa: E402  (buffers + one call per step)
 
 __all__ = ["ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count", "ue_plan",
+           "ue_plan_ex", "ue_reroute_ex", "ue_locality_split", "ue_reroute_local",
+           "ue_plan_opts", "plan_opts", "UE_SOLVER_GREEDY", "UE_SOLVER_BISECT",
+           "UE_ORDER_PREFIX", "UE_ORDER_INTERLEAVE",
            "ue_reroute", "ue_permute", "ue_combine", "ue_combine_backward",
            "ue_permute_backward", "ue_weight_sync", "ue_grad_reduce", "ue_reroute_noalloc",
            "ue_debug_set_lookback_limit",

@@ -13,6 +13,10 @@
 // 50*R*max_r load_r <= 51*Q or no slot is free; else e* = argmax L_e/c_e
 // (exact, ties to the lowest e), r* = argmin load_r over ranks with a free
 // slot (ties to the lowest r); the copy goes into r*'s lowest free slot.
+// With a minimum of m pairs per replica ("UltraEP" README, "Performance
+// Tuning / Replication planning": minimal load allocated to a replica) only
+// experts with L_e >= m*(c_e + 1) may take a copy, and the greedy also stops
+// when none may; m = 0 lets every expert grow.
 //
 // Design (B200): the greedy is serial, so its speed is the latency of one
 // iteration. The choice of e* depends only on the copy counts, never on the
@@ -27,7 +31,8 @@
 //    preserving (two different ratios differ by more than 1/66049, i.e. by
 //    more than 250 after scaling; equal ratios give equal keys). The expert id
 //    sits below the key, so the argmax with ties to the lowest e is two warp
-//    `redux` max reductions.
+//    `redux` max reductions. An expert that may not grow has key 0; when
+//    every key is 0 the expert side pushes an end marker (e = -1).
 //  - warp 0 (rank side) keeps the rank loads and the redundant slots in
 //    registers (lane l owns ranks l, l+32, ... and their slots, so every
 //    load change lands in the lane that owns the rank). Per iteration: the
@@ -64,16 +69,24 @@ __device__ __forceinline__ unsigned long long packed_key(unsigned L, unsigned c,
     return (k << 9) | (unsigned long long)(511 - e);
 }
 
+// may an expert with load L and c copies take copy c+1 and keep at least m
+// pairs on each?
+__device__ __forceinline__ bool may_grow(unsigned L, unsigned c, unsigned m)
+{
+    return (unsigned long long)m * (c + 1u) <= (unsigned long long)L;
+}
+
 struct Pick {
-    int e;         // expert receiving the copy
+    int e;         // expert receiving the copy (-1: no expert may grow)
     unsigned qb;   // floor(L / c) with the new copy count c
     unsigned rem;  // L mod c
     unsigned dq0;  // master quota change: ceil(L/c) - ceil(L/(c-1)) (two's complement)
 };
 
 template <int NJE, int NJR, int SM>
-__global__ void __launch_bounds__(kPlanThreads)
-plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placement out, int* err)
+__global__ void __launch_bounds__(kPlanThreads, 1)
+plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned min_tokens,
+            ue_placement out, int* err)
 {
     __shared__ unsigned long long sRecip[kMaxG + 2];  // ceil(2^64 / c), c = 2 .. G+1
     __shared__ int sL[kMaxE];       // exact load per expert
@@ -129,7 +142,8 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
             const int e = lane + 32 * j;
             Lr[j] = e < E ? (unsigned)sL[e] : 0u;
             cr[j] = 1u;
-            key[j] = e < E ? packed_key(Lr[j], 1u, e, sRecip) : 0ull;
+            key[j] = (e < E && may_grow(Lr[j], 1u, min_tokens)) ? packed_key(Lr[j], 1u, e, sRecip)
+                                                                 : 0ull;
         }
         for (int t = 0; t < G; ++t) {
             if (__any_sync(kFull, sDone != 0)) break;
@@ -138,6 +152,15 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
             for (int j = 0; j < NJE; ++j) best = key[j] > best ? key[j] : best;
             const unsigned hi = __reduce_max_sync(kFull, (unsigned)(best >> 32));
             const unsigned lo = __reduce_max_sync(kFull, (unsigned)(best >> 32) == hi ? (unsigned)best : 0u);
+            if (hi == 0u && lo == 0u) {
+                // no expert may take another copy: end marker
+                if (lane == 0) {
+                    sPick[t] = Pick{-1, 0u, 0u, 0u};
+                    __threadfence_block();
+                    sReady[t] = 1;
+                }
+                break;
+            }
             const int estar = 511 - (int)(lo & 511u);
             const int ej = estar >> 5;
             unsigned Le = 0u, ce = 0u;
@@ -149,7 +172,8 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
                 }
             Le = __shfl_sync(kFull, Le, estar & 31);
             ce = __shfl_sync(kFull, ce, estar & 31) + 1u;
-            const unsigned long long nk = packed_key(Le, ce, estar, sRecip);
+            const unsigned long long nk =
+                may_grow(Le, ce, min_tokens) ? packed_key(Le, ce, estar, sRecip) : 0ull;
             if (lane == (estar & 31)) {
 #pragma unroll
                 for (int j = 0; j < NJE; ++j)
@@ -215,6 +239,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
             }
             __threadfence_block();
             const Pick pk = sPick[iters];
+            if (pk.e < 0) break;  // no expert may take another copy
             const int estar = pk.e;
             const int rj = rstar >> 5;
             const bool rown = lane == (rstar & 31);
@@ -355,34 +380,35 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, ue_placemen
 }
 
 template <int NJE, int NJR>
-cudaError_t launch_s(const Sizes& z, const int32_t* load_e, const ue_placement& out, int* err,
-                     cudaStream_t st)
+cudaError_t launch_s(const Sizes& z, const int32_t* load_e, unsigned m, const ue_placement& out,
+                     int* err, cudaStream_t st)
 {
     if (z.S <= 2)
-        plan_kernel<NJE, NJR, 2><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, out, err);
+        plan_kernel<NJE, NJR, 2><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, m, out, err);
     else
-        plan_kernel<NJE, NJR, 8><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, out, err);
+        plan_kernel<NJE, NJR, 8><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, m, out, err);
     return cudaGetLastError();
 }
 
 template <int NJE>
-cudaError_t launch_r(const Sizes& z, const int32_t* load_e, const ue_placement& out, int* err,
-                     cudaStream_t st)
+cudaError_t launch_r(const Sizes& z, const int32_t* load_e, unsigned m, const ue_placement& out,
+                     int* err, cudaStream_t st)
 {
-    if (z.R <= 32) return launch_s<NJE, 1>(z, load_e, out, err, st);
-    if (z.R <= 64) return launch_s<NJE, 2>(z, load_e, out, err, st);
-    return launch_s<NJE, 4>(z, load_e, out, err, st);
+    if (z.R <= 32) return launch_s<NJE, 1>(z, load_e, m, out, err, st);
+    if (z.R <= 64) return launch_s<NJE, 2>(z, load_e, m, out, err, st);
+    return launch_s<NJE, 4>(z, load_e, m, out, err, st);
 }
 
 }  // namespace
 
-cudaError_t launch_plan(const Sizes& z, const int32_t* load_e,
+cudaError_t launch_plan(const Sizes& z, const int32_t* load_e, int min_tokens,
                         const ue_placement& out, int* err, cudaStream_t st)
 {
-    if (z.E <= 32) return launch_r<1>(z, load_e, out, err, st);
-    if (z.E <= 64) return launch_r<2>(z, load_e, out, err, st);
-    if (z.E <= 128) return launch_r<4>(z, load_e, out, err, st);
-    return launch_r<8>(z, load_e, out, err, st);
+    const unsigned m = (unsigned)min_tokens;
+    if (z.E <= 32) return launch_r<1>(z, load_e, m, out, err, st);
+    if (z.E <= 64) return launch_r<2>(z, load_e, m, out, err, st);
+    if (z.E <= 128) return launch_r<4>(z, load_e, m, out, err, st);
+    return launch_r<8>(z, load_e, m, out, err, st);
 }
 
 }  // namespace ue

@@ -18,6 +18,8 @@ struct ue_ctx {
     int* d_err;             // [2] error code, detail
     unsigned long long* d_status;  // [tiles][E] reroute look-back words
     uint32_t* d_sync;       // [4] reroute ticket, finished CTAs, epoch
+    int32_t* d_first;       // [R][P] locality order: first occurrence index
+    int32_t* d_rowb;        // [R][P] locality order: row base
     int64_t tiles;
     int64_t spin_limit;
     int drop_first;
@@ -95,19 +97,25 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
     ctx->drop_first = 0;
 
     if (ue::plan_permute_shape(ctx->z, ctx->num_sms, &ctx->perm) != cudaSuccess ||
-        ue::plan_combine_shape(ctx->z, ctx->num_sms, &ctx->comb) != cudaSuccess) {
+        ue::plan_combine_shape(ctx->z, ctx->num_sms, &ctx->comb) != cudaSuccess ||
+        ue::plan_bisect_setup(ctx->z) != cudaSuccess) {
         delete ctx;
         cudaGetLastError();
         return UE_ERR_CUDA;
     }
 
     const size_t status_words = (size_t)std::max<int64_t>(ctx->tiles, 1) * ctx->z.E;
+    const size_t table_words = (size_t)ctx->z.R * ctx->z.P;
     if (cudaMalloc(&ctx->d_err, 2 * sizeof(int)) != cudaSuccess ||
         cudaMalloc(&ctx->d_status, status_words * sizeof(unsigned long long)) != cudaSuccess ||
-        cudaMalloc(&ctx->d_sync, 4 * sizeof(uint32_t)) != cudaSuccess) {
+        cudaMalloc(&ctx->d_sync, 4 * sizeof(uint32_t)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_first, table_words * sizeof(int32_t)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_rowb, table_words * sizeof(int32_t)) != cudaSuccess) {
         cudaFree(ctx->d_err);
         cudaFree(ctx->d_status);
         cudaFree(ctx->d_sync);
+        cudaFree(ctx->d_first);
+        cudaFree(ctx->d_rowb);
         delete ctx;
         cudaGetLastError();
         return UE_ERR_NOMEM;
@@ -119,6 +127,8 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
         cudaFree(ctx->d_err);
         cudaFree(ctx->d_status);
         cudaFree(ctx->d_sync);
+        cudaFree(ctx->d_first);
+        cudaFree(ctx->d_rowb);
         delete ctx;
         return UE_ERR_CUDA;
     }
@@ -136,6 +146,8 @@ ue_status ue_destroy(ue_ctx* ctx)
     cudaFree(ctx->d_err);
     cudaFree(ctx->d_status);
     cudaFree(ctx->d_sync);
+    cudaFree(ctx->d_first);
+    cudaFree(ctx->d_rowb);
     ctx->magic = 0;
     delete ctx;
     return st;
@@ -179,7 +191,28 @@ ue_status ue_plan(ue_ctx* ctx, const int32_t* load_e, const ue_placement* out, v
     if (!ctx_ok(ctx) || !aligned(load_e, 4) || !placement_ok(ctx, out))
         return UE_ERR_INVALID_ARG;
     if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
-    return from_cuda(ue::launch_plan(ctx->z, load_e, *out, ctx->d_err, as_stream(stream)));
+    return from_cuda(ue::launch_plan(ctx->z, load_e, 0, *out, ctx->d_err, as_stream(stream)));
+}
+
+ue_status ue_plan_ex(ue_ctx* ctx, const int32_t* load_e, const ue_plan_opts* opts,
+                     const ue_placement* out, void* stream)
+{
+    if (!ctx_ok(ctx) || opts == nullptr || !aligned(load_e, 4) || !placement_ok(ctx, out))
+        return UE_ERR_INVALID_ARG;
+    const ue_plan_opts o = *opts;
+    if (o.solver == UE_SOLVER_GREEDY) {
+        if (o.min_tokens < 0) return UE_ERR_INVALID_ARG;
+        if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+        return from_cuda(ue::launch_plan(ctx->z, load_e, o.min_tokens, *out, ctx->d_err,
+                                         as_stream(stream)));
+    }
+    if (o.solver != UE_SOLVER_BISECT || o.min_tokens < 1 || o.eps_inv < 1 || o.eps_inv > 10000 ||
+        o.threshold < 0 || (o.allow_zero_master != 0 && o.allow_zero_master != 1))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_plan_bisect(ctx->z, load_e, o.eps_inv, o.threshold, o.min_tokens,
+                                            o.allow_zero_master, *out, ctx->d_err,
+                                            as_stream(stream)));
 }
 
 ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
@@ -192,6 +225,46 @@ ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
     return from_cuda(ue::launch_reroute(ctx->z, idx, *plan, phys_slot, dest_row, ctx->d_status,
                                         ctx->d_sync, ctx->spin_limit, ctx->drop_first,
                                         ctx->d_err, as_stream(stream)));
+}
+
+ue_status ue_reroute_ex(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan, int32_t order,
+                        int32_t* phys_slot, int32_t* dest_row, void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(idx, 4) || !placement_ok(ctx, plan) ||
+        !aligned(phys_slot, 4) || !aligned(dest_row, 4) ||
+        (order != UE_ORDER_PREFIX && order != UE_ORDER_INTERLEAVE))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_reroute_order(ctx->z, idx, *plan, order, phys_slot, dest_row,
+                                              ctx->d_status, ctx->d_sync, ctx->spin_limit,
+                                              ctx->drop_first, ctx->d_err, as_stream(stream)));
+}
+
+ue_status ue_locality_split(ue_ctx* ctx, const int32_t* load_re, const ue_placement* plan,
+                            int32_t* src_quota, int32_t* src_offset, void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(load_re, 4) || !placement_ok(ctx, plan) ||
+        !aligned(src_quota, 4) || !aligned(src_offset, 4))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_locality_split(ctx->z, load_re, *plan, src_quota, src_offset,
+                                               ctx->d_err, as_stream(stream)));
+}
+
+ue_status ue_reroute_local(ue_ctx* ctx, const int32_t* idx, const int32_t* load_re,
+                           const ue_placement* plan, const int32_t* src_quota,
+                           const int32_t* src_offset, int32_t* phys_slot, int32_t* dest_row,
+                           void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(idx, 4) || !aligned(load_re, 4) || !placement_ok(ctx, plan) ||
+        !aligned(src_quota, 4) || !aligned(src_offset, 4) || !aligned(phys_slot, 4) ||
+        !aligned(dest_row, 4))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    return from_cuda(ue::launch_reroute_local(ctx->z, idx, load_re, *plan, src_quota, src_offset,
+                                              ctx->d_first, ctx->d_rowb, phys_slot, dest_row,
+                                              ctx->d_status, ctx->d_sync, ctx->spin_limit,
+                                              ctx->drop_first, ctx->d_err, as_stream(stream)));
 }
 
 ue_status ue_permute(ue_ctx* ctx, const uint16_t* hidden, const int32_t* dest_row,

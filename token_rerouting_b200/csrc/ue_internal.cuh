@@ -69,8 +69,15 @@ cudaError_t launch_gate_topk(const Sizes& z, const float* logits, int32_t* idx,
                              float* w, int grid, cudaStream_t st);
 cudaError_t launch_count(const Sizes& z, const int32_t* idx, int32_t* load_re,
                          int32_t* load_e, int* err, cudaStream_t st);
-cudaError_t launch_plan(const Sizes& z, const int32_t* load_e,
+// greedy plan; min_tokens = 0: every expert may take a copy
+cudaError_t launch_plan(const Sizes& z, const int32_t* load_e, int min_tokens,
                         const ue_placement& out, int* err, cudaStream_t st);
+// capacity planner (bisection); plan_bisect_setup sets the kernel's shared
+// memory limit once per context, outside any stream capture
+cudaError_t plan_bisect_setup(const Sizes& z);
+cudaError_t launch_plan_bisect(const Sizes& z, const int32_t* load_e, int eps_inv, int threshold,
+                               int min_tokens, int allow_zero, const ue_placement& out, int* err,
+                               cudaStream_t st);
 // Reroute scratch: tiles*E 64-bit status words and sync[0..2] = {tile
 // ticket, finished CTAs, launch epoch}, zeroed once; each launch leaves them
 // ready for the next one (the last CTA resets the ticket and the counter and
@@ -80,6 +87,21 @@ cudaError_t launch_reroute(const Sizes& z, const int32_t* idx,
                            int32_t* dest_row, unsigned long long* status,
                            uint32_t* sync, int64_t spin_limit,
                            int drop_first, int* err, cudaStream_t st);
+// order: 0 global (r, t, k), 1 interleaved (t, r, k)
+cudaError_t launch_reroute_order(const Sizes& z, const int32_t* idx, const ue_placement& plan,
+                                 int order, int32_t* phys_slot, int32_t* dest_row,
+                                 unsigned long long* status, uint32_t* sync, int64_t spin_limit,
+                                 int drop_first, int* err, cudaStream_t st);
+// locality order: builds the [R][P] tables `first` and `rowb`, then reroutes
+cudaError_t launch_reroute_local(const Sizes& z, const int32_t* idx, const int32_t* load_re,
+                                 const ue_placement& plan, const int32_t* src_quota,
+                                 const int32_t* src_offset, int32_t* first, int32_t* rowb,
+                                 int32_t* phys_slot, int32_t* dest_row,
+                                 unsigned long long* status, uint32_t* sync, int64_t spin_limit,
+                                 int drop_first, int* err, cudaStream_t st);
+cudaError_t launch_locality_split(const Sizes& z, const int32_t* load_re,
+                                  const ue_placement& plan, int32_t* src_quota,
+                                  int32_t* src_offset, int* err, cudaStream_t st);
 // Launch shapes of the row kernels, fixed once per context (ue_init) so that
 // a call only enqueues work (nothing else touches the runtime, which keeps
 // the calls safe under stream capture).

@@ -10,7 +10,8 @@ dispatch (permute) -> experts (outside; identity here unless ``y`` is given)
 from __future__ import annotations
 
 from . import (make_config, placement, ue_combine, ue_count, ue_destroy, ue_gate_topk,
-               ue_get_error, ue_init, ue_permute, ue_plan, ue_reroute)
+               ue_get_error, ue_init, ue_locality_split, ue_permute, ue_plan, ue_plan_ex,
+               ue_reroute, ue_reroute_ex, ue_reroute_local)
 
 
 class Layer:
@@ -44,6 +45,9 @@ class Layer:
                               self.slot_quota, self.slot_offset, self.rank_load, self.stats)
         self.phys_slot = torch.empty((self.N, K), dtype=i32, device=dev)
         self.dest_row = torch.empty((self.N, K), dtype=i32, device=dev)
+        # locality-aware split of the quotas over the source ranks
+        self.src_quota = torch.empty((R, self.P), dtype=i32, device=dev)
+        self.src_offset = torch.empty((R, self.P), dtype=i32, device=dev)
         self.with_rows = with_rows
         if with_rows:
             self.hidden = torch.empty((self.N, d), dtype=torch.bfloat16, device=dev)
@@ -62,6 +66,22 @@ class Layer:
 
     def reroute(self, stream=None):
         ue_reroute(self.ctx, self.idx, self.plan, self.phys_slot, self.dest_row, stream)
+
+    # -- planner variants ("Performance Tuning / Replication planning") -----
+    def plan_ex(self, opts, stream=None):
+        """ue_plan_ex with a ue_plan_opts (see token_rerouting_b200.plan_opts)."""
+        ue_plan_ex(self.ctx, self.load_e, opts, self.plan, stream)
+
+    def reroute_ex(self, order, stream=None):
+        ue_reroute_ex(self.ctx, self.idx, self.plan, order, self.phys_slot, self.dest_row, stream)
+
+    def locality_split(self, stream=None):
+        ue_locality_split(self.ctx, self.load_re, self.plan, self.src_quota, self.src_offset,
+                          stream)
+
+    def reroute_local(self, stream=None):
+        ue_reroute_local(self.ctx, self.idx, self.load_re, self.plan, self.src_quota,
+                         self.src_offset, self.phys_slot, self.dest_row, stream)
 
     def permute(self, stream=None):
         ue_permute(self.ctx, self.hidden, self.dest_row, self.dispatch, stream)
