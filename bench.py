@@ -41,34 +41,18 @@ FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
 # one ncu --set full capture of the same workload at 512 tokens per rank,
-# scaled by 8 to the full 4096 tokens per rank (every kernel's traffic grows
-# in proportion to the tokens), with the SHA-256 prefix of the kernel source
-# it was taken on; a kernel changed since then reports null.
+# scaled by 8 to the full 4096 tokens per rank (the traffic of every kernel
+# but the plan grows in proportion to the tokens; the plan's, a few KB of
+# loads and outputs, does not and is taken as measured), with the SHA-256
+# prefix of the kernel source it was taken on; a kernel changed since then
+# reports null.
 TRAFFIC = {
-    "gate_topk": {
-        "bytes_per_launch": 134512000,
-        "source_sha": "eecff9157bbb7231"
-    },
-    "count": {
-        "bytes_per_launch": 8736000,
-        "source_sha": "27ba6f511329134d"
-    },
-    "plan": {
-        "bytes_per_launch": 224000,
-        "source_sha": "d88f84a3510d0295"
-    },
-    "reroute": {
-        "bytes_per_launch": 8888000,
-        "source_sha": "897786029bfb7b7a"
-    },
-    "permute": {
-        "bytes_per_launch": 18877864000,
-        "source_sha": "07222823ab0e9db7"
-    },
-    "combine": {
-        "bytes_per_launch": 21233264000,
-        "source_sha": "c91a07d4eae7b00b"
-    },
+    "gate_topk": {"bytes_per_launch": 134720000, "source_sha": "2cf60b87ff02f365"},
+    "count": {"bytes_per_launch": 8824000, "source_sha": "df378f26704dc1a3"},
+    "plan": {"bytes_per_launch": 25000, "source_sha": "594eef62c20fb78b"},
+    "reroute": {"bytes_per_launch": 8968000, "source_sha": "f685d38239dc3908"},
+    "permute": {"bytes_per_launch": 18881304000, "source_sha": "07222823ab0e9db7"},
+    "combine": {"bytes_per_launch": 21247792000, "source_sha": "0ebcc3caa2094612"},
 }
 
 
@@ -427,6 +411,97 @@ def run_row(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_planner(args, w):
+    """Planner variants ("UltraEP" README, "Performance Tuning / Replication
+    planning") on the pages' runtime-test layer (EP64, 256 experts, 4 master +
+    2 redundant per rank, top-8, 8k tokens per rank) at its three initial
+    imbalances, or on one given workload: balance reached, replicas, and the
+    device time of every plan and reroute variant. One JSON line per layer
+    instance. The pages' own numbers (one GPU of 64, the load all-gather
+    included) are quoted beside ours for context only: here one GPU plans and
+    reroutes for all 64 ranks."""
+    import numpy as np
+    import torch
+
+    import synth
+    import token_rerouting_b200 as ue
+    from token_rerouting_b200 import build as ue_build
+
+    ue_build.build()
+    dev = torch.device("cuda", 0)
+    st = torch.cuda.current_stream(dev)
+    pages = {1.51: dict(final=1.01, replicas="4 / 38", update_placement_ms=0.067, reroute_ms=0.039),
+             2.01: dict(final=1.01, replicas="5 / 46", update_placement_ms=0.072, reroute_ms=0.037),
+             3.03: dict(final=1.01, replicas="6 / 51", update_placement_ms=0.078, reroute_ms=0.036)}
+    if w.name.startswith("pages_"):
+        instances = [(t, synth.ALPHA_PAGES[i]) for i, t in enumerate((1.51, 2.01, 3.03))]
+    else:
+        instances = [(None, None)]
+    L = ue.Layer(w.R, w.T, w.E, w.K, w.S, 8, device=0, with_rows=False)
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(args.steps):
+            fn()
+        b.record(st)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / args.steps * 1e3  # us
+
+    M, S = w.M, w.S
+    host_of_slot = np.arange(w.P) // (M + S)
+    src_of_pair = np.arange(w.Q) // (w.T * w.K)
+    mean = w.Q / w.R
+
+    def summary(plan):
+        se = plan["slot_expert"]
+        nc = plan["n_copies"]
+        return dict(max_over_mean=float(plan["rank_load"].max() / mean),
+                    replicas=int((se >= 0).sum()), max_replicas_per_expert=int(nc.max() - 1),
+                    stats=plan["stats"].tolist())
+
+    solvers = {"greedy": ue.plan_opts(ue.UE_SOLVER_GREEDY),
+               "greedy_min1024": ue.plan_opts(ue.UE_SOLVER_GREEDY, min_tokens=1024),
+               "bisect": ue.plan_opts(ue.UE_SOLVER_BISECT)}
+    for target, alpha in instances:
+        L.logits.copy_(torch.from_numpy(synth.logits(w, alpha=alpha)))
+        L.gate()
+        L.count()
+        torch.cuda.synchronize(dev)
+        load_e = L.load_e.cpu().numpy()
+        before = float(load_e.reshape(w.R, M).sum(axis=1).max() / mean)
+        res = {}
+        for name, opts in solvers.items():
+            us = timed(lambda: L.plan_ex(opts, st))
+            res[name] = dict(plan_us=us, **summary(L.plan_arrays()))
+            # reroutes under this plan
+            res[name]["reroute_us"] = timed(lambda: L.reroute(st))
+            torch.cuda.synchronize(dev)
+            phys = L.phys_slot.cpu().numpy().ravel()
+            res[name]["remote_pairs_prefix"] = int((host_of_slot[phys] != src_of_pair).sum())
+            res[name]["reroute_interleave_us"] = timed(lambda: L.reroute_ex(ue.UE_ORDER_INTERLEAVE, st))
+            res[name]["locality_split_us"] = timed(lambda: L.locality_split(st))
+            res[name]["reroute_local_us"] = timed(lambda: L.reroute_local(st))
+            torch.cuda.synchronize(dev)
+            sq = L.src_quota.cpu().numpy()
+            res[name]["remote_pairs_local"] = int(sum(sq[r, host_of_slot != r].sum()
+                                                     for r in range(w.R)))
+        rc = L.error()
+        if rc != 0:
+            raise SystemExit(f"device error: {rc}")
+        line = {"row": "planner", "config": dict(workload=w.name, R=w.R, T=w.T, E=w.E, K=w.K,
+                                                   S=w.S, pairs=w.Q, alpha=alpha,
+                                                   target_imbalance=target),
+                "steps": args.steps, "imbalance_before": before, "solvers": res}
+        if target is not None:
+            line["pages_context"] = pages[target]
+        print(json.dumps(line), flush=True)
+    L.close()
+
+
 def synth_logits(w):
     import synth
     return synth.logits(w)
@@ -439,7 +514,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ue", "reference"), default="ue")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", default=None,
+                    help=f"default {DEFAULT_WORKLOAD} (pages_ep64_e256_t8k for --row planner)")
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="shrink T (profiling runs on a small case)")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -447,14 +523,17 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="the 48 x 8 non-stationary sweep, CUDA-graph captured")
-    ap.add_argument("--row", choices=("backward", "weight_sync", "grad_reduce"), default=None,
-                    help="measure one of the rows beside the forward path")
+    ap.add_argument("--row", choices=("backward", "weight_sync", "grad_reduce", "planner"),
+                    default=None, help="measure one of the rows beside the forward path "
+                    "(planner: the planner variants, on pages_ep64_e256_t8k by default)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     import dataclasses
 
     import synth
+    if args.workload is None:
+        args.workload = "pages_ep64_e256_t8k" if args.row == "planner" else DEFAULT_WORKLOAD
     w = synth.WORKLOADS[args.workload]
     if args.tokens_per_rank:
         w = dataclasses.replace(w, T=args.tokens_per_rank, name=f"{w.name}_t{args.tokens_per_rank}")
@@ -463,6 +542,9 @@ def main():
         return
     if args.sweep:
         run_sweep(args)
+        return
+    if args.row == "planner":
+        run_planner(args, w)
         return
     if args.row:
         run_row(args, w)

@@ -36,9 +36,14 @@ CHUNK = 1 << 22
 #                DeepSeek-V3-shaped layer, each drawing 8% of all pairs.
 #   HOT_BOOST_30PCT: boost that sends 30% of tokens to one expert in the
 #                sweep's single-expert case.
+#   ALPHA_PAGES: scales of the s=1.0 Zipf bias that give the EP64, 256-expert
+#                layer of the pages' runtime test ("UltraEP" README, "Tests":
+#                4 master + 2 redundant experts per rank, top-8, 8k tokens per
+#                rank) its three stated initial imbalances, 1.51, 2.01, 3.03.
 ALPHA_QWEN3 = 0.1845703125
 HOT_BOOST_DSV3 = (4.3984375, 4.91796875)
 HOT_BOOST_30PCT = 1.0234375
+ALPHA_PAGES = (0.107421875, 0.177734375, 0.2841796875)
 
 _TAG_LOGITS, _TAG_HIDDEN, _TAG_Y, _TAG_PERM, _TAG_PARAMS = 1, 2, 3, 4, 5
 
@@ -94,6 +99,8 @@ WORKLOADS = {
                  d=5120, recipe="per_rank"),
         Workload("sweep_48x8_r64_e128", 5, R=64, T=4096, E=128, K=8, S=2,
                  d=4096, recipe="sweep", layers=48, microbatches=8),
+        Workload("pages_ep64_e256_t8k", 6, R=64, T=8192, E=256, K=8, S=2,
+                 d=7168, recipe="zipf", zipf_s=1.0),
     ]
 }
 
@@ -176,7 +183,8 @@ def logit_bias(w: Workload, layer: int = 0, mb: int = 0, seed: int = 0,
     info = {}
     if w.recipe == "zipf":
         perm = _perm(E, seed, w.cid, layer, mb)
-        a = (ALPHA_QWEN3 if w.name.startswith("qwen3") else 1.0) if alpha is None else alpha
+        a = ({"qwen3": ALPHA_QWEN3, "pages": ALPHA_PAGES[1]}.get(w.name.split("_")[0], 1.0)
+             if alpha is None else alpha)
         b = a * zipf_log_weights(E, w.zipf_s, perm)
         bias = np.tile(b, (R, 1))
         info.update(perm=perm, alpha=a, s=w.zipf_s)

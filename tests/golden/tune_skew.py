@@ -1,6 +1,7 @@
 """Find the skew constants of the synthetic workloads with the CPU oracle.
 
-Prints ALPHA_QWEN3, HOT_BOOST_DSV3 and HOT_BOOST_30PCT for ``synth``. The
+Prints ALPHA_QWEN3, HOT_BOOST_DSV3, HOT_BOOST_30PCT and ALPHA_PAGES for
+``synth``. The
 values are found by bisection on the oracle's exact histogram:
 
 * Qwen3-shaped layer: scale of the s=1.0 Zipf bias so that the masters-only
@@ -8,6 +9,8 @@ values are found by bisection on the oracle's exact histogram:
 * DeepSeek-V3-shaped layer: additive boosts of the two hotspot experts so
   that each draws 8% of all pairs.
 * Sweep single-expert case: boost so that 30% of tokens route to one expert.
+* The pages' runtime-test layer (EP64, 256 experts): scales of the s=1.0
+  Zipf bias for masters-only max/mean 1.51, 2.01 and 3.03.
 
 Only the oracle and the input generator are used. Run:
     python tests/golden/tune_skew.py
@@ -91,11 +94,27 @@ def tune_30pct():
     return x
 
 
+def tune_pages():
+    """The pages' runtime-test layer (EP64, E=256, M=4, S=2, K=8, T=8192):
+    Zipf scales for masters-only max/mean 1.51, 2.01 and 3.03."""
+    w = synth.WORKLOADS["pages_ep64_e256_t8k"]
+    f = lambda a: masters_max_over_mean(w, loads(w, alpha=a))
+    out = []
+    for target in (1.51, 2.01, 3.03):
+        a, v = bisect(f, 0.0, 4.0, target, 0.005, iters=24)
+        out.append(a)
+        print(f"  alpha {a!r} -> masters-only max/mean {v:.4f} (target {target})")
+    print(f"ALPHA_PAGES = ({out[0]!r}, {out[1]!r}, {out[2]!r})")
+    return out
+
+
 if __name__ == "__main__":
-    which = sys.argv[1:] or ["qwen3", "dsv3", "30pct"]
+    which = sys.argv[1:] or ["qwen3", "dsv3", "30pct", "pages"]
     if "qwen3" in which:
         tune_qwen3()
     if "dsv3" in which:
         tune_dsv3()
     if "30pct" in which:
         tune_30pct()
+    if "pages" in which:
+        tune_pages()

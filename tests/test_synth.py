@@ -75,6 +75,17 @@ def test_sweep_single_expert_case_takes_30_percent_of_tokens():
     assert abs(load_e[info["hot"][0]] / w.N - 0.30) <= 0.005
 
 
+@pytest.mark.slow_cpu
+@pytest.mark.parametrize("i,target", [(0, 1.51), (1, 2.01), (2, 3.03)])
+def test_pages_layer_initial_imbalances(i, target):
+    # the pages' runtime test (EP64, 256 experts, 4 masters per rank) at its
+    # three stated initial imbalances
+    w = synth.WORKLOADS["pages_ep64_e256_t8k"]
+    idx, _ = oracle.gate_topk(synth.logits(w, alpha=synth.ALPHA_PAGES[i]), w.K)
+    _, load_e = oracle.count(idx, w.R, w.T, w.E)
+    assert abs(masters_skew(w, load_e) - target) <= 0.01
+
+
 def test_sweep_uniform_case_has_no_bias():
     w = synth.WORKLOADS["sweep_48x8_r64_e128"]
     bias, info = synth.logit_bias(w, 0, 0)
