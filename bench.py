@@ -652,41 +652,74 @@ def main():
                us_per_layer_incl_combine=1e3 * sum(per_kernel_ms.values()),
                parallelism=f"replicas: {world} independent layer instance(s), one per GPU")
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers. Every step copies
+    # its inputs in from pinned host memory and its result (combine output and
+    # plan stats) back out. Consecutive steps are pipelined over two buffer
+    # sets and three streams, so step s+1's upload, step s's kernels and step
+    # s-1's readback overlap (PCIe is full duplex): a step may start its
+    # kernels once its inputs are in and its buffer set's previous result has
+    # been read out.
     e2e = None
     if not args.no_e2e:
         lg_pin = torch.from_numpy(logits_h).pin_memory()
         hd_pin = torch.from_numpy(hidden_h.view(np.int16)).pin_memory()
-        out_pin = torch.empty(L.out.shape, dtype=torch.float32).pin_memory()
-        st_pin = torch.empty(4, dtype=torch.int32).pin_memory()
-        rl_pin = torch.empty(w.R, dtype=torch.int32).pin_memory()
+        L2 = ue.Layer(w.R, w.T, w.E, w.K, w.S, w.d, device=local)
+        bufs = [L, L2]
+        outs = [torch.empty(L.out.shape, dtype=torch.float32).pin_memory() for _ in bufs]
+        stats_pin = [torch.empty(4 + w.R, dtype=torch.int32).pin_memory() for _ in bufs]
+        s_in, s_run, s_out = (torch.cuda.Stream(dev), torch.cuda.Stream(dev),
+                              torch.cuda.Stream(dev))
+        ev_in = [torch.cuda.Event() for _ in bufs]
+        ev_run = [torch.cuda.Event() for _ in bufs]
+        ev_out = [torch.cuda.Event() for _ in bufs]
+        for b in range(2):  # nothing to wait for on the first use of a set
+            ev_run[b].record(s_run)
+            ev_out[b].record(s_out)
 
-        def e2e_step():
-            L.logits.copy_(lg_pin, non_blocking=True)
-            L.hidden.view(torch.int16).copy_(hd_pin, non_blocking=True)
-            step()
-            out_pin.copy_(L.out, non_blocking=True)
-            st_pin.copy_(L.stats, non_blocking=True)
-            rl_pin.copy_(L.rank_load, non_blocking=True)
+        def e2e_step(i):
+            b = i % 2
+            Lb = bufs[b]
+            s_in.wait_event(ev_run[b])          # the set's last kernels are done with its inputs
+            with torch.cuda.stream(s_in):
+                Lb.logits.copy_(lg_pin, non_blocking=True)
+                Lb.hidden.view(torch.int16).copy_(hd_pin, non_blocking=True)
+            ev_in[b].record(s_in)
+            s_run.wait_event(ev_in[b])
+            s_run.wait_event(ev_out[b])          # its previous result has been read out
+            for f in [Lb.gate, Lb.count, Lb.plan_step, Lb.reroute, Lb.permute, Lb.combine]:
+                f(stream=s_run)
+            ev_run[b].record(s_run)
+            s_out.wait_event(ev_run[b])
+            with torch.cuda.stream(s_out):
+                outs[b].copy_(Lb.out, non_blocking=True)
+                stats_pin[b][:4].copy_(Lb.stats, non_blocking=True)
+                stats_pin[b][4:].copy_(Lb.rank_load, non_blocking=True)
+            ev_out[b].record(s_out)
 
-        for _ in range(2):
-            e2e_step()
+        for i in range(2):
+            e2e_step(i)
+        torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s_in)
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        b_.record(s_out)
         torch.cuda.synchronize(dev)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(a.elapsed_time(b) / args.e2e_steps, world, dev)
+        e2e_ms = max_over_ranks(a.elapsed_time(b_) / args.e2e_steps, world, dev)
+        rc2 = L2.error(s_run) or L.error(s_run)
+        L2.close()
+        if rc2 != 0:
+            raise SystemExit(f"device error in the end-to-end steps: {ue.STATUS.get(rc2, rc2)}")
         h2d = lg_pin.numel() * 4 + hd_pin.numel() * 2
-        d2h = out_pin.numel() * 4 + 4 * 4 + w.R * 4
+        d2h = outs[0].numel() * 4 + stats_pin[0].numel() * 4
         e2e = {"value": world * w.Q / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "what": "pinned host logits + hidden -> device, full path, combine output + "
-                       "plan stats -> host, every step"}
+               "what": "every step: pinned host logits + hidden -> device, the six kernels, "
+                       "fp32 combine output + plan stats -> pinned host; consecutive steps "
+                       "pipelined over two buffer sets and three streams (upload, kernels, "
+                       "readback overlap)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -12,13 +12,13 @@
 // the combine with unit weights and runs in k_combine.cu.)
 //
 // Design (B200): HBM-bound (per pair: 2d bytes of y read, 2d bytes of dy
-// written; per token 4d bytes of dout read once). A group of threads owns a
-// token; each thread owns 16-byte chunks of the row (8 elements), reads the
-// token's fp32 gradient chunk once, then for each k reads the y chunk,
-// accumulates the dot product in fp32 (fixed order) and writes w*dout as
-// bf16. The per-thread partial dots are summed by a fixed tree (warp
-// shuffles, then a shared-memory pass across the token's warps), so dw is
-// deterministic.
+// written; per token 4d bytes of dout read once). One warp owns a token; each
+// lane owns every 32nd 16-byte chunk of the row (8 elements), reads the
+// token's fp32 gradient chunk once, issues the K y-chunk loads before using
+// any, accumulates the K dot products in fp32 (chunks in order) and writes
+// w*dout as bf16. The lanes' partial dots are then summed by a fixed
+// butterfly of warp shuffles, so dw is the same on every run, and no
+// block-wide barrier is needed.
 #include <cuda_bf16.h>
 
 #include "ue_internal.cuh"
@@ -27,6 +27,7 @@ namespace ue {
 namespace {
 
 constexpr int kBwdThreads = 256;
+constexpr int kBwdWarps = kBwdThreads / 32;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
@@ -40,20 +41,13 @@ __global__ void __launch_bounds__(kBwdThreads)
 combine_bwd_kernel(const float* __restrict__ dout, const uint16_t* __restrict__ y,
                    const int32_t* __restrict__ dest_row, const float* __restrict__ w,
                    uint16_t* __restrict__ dy, float* __restrict__ dw, int64_t N, int K, int d,
-                   int tpt, int64_t Q, int* err)
+                   int64_t Q, int* err)
 {
-    __shared__ float s_part[kBwdThreads / 32][KMAX];
     const int C = d >> 3;
-    const int tpb = blockDim.x / tpt;
-    const int sub = threadIdx.x / tpt;
-    const int lt = threadIdx.x - sub * tpt;
     const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int wpt = (tpt + 31) / 32;  // warps per token (tpt >= 32)
-    // token groups never straddle a warp (tpt is a multiple of 32)
-    for (int64_t n0 = (int64_t)blockIdx.x * tpb; n0 < N; n0 += (int64_t)gridDim.x * tpb) {
-        const int64_t n = n0 + sub;
-        const bool live = sub < tpb && n < N;
+    const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t n = gwarp; n < N; n += nwarps) {
         int rows[KMAX];
         float wk[KMAX], part[KMAX];
 #pragma unroll
@@ -61,25 +55,26 @@ combine_bwd_kernel(const float* __restrict__ dout, const uint16_t* __restrict__ 
             rows[k] = -1;
             wk[k] = 0.0f;
             part[k] = 0.0f;
-            if (live && k < K) {
+            if (k < K) {
                 const int r = __ldg(dest_row + n * K + k);
                 if (r >= 0 && (int64_t)r < Q) {
                     rows[k] = r;
                     wk[k] = __ldg(w + n * K + k);
-                } else if (lt == 0) {
+                } else if (lane == 0) {
                     raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(n * K + k, (int64_t)INT_MAX));
                 }
             }
         }
-        for (int c = lt; live && c < C; c += tpt) {
-            const float4 g0 = __ldcs(reinterpret_cast<const float4*>(dout + n * d) + 2 * c);
-            const float4 g1 = __ldcs(reinterpret_cast<const float4*>(dout + n * d) + 2 * c + 1);
-            const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        const float4* g_row = reinterpret_cast<const float4*>(dout + n * d);
+        for (int c = lane; c < C; c += 32) {
+            const float4 g0 = __ldcs(g_row + 2 * c);
+            const float4 g1 = __ldcs(g_row + 2 * c + 1);
             uint4 v[KMAX];
 #pragma unroll
             for (int k = 0; k < KMAX; ++k)
                 v[k] = rows[k] >= 0 ? __ldcs(reinterpret_cast<const uint4*>(y + (int64_t)rows[k] * d) + c)
                                     : make_uint4(0u, 0u, 0u, 0u);
+            const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
             for (int k = 0; k < KMAX; ++k) {
                 if (rows[k] < 0) continue;
@@ -97,59 +92,64 @@ combine_bwd_kernel(const float* __restrict__ dout, const uint16_t* __restrict__ 
                 __stcs(reinterpret_cast<uint4*>(dy + (int64_t)rows[k] * d) + c, o);
             }
         }
-        // dw: fixed-order tree over the token's threads
+        // dw: fixed butterfly over the warp; lane k writes dw[n][k]
+        float mine = 0.0f;
 #pragma unroll
         for (int k = 0; k < KMAX; ++k) {
             float p = part[k];
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(kFull, p, off);
-            if (lane == 0) s_part[warp][k] = p;
+            if (lane == k) mine = p;
         }
-        __syncthreads();
-        if (live && lt == 0) {
-            const int w0 = warp;  // the token's first warp
-            for (int k = 0; k < K && k < KMAX; ++k) {
-                float acc = 0.0f;
-                for (int ww = 0; ww < wpt; ++ww) acc += s_part[w0 + ww][k];
-                if (rows[k] >= 0) dw[n * K + k] = acc;
-            }
+        if (lane < K && lane < KMAX) {
+            // every lane holds the rows of all K pairs; pick pair (n, lane)'s
+            // without dynamic register indexing
+            int r_l = -1;
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k)
+                if (k == lane) r_l = rows[k];
+            if (r_l >= 0) dw[n * K + lane] = mine;
         }
-        __syncthreads();
     }
 }
 
 template <int KMAX>
-cudaError_t launch_k(const Sizes& z, const float* dout, const uint16_t* y, const int32_t* dest_row,
-                     const float* w, uint16_t* dy, float* dw, int num_sms, int* err,
-                     cudaStream_t st)
+cudaError_t shape_k(const Sizes& z, int num_sms, int* grid)
 {
-    const int C = z.d / 8;
-    int tpt = 32;
-    while (tpt < C && tpt < kBwdThreads) tpt <<= 1;
-    const int tpb = kBwdThreads / tpt;
     int per_sm = 0;
     cudaError_t ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_bwd_kernel<KMAX>,
                                                                    kBwdThreads, 0);
     if (ce != cudaSuccess) return ce;
     per_sm = std::max(per_sm, 1);
-    const int64_t need = std::max<int64_t>(1, (z.N + tpb - 1) / tpb);
-    const int grid = (int)std::min<int64_t>(need, (int64_t)num_sms * per_sm);
-    combine_bwd_kernel<KMAX><<<grid, kBwdThreads, 0, st>>>(dout, y, dest_row, w, dy, dw, z.N, z.K,
-                                                           z.d, tpt, z.Q, err);
-    return cudaGetLastError();
+    const int64_t need = std::max<int64_t>(1, (z.N + kBwdWarps - 1) / kBwdWarps);
+    *grid = (int)std::min<int64_t>(need, (int64_t)num_sms * per_sm);
+    return cudaSuccess;
 }
 
 }  // namespace
 
+cudaError_t plan_combine_backward_grid(const Sizes& z, int num_sms, int* grid)
+{
+    if (z.K <= 4) return shape_k<4>(z, num_sms, grid);
+    if (z.K <= 8) return shape_k<8>(z, num_sms, grid);
+    if (z.K <= 16) return shape_k<16>(z, num_sms, grid);
+    return shape_k<32>(z, num_sms, grid);
+}
+
 cudaError_t launch_combine_backward(const Sizes& z, const float* dout, const uint16_t* y,
                                     const int32_t* dest_row, const float* w, uint16_t* dy,
-                                    float* dw, int num_sms, int* err, cudaStream_t st)
+                                    float* dw, int grid, int* err, cudaStream_t st)
 {
     if (z.N == 0) return cudaSuccess;
-    if (z.K <= 4) return launch_k<4>(z, dout, y, dest_row, w, dy, dw, num_sms, err, st);
-    if (z.K <= 8) return launch_k<8>(z, dout, y, dest_row, w, dy, dw, num_sms, err, st);
-    if (z.K <= 16) return launch_k<16>(z, dout, y, dest_row, w, dy, dw, num_sms, err, st);
-    return launch_k<32>(z, dout, y, dest_row, w, dy, dw, num_sms, err, st);
+#define UE_BWD(KM)                                                                              \
+    combine_bwd_kernel<KM><<<grid, kBwdThreads, 0, st>>>(dout, y, dest_row, w, dy, dw, z.N, z.K, \
+                                                         z.d, z.Q, err)
+    if (z.K <= 4) UE_BWD(4);
+    else if (z.K <= 8) UE_BWD(8);
+    else if (z.K <= 16) UE_BWD(16);
+    else UE_BWD(32);
+#undef UE_BWD
+    return cudaGetLastError();
 }
 
 }  // namespace ue
