@@ -255,7 +255,9 @@ def run_sweep(args):
     """All 48 x 8 instances of the non-stationary sweep through one CUDA graph
     of the whole path. Each instance's logits are staged into the input
     buffer outside the timed region; each replay is timed with CUDA events.
-    Reports the distribution of us per layer and of the imbalance."""
+    Reports the distribution of us per layer and of the imbalance. --planner
+    bisect plans with the capacity planner at the pages' defaults instead of
+    the greedy rule."""
     import numpy as np
     import torch
 
@@ -269,15 +271,28 @@ def run_sweep(args):
     L = ue.Layer(w.R, w.T, w.E, w.K, w.S, w.d, device=0)
     L.hidden.copy_(torch.from_numpy(synth.hidden(w).view(np.int16)).to(dev).view(torch.bfloat16))
     L.logits.copy_(torch.from_numpy(synth.logits(w, 0, 0)))
+    opts = ue.plan_opts(ue.UE_SOLVER_BISECT) if args.planner == "bisect" else None
+
+    def run_once(st):
+        L.gate(st)
+        L.count(st)
+        if opts is None:
+            L.plan_step(st)
+        else:
+            L.plan_ex(opts, st)
+        L.reroute(st)
+        L.permute(st)
+        L.combine(stream=st)
+
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.stream(s):
         for _ in range(max(3, args.warmup)):
-            L.run(stream=s)
+            run_once(s)
     torch.cuda.synchronize(dev)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=s):
-        L.run(stream=s)
+        run_once(s)
     torch.cuda.synchronize(dev)
     stage = torch.empty(L.logits.shape, dtype=torch.float32).pin_memory()
     times, before, after, copies = [], [], [], []
@@ -297,7 +312,7 @@ def run_sweep(args):
             st = L.stats.cpu().numpy()
             before.append(float(st[1]) / (w.Q / w.R))
             after.append(float(st[2]) / (w.Q / w.R))
-            copies.append(int(st[0]))
+            copies.append(int((L.slot_expert[: w.G] >= 0).sum().item()))
     clk = clocks.stop()
     rc = L.error()
     L.close()
@@ -317,6 +332,9 @@ def run_sweep(args):
         "config": {"workload": w.name, "R": w.R, "T": w.T, "E": w.E, "K": w.K, "S": w.S,
                    "d": w.d, "instances": len(times), "pairs_per_instance": w.Q,
                    "graph": "whole path captured once, replayed per instance",
+                   "planner": args.planner + ("" if opts is None else
+                                              " (capacity planner: eps 0.01, early stop 1.0, "
+                                              "minimum 1024 pairs per replica)"),
                    "l2": "inputs larger than L2"},
         "us_per_layer": dist(times), "max_over_mean_before": dist(before),
         "max_over_mean_after": dist(after), "copies": dist(copies), "clocks": clk,
@@ -327,6 +345,10 @@ def run_sweep(args):
 
 # ------------------------------------------------------------------- rows ----
 EXPERT_NUMEL = 2 * 4096 * 1536 + 4096 * 1536  # Qwen3-235B expert: fc1 2hf + fc2 hf
+
+
+def expert_numel(args):
+    return args.expert_numel or EXPERT_NUMEL
 
 
 def run_row(args, w):
@@ -379,22 +401,24 @@ def run_row(args, w):
         se = plan["slot_expert"]
         used = int((se >= 0).sum())
         cnt = np.bincount(se[se >= 0], minlength=w.E)
+        numel = expert_numel(args)
         if args.row == "weight_sync":
-            bpe = EXPERT_NUMEL * 2
-            master = torch.randint(-30000, 30000, (w.E, EXPERT_NUMEL), dtype=torch.int16,
+            bpe = numel * 2
+            master = torch.randint(-30000, 30000, (w.E, numel), dtype=torch.int16,
                                    device=dev, generator=gen)
-            reps = torch.empty((w.G, EXPERT_NUMEL), dtype=torch.int16, device=dev)
+            reps = torch.empty((w.G, numel), dtype=torch.int16, device=dev)
             t = timed(lambda: ue.ue_weight_sync(L.ctx, L.plan, master, reps, bpe, st))
             kernels["weight_sync"] = (t, 2 * used * bpe)
         else:
-            master = torch.randn((w.E, EXPERT_NUMEL), dtype=torch.float32, device=dev, generator=gen)
-            reps = torch.randn((w.G, EXPERT_NUMEL), dtype=torch.float32, device=dev, generator=gen)
-            t = timed(lambda: ue.ue_grad_reduce(L.ctx, L.plan, reps, master, EXPERT_NUMEL, st))
+            master = torch.randn((w.E, numel), dtype=torch.float32, device=dev, generator=gen)
+            reps = torch.randn((w.G, numel), dtype=torch.float32, device=dev, generator=gen)
+            t = timed(lambda: ue.ue_grad_reduce(L.ctx, L.plan, reps, master, numel, st))
             nrep = int((cnt > 0).sum())
-            kernels["grad_reduce"] = (t, 4 * EXPERT_NUMEL * (2 * nrep + used))
-        workload = dict(workload=w.name, expert_numel=EXPERT_NUMEL, replicas=used,
+            kernels["grad_reduce"] = (t, 4 * numel * (2 * nrep + used))
+        workload = dict(workload=w.name, expert_numel=numel, replicas=used,
                         replicated_experts=int((cnt > 0).sum()),
-                        expert_shape="Qwen3-235B expert: fc1 2*4096*1536 + fc2 4096*1536")
+                        expert_shape=("Qwen3-235B expert: fc1 2*4096*1536 + fc2 4096*1536"
+                                      if numel == EXPERT_NUMEL else "reduced (profiling)"))
     rc = L.error()
     L.close()
     if rc != 0:
@@ -519,10 +543,14 @@ def main():
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="shrink T (profiling runs on a small case)")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--expert-numel", type=int, default=0,
+                    help="expert size for --row weight_sync / grad_reduce (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--sweep", action="store_true",
                     help="the 48 x 8 non-stationary sweep, CUDA-graph captured")
+    ap.add_argument("--planner", choices=("greedy", "bisect"), default="greedy",
+                    help="planner of the sweep (greedy: the path's rule)")
     ap.add_argument("--row", choices=("backward", "weight_sync", "grad_reduce", "planner"),
                     default=None, help="measure one of the rows beside the forward path "
                     "(planner: the planner variants, on pages_ep64_e256_t8k by default)")

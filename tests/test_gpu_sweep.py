@@ -10,6 +10,13 @@ Every instance is checked on the device by properties that hold at any size
 quota; each pair lands on a copy of its own expert; rank loads sum to the
 pairs). Eight instances, the two special ones included, are compared with
 the oracle element by element on the routing and on sampled dispatch rows.
+
+The sweep runs twice: with the path's greedy plan, and with the capacity
+planner at the pages' defaults ("UltraEP" README, "Performance Tuning /
+Replication planning": eps 0.01, early stop at 1.0, at least 1024 pairs per
+replica), whose every instance is also checked against its own guarantees
+(rank loads within the chosen capacity C(k) = floor(k Q / (100 R)), every
+replica at least 1024 pairs).
 """
 import numpy as np
 import pytest
@@ -35,10 +42,25 @@ def slot_owner(L, dev):
     return owner
 
 
-def test_sweep_graph_captured():
+@pytest.mark.parametrize("planner", ["greedy", "bisect"])
+def test_sweep_graph_captured(planner):
+    import token_rerouting_b200 as ue
     w = synth.WORKLOADS["sweep_48x8_r64_e128"]
     L = gh.make_layer(w.R, w.T, w.E, w.K, w.S, w.d)
     dev = L.device
+    opts = ue.plan_opts(ue.UE_SOLVER_BISECT) if planner == "bisect" else None
+
+    def run_once(st):
+        L.gate(st)
+        L.count(st)
+        if opts is None:
+            L.plan_step(st)
+        else:
+            L.plan_ex(opts, st)
+        L.reroute(st)
+        L.permute(st)
+        L.combine(stream=st)
+
     try:
         hidden = synth.hidden(w)
         L.hidden.copy_(gh.bf16_to_device(hidden, dev))
@@ -46,12 +68,12 @@ def test_sweep_graph_captured():
         s = torch.cuda.Stream(device=dev)
         s.wait_stream(torch.cuda.current_stream(dev))
         with torch.cuda.stream(s):
-            L.run(stream=s)
+            run_once(s)
         torch.cuda.current_stream(dev).wait_stream(s)
         torch.cuda.synchronize(dev)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=s):
-            L.run(stream=s)
+            run_once(s)
         torch.cuda.synchronize(dev)
 
         rng = np.random.default_rng(5)
@@ -79,8 +101,23 @@ def test_sweep_graph_captured():
                 iters.append(int(st[0]))
                 skew_before.append(st[1] / (w.Q / w.R))
                 skew_after.append(st[2] / (w.Q / w.R))
+                if opts is not None:
+                    cap = int(st[3]) * w.Q // (100 * w.R)
+                    assert int(L.rank_load.max()) <= cap, (layer, mb)
+                    used = L.slot_expert[: w.G] >= 0
+                    if bool(used.any()):
+                        rep_q = L.slot_quota.view(w.R, w.M + w.S)[:, w.M:].flatten()[used]
+                        assert int(rep_q.min()) >= 1024, (layer, mb)
                 if (layer, mb) in exact:
-                    o = oracle.run_path(logits, w.R, w.T, w.S, w.K)
+                    if opts is None:
+                        o = oracle.run_path(logits, w.R, w.T, w.S, w.K)
+                    else:
+                        idx, wts = oracle.gate_topk(logits, w.K)
+                        load_re, load_e = oracle.count(idx, w.R, w.T, w.E)
+                        pl = oracle.plan_bisect(load_e, w.R, w.S)
+                        phys, dest = oracle.reroute(idx, w.R, w.E, w.S, pl)
+                        o = dict(idx=idx, w=wts, load_re=load_re, load_e=load_e, plan=pl,
+                                 phys_slot=phys, dest_row=dest)
                     gh.assert_routing_equal(gh.routing_results(L), o)
                     rows = np.sort(rng.choice(w.Q, 2048, replace=False))
                     got = gh.bf16_to_host_u16(L.dispatch[torch.from_numpy(rows).to(dev)])
@@ -89,6 +126,10 @@ def test_sweep_graph_captured():
         assert L.error() == 0
         # the sweep spans balanced and heavily skewed instances
         assert min(skew_before) < 1.1 and max(skew_before) > 2.0
+        if opts is not None:
+            # the capacity planner brings every instance to within a few
+            # grid steps of the mean
+            assert max(skew_after) < 1.1, max(skew_after)
         assert len(iters) == w.layers * w.microbatches
     finally:
         L.close()

@@ -36,8 +36,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return a | (b << 16);
 }
 
+// K <= 8 fits in 80 registers without spilling, which leaves room for three
+// CTAs (24 token warps) per SM; larger K keeps the default budget.
 template <int KMAX>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kBwdThreads, KMAX <= 8 ? 3 : 1)
 combine_bwd_kernel(const float* __restrict__ dout, const uint16_t* __restrict__ y,
                    const int32_t* __restrict__ dest_row, const float* __restrict__ w,
                    uint16_t* __restrict__ dy, float* __restrict__ dw, int64_t N, int K, int d,
