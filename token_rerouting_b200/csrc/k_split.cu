@@ -16,63 +16,78 @@
 //   src_offset[r][p]  dispatch row of the first of them: a slot holds its
 //                     pairs by source rank, then in the source's own order.
 //
-// Design: one CTA per expert. The passes are short serial walks (at most
-// 1 + G copies and R sources) done by one thread in shared memory; they
-// produce at most 2*(1 + G) + R nonzero entries, each (r, j) at most once
-// (after copy j's local step either its host has no pairs left or its quota
-// is full), so the block zeroes the expert's [R] x [copies] block of the
-// output and then stores the entries. The row offsets are a scan over r per
-// copy. Empty redundant slots are written by the CTA of their rank's first
-// master.
+// Design: one CTA per expert, no serial walk. The remote pass is the
+// north-west-corner fill of the copies' remaining quotas (copy order) from
+// the sources' remaining pairs (ascending r), so the pairs source r gives
+// copy j are the overlap of j's interval [A_j, A_j + q'_j) and r's interval
+// [B_r, B_r + s'_r) on the line of cumulative remainders (A, B exclusive
+// prefix sums). Steps: each copy's own-rank take (a thread per copy; copies
+// that share a host are taken in copy order), the remainders, two warp
+// scans, and one thread per copy sweeping the source ranks once to write both
+// output columns (pairs and first row) with no global reads. Empty redundant
+// slots are written by the CTA of their rank's first master.
 #include "ue_internal.cuh"
 
 namespace ue {
 namespace {
 
 constexpr int kSplitThreads = 128;
-constexpr int kMaxEntries = 2 * (1 + kMaxG) + kMaxR;
+constexpr int kMaxCopies = 1 + kMaxG;
+
+// exclusive scan of v[0..n) into out[0..n), by one warp; returns the total
+__device__ int warp_exclusive_scan(const int* v, int* out, int n, int lane)
+{
+    int base = 0;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+        const int i = i0 + lane;
+        const int x = i < n ? v[i] : 0;
+        int incl = x;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off) incl += y;
+        }
+        if (i < n) out[i] = base + incl - x;
+        base += __shfl_sync(kFull, incl, 31);
+    }
+    return base;
+}
 
 __global__ void __launch_bounds__(kSplitThreads)
 locality_split_kernel(const int32_t* __restrict__ load_re, int R, int E, int S,
                       ue_placement plan, int32_t* __restrict__ src_quota,
                       int32_t* __restrict__ src_offset, int* err)
 {
-    __shared__ int s_cp[1 + kMaxG];   // physical slot of copy j
-    __shared__ int s_q[1 + kMaxG];    // quota left of copy j
-    __shared__ int s_s[kMaxR];        // pairs left of source rank r
-    __shared__ int s_er[kMaxEntries], s_ej[kMaxEntries], s_ea[kMaxEntries];
-    __shared__ int s_n, s_ne, s_bad;
+    __shared__ int s_cp[kMaxCopies];   // physical slot of copy j
+    __shared__ int s_q[kMaxCopies];    // quota of copy j, then what is left after its own-rank take
+    __shared__ int s_loc[kMaxCopies];  // pairs copy j takes from its own rank
+    __shared__ int s_A[kMaxCopies];    // exclusive prefix of the copies' remainders
+    __shared__ int s_s[kMaxR];         // pairs of source rank r, then what is left
+    __shared__ int s_B[kMaxR];         // exclusive prefix of the sources' remainders
+    __shared__ int s_n, s_tq, s_ts;
     const int e = blockIdx.x;
     const int M = E / R;
     const int G = R * S;
     const int P = R * (M + S);
     const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
     const int h0 = e / M;
 
-    if (tid < 32) {
+    if (warp == 0) {
+        // copies in copy order: the master, then replicas by ascending g
         int n = 1;
-        if (tid == 0) s_cp[0] = h0 * (M + S) + e % M;
+        if (lane == 0) s_cp[0] = h0 * (M + S) + e % M;
         for (int g0 = 0; g0 < G; g0 += 32) {
-            const int g = g0 + tid;
+            const int g = g0 + lane;
             const bool mine = g < G && __ldg(plan.slot_expert + g) == e;
             const unsigned b = __ballot_sync(kFull, mine);
-            if (mine) s_cp[n + __popc(b & ((1u << tid) - 1u))] = (g / S) * (M + S) + M + g % S;
+            if (mine) s_cp[n + __popc(b & ((1u << lane) - 1u))] = (g / S) * (M + S) + M + g % S;
             n += __popc(b);
         }
-        if (tid == 0) {
-            s_n = n;
-            s_ne = 0;
-            s_bad = 0;
-        }
+        if (lane == 0) s_n = n;
     }
     for (int r = tid; r < R; r += blockDim.x) s_s[r] = __ldg(load_re + (size_t)r * E + e);
-    __syncthreads();
-    const int n = s_n;
-    for (int j = tid; j < n; j += blockDim.x) s_q[j] = __ldg(plan.slot_quota + s_cp[j]);
-    for (int x = tid; x < R * n; x += blockDim.x) {
-        const int r = x / n, j = x - r * n;
-        src_quota[(size_t)r * P + s_cp[j]] = 0;
-    }
     if (e % M == 0) {
         // empty redundant slots of this rank: no pairs, rows at the slot's start
         for (int x = tid; x < R * S; x += blockDim.x) {
@@ -88,59 +103,54 @@ locality_split_kernel(const int32_t* __restrict__ load_re, int R, int E, int S,
         }
     }
     __syncthreads();
-    if (tid == 0) {
-        long long sum_s = 0, sum_q = 0;
-        for (int r = 0; r < R; ++r) sum_s += s_s[r];
-        for (int j = 0; j < n; ++j) sum_q += s_q[j];
-        int ne = 0;
-        if (sum_s != sum_q) {
-            raise_error(err, UE_ERR_DEVICE_BOUNDS, e);
-            s_bad = 1;
-        } else {
-            // local pass
-            for (int j = 0; j < n; ++j) {
-                const int h = s_cp[j] / (M + S);
-                const int a = min(s_s[h], s_q[j]);
-                if (a > 0) {
-                    s_er[ne] = h;
-                    s_ej[ne] = j;
-                    s_ea[ne] = a;
-                    ++ne;
-                    s_s[h] -= a;
-                    s_q[j] -= a;
-                }
-            }
-            // remote pass: sources in ascending r (what earlier copies took
-            // is gone, so one pointer over r serves every copy)
-            int r = 0;
-            for (int j = 0; j < n; ++j) {
-                while (s_q[j] > 0 && r < R) {
-                    const int a = min(s_s[r], s_q[j]);
-                    if (a > 0) {
-                        s_er[ne] = r;
-                        s_ej[ne] = j;
-                        s_ea[ne] = a;
-                        ++ne;
-                        s_s[r] -= a;
-                        s_q[j] -= a;
-                    }
-                    if (s_s[r] == 0) ++r;
-                }
-            }
+    const int n = s_n;
+    for (int j = tid; j < n; j += blockDim.x) s_q[j] = __ldg(plan.slot_quota + s_cp[j]);
+    __syncthreads();
+    // local pass: copy j takes min(what its host has left, its quota); the
+    // copies before it on the same host have taken first
+    for (int j = tid; j < n; j += blockDim.x) {
+        const int h = s_cp[j] / (M + S);
+        int left = s_s[h], take = 0;
+        for (int jj = 0; jj <= j; ++jj) {
+            if (s_cp[jj] / (M + S) != h) continue;
+            take = min(left, s_q[jj]);
+            left -= take;
         }
-        s_ne = ne;
+        s_loc[j] = take;
     }
     __syncthreads();
-    const int ne = s_ne;
-    for (int x = tid; x < ne; x += blockDim.x)
-        src_quota[(size_t)s_er[x] * P + s_cp[s_ej[x]]] = s_ea[x];
+    for (int j = tid; j < n; j += blockDim.x) {
+        s_q[j] -= s_loc[j];
+        atomicSub(&s_s[s_cp[j] / (M + S)], s_loc[j]);
+    }
     __syncthreads();
+    // prefix sums of the remainders (copies in copy order, sources by r)
+    if (warp == 0) {
+        const int t = warp_exclusive_scan(s_q, s_A, n, lane);
+        if (lane == 0) s_tq = t;
+    } else if (warp == 1) {
+        const int t = warp_exclusive_scan(s_s, s_B, R, lane);
+        if (lane == 0) s_ts = t;
+    }
+    __syncthreads();
+    // the loads must sum to the quotas (equal local takes leave the
+    // remainders' totals equal exactly when they do)
+    const bool ok = s_tq == s_ts;
+    if (!ok && tid == 0) raise_error(err, UE_ERR_DEVICE_BOUNDS, e);
     for (int j = tid; j < n; j += blockDim.x) {
         const int p = s_cp[j];
+        const int h = p / (M + S);
+        const int a0 = s_A[j], a1 = a0 + s_q[j];
         int run = __ldg(plan.slot_offset + p);
         for (int r = 0; r < R; ++r) {
+            int x = 0;
+            if (ok) {
+                const int b0 = s_B[r], b1 = b0 + s_s[r];
+                x = max(0, min(a1, b1) - max(a0, b0)) + (r == h ? s_loc[j] : 0);
+            }
+            src_quota[(size_t)r * P + p] = x;
             src_offset[(size_t)r * P + p] = run;
-            run += src_quota[(size_t)r * P + p];
+            run += x;
         }
     }
 }
