@@ -98,3 +98,43 @@ def test_host_rejects_misaligned_and_overlapping_rows(layer):
         ue.ue_combine(layer.ctx, layer.dispatch, layer.dest_row, layer.w,
                       layer.out.data_ptr() + 4)
     assert layer.error() == ue.UE_OK
+
+
+def test_variant_paths_report_bad_ids_and_loads(layer):
+    """The planner variants' kernels check their inputs the same way: a
+    negative load in the capacity planner, an out-of-range id in the
+    interleaved and locality reroutes; the context then runs clean."""
+    w = synth.custom(R, T, E, K, S, d, cid=504)
+    logits = synth.logits(w)
+    gh.load_inputs(layer, logits)
+    layer.run_routing()
+    assert layer.error() == ue.UE_OK
+    bisect = ue.plan_opts(ue.UE_SOLVER_BISECT, min_tokens=4)
+    good_load = layer.load_e.clone()
+    layer.load_e[9] = -1
+    layer.plan_ex(bisect)
+    assert layer.error() == ue.UE_ERR_DEVICE_BOUNDS
+    layer.load_e.copy_(good_load)
+    layer.plan_ex(bisect)
+    layer.locality_split()
+    assert layer.error() == ue.UE_OK
+    layer.idx[11, 2] = E
+    layer.reroute_ex(ue.UE_ORDER_INTERLEAVE)
+    assert layer.error() == ue.UE_ERR_DEVICE_BOUNDS
+    assert int(layer.dest_row[11, 2]) == -1
+    layer.reroute_local()
+    assert layer.error() == ue.UE_ERR_DEVICE_BOUNDS
+    assert int(layer.phys_slot[11, 2]) == -1
+    check_clean_run(layer, logits)
+
+
+def test_variant_calls_reject_bad_arguments(layer):
+    with pytest.raises(ue.UEError):
+        ue.ue_reroute_ex(layer.ctx, layer.idx, layer.plan, 7, layer.phys_slot, layer.dest_row)
+    with pytest.raises(ue.UEError):
+        ue.ue_locality_split(layer.ctx, layer.load_re, layer.plan,
+                             layer.src_quota.data_ptr() + 2, layer.src_offset)
+    with pytest.raises(ue.UEError):
+        ue.ue_reroute_local(layer.ctx, layer.idx, layer.load_re, layer.plan, layer.src_quota,
+                            layer.src_offset, layer.phys_slot, layer.dest_row.data_ptr() + 1)
+    assert layer.error() == ue.UE_OK
