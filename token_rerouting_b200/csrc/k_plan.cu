@@ -37,9 +37,12 @@
 //    registers (lane l owns ranks l, l+32, ... and their slots, so every
 //    load change lands in the lane that owns the rank). Per iteration: the
 //    stop test and the least loaded rank with a free slot (three `redux`
-//    reductions), the placement, and the new quotas of e*'s copies: its
-//    replicas are found by ballots in ascending slot order; the master's
-//    quota goes from ceil(L/(c-1)) to ceil(L/c).
+//    reductions, with the pick's ready flag loaded before them), the
+//    placement in r*'s lowest free slot, and the new quotas of e*'s copies: the
+//    master's goes from ceil(L/(c-1)) to ceil(L/c); a first replica takes
+//    floor(L/2); later replicas are found by ballots in ascending slot order.
+//    The count of co-located copies does not depend on the order of
+//    placement and is taken from the final slots.
 // Warp 1 needs far fewer instructions per step, so warp 0 rarely waits; its
 // wait on a queue entry is bounded. The rest of the CTA writes the outputs
 // and scans the slot offsets at the end.
@@ -78,7 +81,8 @@ __device__ __forceinline__ bool may_grow(unsigned L, unsigned c, unsigned m)
 
 struct Pick {
     int e;         // expert receiving the copy (-1: no expert may grow)
-    unsigned qb;   // floor(L / c) with the new copy count c
+    unsigned c;    // its copy count with the new copy
+    unsigned qb;   // floor(L / c)
     unsigned rem;  // L mod c
     unsigned dq0;  // master quota change: ceil(L/c) - ceil(L/(c-1)) (two's complement)
 };
@@ -101,6 +105,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
     __shared__ unsigned long long sQ;
     __shared__ int sStats[4];
     __shared__ int sWarpSum[kPlanWarps];
+    __shared__ int sColoc;
 
     const int M = E / R;
     const int G = R * S;
@@ -111,6 +116,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
         sQ = 0ull;
         sUsedPicks = 0;
         sDone = 0;
+        sColoc = 0;
     }
     for (int r = tid; r < R; r += blockDim.x) sRank[r] = 0;
     for (int g = tid; g < G; g += blockDim.x) sReady[g] = 0;
@@ -155,7 +161,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
             if (hi == 0u && lo == 0u) {
                 // no expert may take another copy: end marker
                 if (lane == 0) {
-                    sPick[t] = Pick{-1, 0u, 0u, 0u};
+                    sPick[t] = Pick{-1, 0u, 0u, 0u, 0u};
                     __threadfence_block();
                     sReady[t] = 1;
                 }
@@ -187,7 +193,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
                 const unsigned rem = Le - qb * ce;
                 const unsigned q0_new = qb + (rem > 0u ? 1u : 0u);
                 const unsigned q0_old = div_by(Le + ce - 2u, ce - 1u, sRecip);
-                sPick[t] = Pick{estar, qb, rem, q0_new - q0_old};
+                sPick[t] = Pick{estar, ce, qb, rem, q0_new - q0_old};
                 __threadfence_block();
                 sReady[t] = 1;
             }
@@ -210,9 +216,16 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
                 slotQ[j][s] = 0;
             }
         }
-        int iters = 0, colocated = 0;
+        int iters = 0;
         unsigned max_before = 0u;
         for (;;) {
+            // this iteration's pick: its flag is read first, so that the load
+            // overlaps the reductions below (acquire orders the pick read)
+            int ready = 0;
+            asm volatile("ld.acquire.cta.shared.u32 %0, [%1];"
+                         : "=r"(ready)
+                         : "r"((unsigned)__cvta_generic_to_shared((const void*)&sReady[iters]))
+                         : "memory");
             unsigned maxl = 0u, bestl = 0xffffffffu, bestr = 0xffffffffu;
 #pragma unroll
             for (int j = 0; j < NJR; ++j) {
@@ -229,33 +242,31 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
             if (ml == 0xffffffffu) break;  // no free slot anywhere
             const int rstar = (int)__reduce_min_sync(kFull, bestl == ml ? bestr : 0xffffffffu);
 
-            // this iteration's expert, from the expert side's queue
-            int ready = sReady[iters];
-            for (long long spin = 0; !ready && spin < kPickWaitLimit; ++spin) ready = sReady[iters];
+            // the pick is normally ready long before: the expert side needs
+            // far fewer instructions per step. The wait is bounded.
+            for (long long spin = 0; !ready && spin < kPickWaitLimit; ++spin)
+                asm volatile("ld.acquire.cta.shared.u32 %0, [%1];"
+                             : "=r"(ready)
+                             : "r"((unsigned)__cvta_generic_to_shared((const void*)&sReady[iters]))
+                             : "memory");
             ready = __all_sync(kFull, ready);
             if (!ready) {
                 if (lane == 0) raise_error(err, UE_ERR_TIMEOUT, iters);
                 break;
             }
-            __threadfence_block();
             const Pick pk = sPick[iters];
             if (pk.e < 0) break;  // no expert may take another copy
             const int estar = pk.e;
             const int rj = rstar >> 5;
             const bool rown = lane == (rstar & 31);
 
-            // r*'s lowest free slot; does r* already hold a copy of e*?
+            // the new copy goes into r*'s lowest free slot (the slot index is
+            // made warp-uniform so that the slot arrays stay in registers)
             int s_new = 0;
-            bool held = false;
 #pragma unroll
             for (int j = 0; j < NJR; ++j)
-                if (j == rj) {
-                    s_new = used[j];
-#pragma unroll
-                    for (int s = 0; s < SM; ++s) held |= rown && s < S && slotE[j][s] == estar;
-                }
+                if (j == rj) s_new = used[j];
             s_new = __shfl_sync(kFull, s_new, rstar & 31);
-            if (estar / M == rstar || __any_sync(kFull, held)) colocated += 1;
             if (rown) {
 #pragma unroll
                 for (int j = 0; j < NJR; ++j)
@@ -273,31 +284,47 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
                 for (int j = 0; j < NJR; ++j)
                     if (j == (rm >> 5)) load[j] += pk.dq0;
             }
-            // replicas, ascending slot g = r*S + s (r = lane + 32 j)
-            unsigned before = 0u;
-            const unsigned lt = (1u << lane) - 1u;
+            if (pk.c == 2u) {
+                // first replica: the only other copy is the master, and the
+                // replica's quota is floor(L/2) (L mod 2 < 2 keeps the +1 on
+                // the master)
+                if (rown) {
 #pragma unroll
-            for (int j = 0; j < NJR; ++j) {
-                unsigned lower = 0u;   // e* replicas in lower lanes of group j
-                unsigned total = 0u;   // e* replicas in group j
+                    for (int j = 0; j < NJR; ++j)
+                        if (j == rj) {
 #pragma unroll
-                for (int s = 0; s < SM; ++s) {
-                    const unsigned msk = __ballot_sync(kFull, s < S && slotE[j][s] == estar);
-                    lower += __popc(msk & lt);
-                    total += __popc(msk);
+                            for (int s = 0; s < SM; ++s)
+                                if (s < S && slotE[j][s] == estar) slotQ[j][s] = (int)pk.qb;
+                            load[j] += pk.qb;
+                        }
                 }
-                unsigned mine = 0u;  // e* replicas in this lane's lower slots
+            } else {
+                // replicas, ascending slot g = r*S + s (r = lane + 32 j)
+                unsigned before = 0u;
+                const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-                for (int s = 0; s < SM; ++s) {
-                    if (s < S && slotE[j][s] == estar) {
-                        const unsigned pos = 1u + before + lower + mine;
-                        const int qn = (int)(pk.qb + (pos < pk.rem ? 1u : 0u));
-                        load[j] = load[j] + (unsigned)(qn - slotQ[j][s]);
-                        slotQ[j][s] = qn;
-                        mine += 1u;
+                for (int j = 0; j < NJR; ++j) {
+                    unsigned lower = 0u;   // e* replicas in lower lanes of group j
+                    unsigned total = 0u;   // e* replicas in group j
+#pragma unroll
+                    for (int s = 0; s < SM; ++s) {
+                        const unsigned msk = __ballot_sync(kFull, s < S && slotE[j][s] == estar);
+                        lower += __popc(msk & lt);
+                        total += __popc(msk);
                     }
+                    unsigned mine = 0u;  // e* replicas in this lane's lower slots
+#pragma unroll
+                    for (int s = 0; s < SM; ++s) {
+                        if (s < S && slotE[j][s] == estar) {
+                            const unsigned pos = 1u + before + lower + mine;
+                            const int qn = (int)(pk.qb + (pos < pk.rem ? 1u : 0u));
+                            load[j] = load[j] + (unsigned)(qn - slotQ[j][s]);
+                            slotQ[j][s] = qn;
+                            mine += 1u;
+                        }
+                    }
+                    before += total;
                 }
-                before += total;
             }
             iters += 1;
         }
@@ -321,7 +348,6 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
             sStats[0] = iters;
             sStats[1] = (int)max_before;
             sStats[2] = (int)mx;
-            sStats[3] = colocated;
             sUsedPicks = iters;
             sDone = 1;
         }
@@ -333,12 +359,26 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
     for (int e = tid; e < E; e += blockDim.x) sC[e] = 1;
     __syncthreads();
     for (int t = tid; t < iters; t += blockDim.x) atomicAdd(&sC[sPick[t].e], 1);
+    // copies placed on a rank that already held a copy of the same expert:
+    // for each (expert, rank) every copy but the first one there, which is
+    // the same count whatever the order of placement (a replica counts unless
+    // it is the lowest slot of its expert on a rank without the master)
+    for (int g = tid; g < G; g += blockDim.x) {
+        const int e = sSlotE[g];
+        if (e >= 0) {
+            const int r = g / S, sl = g - r * S;
+            bool first = r != e / M;
+            for (int s2 = 0; s2 < sl; ++s2) first = first && sSlotE[r * S + s2] != e;
+            if (!first) atomicAdd(&sColoc, 1);
+        }
+    }
     __syncthreads();
 
     for (int e = tid; e < E; e += blockDim.x) out.n_copies[e] = sC[e];
     for (int g = tid; g < G; g += blockDim.x) out.slot_expert[g] = sSlotE[g];
     for (int r = tid; r < R; r += blockDim.x) out.rank_load[r] = sRank[r];
-    if (tid < 4) out.stats[tid] = sStats[tid];
+    if (tid < 3) out.stats[tid] = sStats[tid];
+    if (tid == 3) out.stats[3] = sColoc;
 
     // slot quotas in physical order and their exclusive running sum; each
     // thread owns slots 2*tid and 2*tid+1 (P <= 512). A master's quota is
