@@ -420,6 +420,7 @@ def run_row(args, w):
                         expert_shape=("Qwen3-235B expert: fc1 2*4096*1536 + fc2 4096*1536"
                                       if numel == EXPERT_NUMEL else "reduced (profiling)"))
     rc = L.error()
+    se_host = L.plan_arrays()["slot_expert"]
     L.close()
     if rc != 0:
         raise SystemExit(f"device error: {rc}")
@@ -432,7 +433,59 @@ def run_row(args, w):
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": out[dom]["gbs"], "peak": peak,
                          "unit": "GB/s", "frac": out[dom]["frac_of_peak"],
                          "peak_kind": f"of {peak_kind}"}}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = row_oracle_baseline(args, w, se_host)
     print(json.dumps(line), flush=True)
+
+
+def row_oracle_baseline(args, w, slot_expert):
+    """The oracle (single-threaded C, fp64 where the row computes in floating
+    point) on a bounded sample of the same row, reported in the row's units
+    (algorithmic GB/s of the sample over the oracle's time)."""
+    import numpy as np
+
+    import oracle
+    import synth
+    if args.row == "backward":
+        n, K, d = 4096, w.K, w.d
+        dest = np.arange(n * K, dtype=np.int32).reshape(n, K)
+        wts = np.random.default_rng(0).random((n, K)).astype(np.float32)
+        dout = synth.normal_f32(n * d, 0, 61).reshape(n, d)
+        y = synth.bf16_normal(n * K, d, 0, 62)
+        t0 = time.perf_counter()
+        oracle.combine_backward(dout, y, K, dest, wts)
+        oracle.permute_backward(y, n, K, dest)
+        secs = time.perf_counter() - t0
+        by = (4 * n * d + 2 * n * K * d + 8 * n * K + 2 * n * K * d + 4 * n * K) + \
+             (2 * n * K * d + 4 * n * K + 4 * n * d)
+        sample = f"{n} tokens x K={K} x d={d}: combine backward + permute backward"
+    else:
+        numel = expert_numel(args)
+        used = [g for g in range(len(slot_expert)) if slot_expert[g] >= 0][:8]
+        experts = sorted({int(slot_expert[g]) for g in used})
+        remap = {e: i for i, e in enumerate(experts)}
+        se = np.array([remap[int(slot_expert[g])] for g in used], dtype=np.int32)
+        rng = np.random.default_rng(0)
+        if args.row == "weight_sync":
+            bpe = numel * 2
+            master = rng.integers(0, 256, size=(len(experts), bpe), dtype=np.uint8)
+            reps = np.zeros((len(used), bpe), dtype=np.uint8)
+            t0 = time.perf_counter()
+            oracle.weight_sync(se, master, reps)
+            secs = time.perf_counter() - t0
+            by = 2 * len(used) * bpe
+        else:
+            master = rng.standard_normal((len(experts), numel), dtype=np.float32)
+            reps = rng.standard_normal((len(used), numel), dtype=np.float32)
+            t0 = time.perf_counter()
+            oracle.grad_reduce(se, reps, master)
+            secs = time.perf_counter() - t0
+            by = 4 * numel * (2 * len(experts) + len(used))
+        sample = (f"{len(used)} replica slots of {len(experts)} experts, "
+                  f"{numel} elements per expert")
+    gbs = by / secs / 1e9
+    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample,
+            "seconds": secs}
 
 
 def run_planner(args, w):
@@ -520,10 +573,37 @@ def run_planner(args, w):
                                                    S=w.S, pairs=w.Q, alpha=alpha,
                                                    target_imbalance=target),
                 "steps": args.steps, "imbalance_before": before, "solvers": res}
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = planner_oracle_baseline(w, synth.logits(w, alpha=alpha))
         if target is not None:
             line["pages_context"] = pages[target]
         print(json.dumps(line), flush=True)
     L.close()
+
+
+def planner_oracle_baseline(w, logits):
+    """The oracle's planner variants on the same layer instance (its own
+    top-k and counts), single-threaded: microseconds per call."""
+    import oracle
+    idx, _ = oracle.gate_topk(logits, w.K)
+    load_re, load_e = oracle.count(idx, w.R, w.T, w.E)
+    us = {}
+
+    def timed(name, fn):
+        t0 = time.perf_counter()
+        r = fn()
+        us[name] = (time.perf_counter() - t0) * 1e6
+        return r
+
+    timed("plan_greedy", lambda: oracle.plan(load_e, w.R, w.S))
+    pl = timed("plan_bisect", lambda: oracle.plan_bisect(load_e, w.R, w.S))
+    timed("reroute_prefix", lambda: oracle.reroute(idx, w.R, w.E, w.S, pl))
+    timed("reroute_interleave", lambda: oracle.reroute_interleave(idx, w.R, w.T, w.E, w.S, pl))
+    sq, so = timed("locality_split", lambda: oracle.locality_split(load_re, w.S, pl))
+    timed("reroute_local", lambda: oracle.reroute_local(idx, w.R, w.T, w.E, w.S, pl, sq, so))
+    return {"unit": "us per call", "us": us, "cores": 1, "kind": "oracle",
+            "sample": "the whole layer instance (the oracle's own top-k and counts; the capacity "
+                      "plan feeds the reroutes)"}
 
 
 def synth_logits(w):
@@ -620,35 +700,62 @@ def main():
         raise SystemExit(f"device error after warm-up: {ue.STATUS.get(rc, rc)}")
     plan0 = L.plan_arrays()
 
+    # the step as one CUDA graph of the six kernels (captured once, outside
+    # the timed region), so that the timed steps carry no launch gaps
+    gstream = torch.cuda.Stream(dev)
+    gstream.wait_stream(stream)
+    with torch.cuda.stream(gstream):
+        for f in steps_fn:
+            f(stream=gstream)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=gstream):
+        for f in steps_fn:
+            f(stream=gstream)
+    torch.cuda.synchronize(dev)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.2)
-    # kernel-level events: ev[s][k] .. ev[s][k+1] brackets kernel k of step s
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(steps_fn) + 1)]
-           for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for s in range(args.steps):
-        ev = evs[s]
-        ev[0].record(stream)
-        for k, f in enumerate(steps_fn):
-            f(stream=stream)
-            ev[k + 1].record(stream)
+        graph.replay()
     end.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    clk = clocks.stop()
     total_ms = start.elapsed_time(end)
     rc = L.error(stream)
     if rc != 0:
         raise SystemExit(f"device error in the timed region: {ue.STATUS.get(rc, rc)}")
 
+    # per-kernel breakdown from eager launches bracketed by events (not part
+    # of the value): ev[s][k] .. ev[s][k+1] brackets kernel k of step s
+    nk = min(args.steps, 50)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(steps_fn) + 1)]
+           for _ in range(nk)]
+    for s in range(nk):
+        ev = evs[s]
+        ev[0].record(stream)
+        for k, f in enumerate(steps_fn):
+            f(stream=stream)
+            ev[k + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    rc = L.error(stream)
+    if rc != 0:
+        raise SystemExit(f"device error in the breakdown steps: {ue.STATUS.get(rc, rc)}")
+    del graph
+
     per_kernel_ms = {name: statistics.fmean(evs[s][k].elapsed_time(evs[s][k + 1])
-                                            for s in range(args.steps))
+                                            for s in range(nk))
                      for k, name in enumerate(KERNELS)}
     ms_step_local = total_ms / args.steps
     ms_step = max_over_ranks(ms_step_local, world, dev)
@@ -678,6 +785,8 @@ def main():
     gate_to_permute = sum(per_kernel_ms[k] for k in KERNELS[:5])
     cfg.update(us_per_layer_gate_to_permute=1e3 * gate_to_permute,
                us_per_layer_incl_combine=1e3 * sum(per_kernel_ms.values()),
+               timing="each timed step replays one CUDA graph of the six kernels; per-kernel "
+                      "times from eager launches bracketed by CUDA events",
                parallelism=f"replicas: {world} independent layer instance(s), one per GPU")
 
     # end to end through the public API with host buffers. Every step copies
