@@ -34,8 +34,9 @@
 // records UE_ERR_TIMEOUT and writes nothing. Finally each warp re-walks its
 // 512 pairs in order, ranking equal ids within 32 lanes (the lanes holding
 // the same id come from nine ballots over the id's bits), and writes the
-// physical slot and dispatch row; the copy index comes from one exact
-// multiply-high by a per-expert reciprocal.
+// physical slot and dispatch row; for floor-form quotas the copy index comes
+// from one exact multiply-high by a per-expert reciprocal, otherwise from the
+// binary search.
 // The status words carry the launch's tag, so nothing is cleared between
 // launches: words of earlier launches read as "not yet published". The last
 // CTA to finish resets the ticket and the counter and advances the epoch.
