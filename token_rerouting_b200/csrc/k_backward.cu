@@ -12,22 +12,26 @@
 // the combine with unit weights and runs in k_combine.cu.)
 //
 // Design (B200): HBM-bound (per pair: 2d bytes of y read, 2d bytes of dy
-// written; per token 4d bytes of dout read once). One warp owns a token; each
-// lane owns every 32nd 16-byte chunk of the row (8 elements), reads the
-// token's fp32 gradient chunk once, issues the K y-chunk loads before using
-// any, accumulates the K dot products in fp32 (chunks in order) and writes
-// w*dout as bf16. The lanes' partial dots are then summed by a fixed
-// butterfly of warp shuffles, so dw is the same on every run, and no
-// block-wide barrier is needed.
+// written; per token 4d bytes of dout read once), the same scattered-write
+// pattern as the permute, and built like it: short-lived CTAs, each token
+// owned by a group of whole warps with one 16-byte chunk (8 elements) per
+// thread. A thread reads the token's fp32 gradient chunk once, issues its K
+// y-chunk loads before using any, accumulates the K dot products in fp32 and
+// writes w*dout as bf16. dw is then summed by a fixed butterfly of warp
+// shuffles and a fixed-order pass over the token's warps, so it is the same
+// on every run. For the common shapes (K = 4 or 8, d <= 8192) a CTA holds
+// one token and a thread exactly one chunk, with no loop and the row checks
+// kept off the hot path (a row out of range is masked and reported after the
+// work), which keeps it near 50 registers: two 512-thread CTAs per SM. Other
+// shapes loop over their chunks. (A persistent warp-per-token form reached
+// 0.90 of the copy bandwidth; the same CTA shape with a chunk loop, per-pair
+// branches or several tokens per CTA spilled registers and reached 0.87-0.90.)
 #include <cuda_bf16.h>
 
 #include "ue_internal.cuh"
 
 namespace ue {
 namespace {
-
-constexpr int kBwdThreads = 256;
-constexpr int kBwdWarps = kBwdThreads / 32;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
@@ -36,116 +40,227 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return a | (b << 16);
 }
 
-// K <= 8 fits in 80 registers without spilling, which leaves room for three
-// CTAs (24 token warps) per SM; larger K keeps the default budget.
+// dy chunk = w * dout chunk, rounded to bf16
+__device__ __forceinline__ uint4 scaled_bf16(float wk, const float (&g)[8])
+{
+    uint4 o;
+    o.x = pack_bf16x2(wk * g[0], wk * g[1]);
+    o.y = pack_bf16x2(wk * g[2], wk * g[3]);
+    o.z = pack_bf16x2(wk * g[4], wk * g[5]);
+    o.w = pack_bf16x2(wk * g[6], wk * g[7]);
+    return o;
+}
+
+// part += <g, bf16 chunk v>, elements in order
+__device__ __forceinline__ float dot_bf16(float part, const float (&g)[8], uint4 v)
+{
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        part = fmaf(g[2 * q], __uint_as_float(u[q] << 16), part);
+        part = fmaf(g[2 * q + 1], __uint_as_float(u[q] & 0xffff0000u), part);
+    }
+    return part;
+}
+
+// One chunk per thread, K known at compile time (4 or 8), d <= 8192: one
+// token per CTA, blockDim = cw = the row's chunks rounded up to whole warps. A row out of range is only masked: its loads read row 0, which is
+// in range, it stores nothing, and the error is recorded after the work.
+template <int K>
+__global__ void __launch_bounds__(1024)
+combine_bwd_chunk_kernel(const float* __restrict__ dout, const uint16_t* __restrict__ y,
+                         const int32_t* __restrict__ dest_row, const float* __restrict__ w,
+                         uint16_t* __restrict__ dy, float* __restrict__ dw, int64_t N, int d,
+                         int cw, int64_t Q, int* err)
+{
+    constexpr unsigned kAll = (1u << K) - 1u;
+    __shared__ float s_part[32][K];
+    const int C = d >> 3;
+    const int c = threadIdx.x;             // this thread's chunk of the row
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t n = blockIdx.x;
+    const bool live = n < N;
+    int rows[K];
+    float wk[K], part[K];
+    unsigned valid = 0u;  // pairs with a row in range
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        const int r = live ? __ldg(dest_row + n * K + k) : 0;
+        const bool ok = (unsigned long long)(unsigned)r < (unsigned long long)Q;  // r >= 0 && r < Q
+        rows[k] = ok ? r : 0;
+        valid |= ok ? (1u << k) : 0u;
+        wk[k] = live ? __ldg(w + n * K + k) : 0.0f;
+        part[k] = 0.0f;
+    }
+    if (live && c < C) {
+        const float4* g_row = reinterpret_cast<const float4*>(dout + n * d);
+        const float4 g0 = __ldcs(g_row + 2 * c);
+        const float4 g1 = __ldcs(g_row + 2 * c + 1);
+        const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        uint4 v[K];
+#pragma unroll
+        for (int k = 0; k < K; ++k)
+            v[k] = __ldcs(reinterpret_cast<const uint4*>(y + (int64_t)rows[k] * d) + c);
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            part[k] = dot_bf16(part[k], g, v[k]);
+            if ((valid >> k) & 1u)
+                __stcs(reinterpret_cast<uint4*>(dy + (int64_t)rows[k] * d) + c, scaled_bf16(wk[k], g));
+        }
+    }
+    // dw: butterfly inside each warp, then the token's warps in order
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        float p = part[k];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(kFull, p, off);
+        if (lane == 0) s_part[warp][k] = p;
+    }
+    __syncthreads();
+    if (live && c < K && ((valid >> c) & 1u)) {
+        const int wpt = cw / 32;
+        float acc = 0.0f;
+        for (int ww = 0; ww < wpt; ++ww) acc += s_part[ww][c];
+        dw[n * K + c] = acc;
+    }
+    if (live && c == 0 && valid != kAll) {
+        const int k = __ffs(~valid & kAll) - 1;  // the first pair out of range
+        raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(n * K + k, (int64_t)INT_MAX));
+    }
+}
+
+// threads per CTA of the looping kernel, by the largest K (registers: K rows,
+// weights and partial dots, plus K 16-byte chunks in flight)
 template <int KMAX>
-__global__ void __launch_bounds__(kBwdThreads, KMAX <= 8 ? 3 : 1)
+__host__ __device__ constexpr int bwd_threads() { return KMAX <= 8 ? 512 : (KMAX <= 16 ? 256 : 128); }
+
+// Any other shape: a thread loops over its chunks of the row; any K <= KMAX.
+template <int KMAX>
+__global__ void __launch_bounds__(bwd_threads<KMAX>())
 combine_bwd_kernel(const float* __restrict__ dout, const uint16_t* __restrict__ y,
                    const int32_t* __restrict__ dest_row, const float* __restrict__ w,
                    uint16_t* __restrict__ dy, float* __restrict__ dw, int64_t N, int K, int d,
-                   int64_t Q, int* err)
+                   int cw, int64_t Q, int* err)
 {
+    constexpr int NT = bwd_threads<KMAX>();
+    __shared__ float s_part[NT / 32][KMAX];
     const int C = d >> 3;
+    const int tpc = NT / cw;               // tokens per CTA
+    const int sub = threadIdx.x / cw;      // the token within the CTA
+    const int lt = threadIdx.x - sub * cw; // the thread within the token's group
     const int lane = threadIdx.x & 31;
-    const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t n = gwarp; n < N; n += nwarps) {
-        int rows[KMAX];
-        float wk[KMAX], part[KMAX];
+    const int warp = threadIdx.x >> 5;
+    const int64_t n = (int64_t)blockIdx.x * tpc + sub;
+    const bool live = sub < tpc && n < N;
+    int rows[KMAX];
+    float wk[KMAX], part[KMAX];
 #pragma unroll
-        for (int k = 0; k < KMAX; ++k) {
-            rows[k] = -1;
-            wk[k] = 0.0f;
-            part[k] = 0.0f;
-            if (k < K) {
-                const int r = __ldg(dest_row + n * K + k);
-                if (r >= 0 && (int64_t)r < Q) {
-                    rows[k] = r;
-                    wk[k] = __ldg(w + n * K + k);
-                } else if (lane == 0) {
-                    raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(n * K + k, (int64_t)INT_MAX));
-                }
+    for (int k = 0; k < KMAX; ++k) {
+        rows[k] = -1;
+        wk[k] = 0.0f;
+        part[k] = 0.0f;
+        if (live && k < K) {
+            const int r = __ldg(dest_row + n * K + k);
+            if (r >= 0 && (int64_t)r < Q) {
+                rows[k] = r;
+                wk[k] = __ldg(w + n * K + k);
+            } else if (lt == 0) {
+                raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(n * K + k, (int64_t)INT_MAX));
             }
         }
-        const float4* g_row = reinterpret_cast<const float4*>(dout + n * d);
-        for (int c = lane; c < C; c += 32) {
-            const float4 g0 = __ldcs(g_row + 2 * c);
-            const float4 g1 = __ldcs(g_row + 2 * c + 1);
-            uint4 v[KMAX];
+    }
+    const float4* g_row = reinterpret_cast<const float4*>(dout + (live ? n : 0) * d);
+    for (int c = lt; live && c < C; c += cw) {
+        const float4 g0 = __ldcs(g_row + 2 * c);
+        const float4 g1 = __ldcs(g_row + 2 * c + 1);
+        uint4 v[KMAX];
 #pragma unroll
-            for (int k = 0; k < KMAX; ++k)
-                v[k] = rows[k] >= 0 ? __ldcs(reinterpret_cast<const uint4*>(y + (int64_t)rows[k] * d) + c)
-                                    : make_uint4(0u, 0u, 0u, 0u);
-            const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-            for (int k = 0; k < KMAX; ++k) {
-                if (rows[k] < 0) continue;
-                const uint32_t u[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    part[k] = fmaf(g[2 * q], __uint_as_float(u[q] << 16), part[k]);
-                    part[k] = fmaf(g[2 * q + 1], __uint_as_float(u[q] & 0xffff0000u), part[k]);
-                }
-                uint4 o;
-                o.x = pack_bf16x2(wk[k] * g[0], wk[k] * g[1]);
-                o.y = pack_bf16x2(wk[k] * g[2], wk[k] * g[3]);
-                o.z = pack_bf16x2(wk[k] * g[4], wk[k] * g[5]);
-                o.w = pack_bf16x2(wk[k] * g[6], wk[k] * g[7]);
-                __stcs(reinterpret_cast<uint4*>(dy + (int64_t)rows[k] * d) + c, o);
-            }
-        }
-        // dw: fixed butterfly over the warp; lane k writes dw[n][k]
-        float mine = 0.0f;
+        for (int k = 0; k < KMAX; ++k)
+            v[k] = rows[k] >= 0 ? __ldcs(reinterpret_cast<const uint4*>(y + (int64_t)rows[k] * d) + c)
+                                : make_uint4(0u, 0u, 0u, 0u);
+        const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
         for (int k = 0; k < KMAX; ++k) {
-            float p = part[k];
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(kFull, p, off);
-            if (lane == k) mine = p;
+            if (rows[k] < 0) continue;
+            part[k] = dot_bf16(part[k], g, v[k]);
+            __stcs(reinterpret_cast<uint4*>(dy + (int64_t)rows[k] * d) + c, scaled_bf16(wk[k], g));
         }
-        if (lane < K && lane < KMAX) {
-            // every lane holds the rows of all K pairs; pick pair (n, lane)'s
-            // without dynamic register indexing
-            int r_l = -1;
+    }
+    // dw: butterfly inside each warp, then the token's warps in order
 #pragma unroll
-            for (int k = 0; k < KMAX; ++k)
-                if (k == lane) r_l = rows[k];
-            if (r_l >= 0) dw[n * K + lane] = mine;
-        }
+    for (int k = 0; k < KMAX; ++k) {
+        float p = part[k];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(kFull, p, off);
+        if (lane == 0) s_part[warp][k] = p;
+    }
+    __syncthreads();
+    if (live && lt < K) {
+        const int wpt = cw / 32;
+        const int w0 = (sub * cw) / 32;
+        float acc = 0.0f;
+        for (int ww = 0; ww < wpt; ++ww) acc += s_part[w0 + ww][lt];
+        // every thread of the group holds the rows; pick pair (n, lt)'s
+        int r_l = -1;
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k)
+            if (k == lt) r_l = rows[k];
+        if (r_l >= 0) dw[n * K + lt] = acc;
     }
 }
 
 template <int KMAX>
-cudaError_t shape_k(const Sizes& z, int num_sms, int* grid)
+void shape_loop(const Sizes& z, BwdShape* out)
 {
-    int per_sm = 0;
-    cudaError_t ce = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_bwd_kernel<KMAX>,
-                                                                   kBwdThreads, 0);
-    if (ce != cudaSuccess) return ce;
-    per_sm = std::max(per_sm, 1);
-    const int64_t need = std::max<int64_t>(1, (z.N + kBwdWarps - 1) / kBwdWarps);
-    *grid = (int)std::min<int64_t>(need, (int64_t)num_sms * per_sm);
-    return cudaSuccess;
+    constexpr int NT = bwd_threads<KMAX>();
+    const int C = z.d / 8;
+    const int cw = std::min(((C + 31) / 32) * 32, NT);  // whole warps per token
+    const int tpc = NT / cw;
+    out->cw = cw;
+    out->threads = NT;
+    out->single = 0;
+    out->grid = (int)std::max<int64_t>(1, (z.N + tpc - 1) / tpc);
 }
 
 }  // namespace
 
-cudaError_t plan_combine_backward_grid(const Sizes& z, int num_sms, int* grid)
+cudaError_t plan_combine_backward_shape(const Sizes& z, BwdShape* out)
 {
-    if (z.K <= 4) return shape_k<4>(z, num_sms, grid);
-    if (z.K <= 8) return shape_k<8>(z, num_sms, grid);
-    if (z.K <= 16) return shape_k<16>(z, num_sms, grid);
-    return shape_k<32>(z, num_sms, grid);
+    const int C = z.d / 8;
+    if ((z.K == 4 || z.K == 8) && C <= 1024) {
+        // one chunk per thread, one token per CTA
+        const int cw = ((C + 31) / 32) * 32;
+        out->cw = cw;
+        out->threads = cw;
+        out->single = 1;
+        out->grid = (int)std::max<int64_t>(1, z.N);
+        return cudaSuccess;
+    }
+    if (z.K <= 4) shape_loop<4>(z, out);
+    else if (z.K <= 8) shape_loop<8>(z, out);
+    else if (z.K <= 16) shape_loop<16>(z, out);
+    else shape_loop<32>(z, out);
+    return cudaSuccess;
 }
 
-cudaError_t launch_combine_backward(const Sizes& z, const float* dout, const uint16_t* y,
-                                    const int32_t* dest_row, const float* w, uint16_t* dy,
-                                    float* dw, int grid, int* err, cudaStream_t st)
+cudaError_t launch_combine_backward(const Sizes& z, const BwdShape& sh, const float* dout,
+                                    const uint16_t* y, const int32_t* dest_row, const float* w,
+                                    uint16_t* dy, float* dw, int* err, cudaStream_t st)
 {
     if (z.N == 0) return cudaSuccess;
-#define UE_BWD(KM)                                                                              \
-    combine_bwd_kernel<KM><<<grid, kBwdThreads, 0, st>>>(dout, y, dest_row, w, dy, dw, z.N, z.K, \
-                                                         z.d, z.Q, err)
+    if (sh.single) {
+        if (z.K == 8)
+            combine_bwd_chunk_kernel<8><<<sh.grid, sh.cw, 0, st>>>(
+                dout, y, dest_row, w, dy, dw, z.N, z.d, sh.cw, z.Q, err);
+        else
+            combine_bwd_chunk_kernel<4><<<sh.grid, sh.cw, 0, st>>>(
+                dout, y, dest_row, w, dy, dw, z.N, z.d, sh.cw, z.Q, err);
+        return cudaGetLastError();
+    }
+#define UE_BWD(KM)                                                                               \
+    combine_bwd_kernel<KM><<<sh.grid, bwd_threads<KM>(), 0, st>>>(dout, y, dest_row, w, dy, dw,  \
+                                                                  z.N, z.K, z.d, sh.cw, z.Q, err)
     if (z.K <= 4) UE_BWD(4);
     else if (z.K <= 8) UE_BWD(8);
     else if (z.K <= 16) UE_BWD(16);

@@ -15,7 +15,7 @@ struct ue_ctx {
     int gate_grid;
     ue::PermuteShape perm;
     ue::CombineShape comb;
-    int bwd_grid;           // combine backward: CTAs of 8 token warps
+    ue::BwdShape bwd;       // combine backward launch shape
     int* d_err;             // [2] error code, detail
     unsigned long long* d_status;  // [tiles][E] reroute look-back words
     uint32_t* d_sync;       // [4] reroute ticket, finished CTAs, epoch
@@ -99,7 +99,7 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
 
     if (ue::plan_permute_shape(ctx->z, ctx->num_sms, &ctx->perm) != cudaSuccess ||
         ue::plan_combine_shape(ctx->z, ctx->num_sms, &ctx->comb) != cudaSuccess ||
-        ue::plan_combine_backward_grid(ctx->z, ctx->num_sms, &ctx->bwd_grid) != cudaSuccess ||
+        ue::plan_combine_backward_shape(ctx->z, &ctx->bwd) != cudaSuccess ||
         ue::plan_bisect_setup(ctx->z) != cudaSuccess) {
         delete ctx;
         cudaGetLastError();
@@ -301,8 +301,8 @@ ue_status ue_combine_backward(ue_ctx* ctx, const float* dout, const uint16_t* y,
         !aligned(w, 4) || !aligned(dy, 16) || !aligned(dw, 4))
         return UE_ERR_INVALID_ARG;
     if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
-    return from_cuda(ue::launch_combine_backward(ctx->z, dout, y, dest_row, w, dy, dw,
-                                                 ctx->bwd_grid, ctx->d_err, as_stream(stream)));
+    return from_cuda(ue::launch_combine_backward(ctx->z, ctx->bwd, dout, y, dest_row, w, dy, dw,
+                                                 ctx->d_err, as_stream(stream)));
 }
 
 ue_status ue_permute_backward(ue_ctx* ctx, const uint16_t* ddispatch, const int32_t* dest_row,

@@ -125,10 +125,14 @@ int gate_topk_grid(const Sizes& z, int num_sms);
 
 // Beside the forward path: backward of the combine (the permute's backward
 // is launch_combine with w == nullptr), weight sync and gradient reduction.
-cudaError_t plan_combine_backward_grid(const Sizes& z, int num_sms, int* grid);
-cudaError_t launch_combine_backward(const Sizes& z, const float* dout, const uint16_t* y,
-                                    const int32_t* dest_row, const float* w, uint16_t* dy,
-                                    float* dw, int grid, int* err, cudaStream_t st);
+struct BwdShape {
+    int grid, threads, cw;  // cw: threads per token (whole warps)
+    int single;             // 1: one chunk per thread (K = 4 or 8, d <= 8192)
+};
+cudaError_t plan_combine_backward_shape(const Sizes& z, BwdShape* out);
+cudaError_t launch_combine_backward(const Sizes& z, const BwdShape& sh, const float* dout,
+                                    const uint16_t* y, const int32_t* dest_row, const float* w,
+                                    uint16_t* dy, float* dw, int* err, cudaStream_t st);
 cudaError_t launch_weight_sync(const Sizes& z, const int32_t* slot_expert, const void* master,
                                void* replicas, int64_t bytes_per_expert, int num_sms, int* err,
                                cudaStream_t st);
