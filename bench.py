@@ -49,12 +49,11 @@ FALLBACK_HBM_GBS = 6650.0
 TRAFFIC = {
     "gate_topk": {"bytes_per_launch": 134720000, "source_sha": "2cf60b87ff02f365"},
     "count": {"bytes_per_launch": 8824000, "source_sha": "df378f26704dc1a3"},
-    "plan": {"bytes_per_launch": 25000, "source_sha": "594eef62c20fb78b"},
-    "reroute": {"bytes_per_launch": 8968000, "source_sha": "f685d38239dc3908"},
-    "permute": {"bytes_per_launch": 18881304000, "source_sha": "07222823ab0e9db7"},
-    "combine": {"bytes_per_launch": 21247792000, "source_sha": "0ebcc3caa2094612"},
+    "plan": {"bytes_per_launch": 29000, "source_sha": "2edfc203d9880067"},
+    "reroute": {"bytes_per_launch": 8968000, "source_sha": "237f5cbb848c661f"},
+    "permute": {"bytes_per_launch": 18890168000, "source_sha": "07222823ab0e9db7"},
+    "combine": {"bytes_per_launch": 21243824000, "source_sha": "0ebcc3caa2094612"},
 }
-
 
 def sha_of(path):
     with open(path, "rb") as f:
