@@ -47,7 +47,7 @@ FALLBACK_HBM_GBS = 6650.0
 # prefix of the kernel source it was taken on; a kernel changed since then
 # reports null.
 TRAFFIC = {
-    "gate_topk": {"bytes_per_launch": 134720000, "source_sha": "2cf60b87ff02f365"},
+    "gate_topk": {"bytes_per_launch": 134480000, "source_sha": "f9c2f7be091df85a"},
     "count": {"bytes_per_launch": 8824000, "source_sha": "df378f26704dc1a3"},
     "plan": {"bytes_per_launch": 29000, "source_sha": "2edfc203d9880067"},
     "reroute": {"bytes_per_launch": 8968000, "source_sha": "237f5cbb848c661f"},

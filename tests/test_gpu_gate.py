@@ -1,0 +1,100 @@
+"""GPU parity of the gate's two selection paths for K = 8 and E = 128 or 256.
+
+The fast path ranks packed keys (an order key whose low log2(E) bits carry
+the expert id) and re-selects, with full keys and the lower-id tie rule, every
+row whose first K+1 picks are not separated above the dropped bits. These
+tests mix, inside the same warp groups of four rows, rows of distinct normal
+logits (packed picks kept), rows of exact ties and signed zeros, and rows of
+values a few fp32 ulps apart (both re-selected), with a ragged last group.
+Both paths must give the oracle's ids bit for bit and its weights within one
+fp32 ulp; a logits buffer that is not 16-byte aligned takes the generic
+kernel, which must agree as well.
+
+"UltraEP" README, "Interface / 2. Forward and backward" (probs, routing_map
+from the router); "What Happened" (routing from the exact probabilities).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import token_rerouting_b200 as ue
+from tests import gpu_helpers as gh
+
+pytestmark = pytest.mark.gpu
+
+
+def mixed_logits(N, E, seed):
+    rng = np.random.default_rng(seed)
+    out = rng.standard_normal((N, E)).astype(np.float32)
+    kind = rng.integers(0, 4, size=N)
+    ties = np.array([-1.0, -0.0, 0.0, 0.5, 1.0], dtype=np.float32)
+    t_rows = kind == 1
+    out[t_rows] = ties[rng.integers(0, len(ties), size=(int(t_rows.sum()), E))]
+    c_rows = kind == 2
+    steps = rng.integers(0, 200, size=(int(c_rows.sum()), E)).astype(np.float64)
+    out[c_rows] = (1.0 + steps * 2.0 ** -23).astype(np.float32)
+    # kind 3: normal rows whose two leaders sit one ulp apart
+    n_rows = np.flatnonzero(kind == 3)
+    lead = np.argmax(out[n_rows], axis=1)
+    other = (lead + 1 + rng.integers(0, E - 1, size=len(n_rows))) % E
+    top = out[n_rows, lead]
+    out[n_rows, other] = np.nextafter(top, np.float32(-np.inf))
+    return out
+
+
+def run_gate(E, N, logits, offset_floats=0):
+    R = 2 if N % 2 == 0 else 1
+    T = N // R
+    K = 8
+    dev = torch.device("cuda", 0)
+    cfg = ue.make_config(R, T, E, K, 1, 8)
+    ctx = ue.ue_init(cfg, 0)
+    try:
+        buf = torch.empty(N * E + offset_floats, dtype=torch.float32, device=dev)
+        lg = buf[offset_floats:]
+        lg.copy_(torch.from_numpy(np.ascontiguousarray(logits).ravel()))
+        idx = torch.full((N, K), -7, dtype=torch.int32, device=dev)
+        w = torch.full((N, K), -1.0, dtype=torch.float32, device=dev)
+        ue.ue_gate_topk(ctx, lg, idx, w)
+        assert ue.ue_get_error(ctx) == ue.UE_OK
+        torch.cuda.synchronize()
+        return idx.cpu().numpy(), w.cpu().numpy()
+    finally:
+        ue.ue_destroy(ctx)
+
+
+@pytest.mark.parametrize("E", [128, 256])
+@pytest.mark.parametrize("N", [2002, 4099])
+def test_packed_and_exact_rows_in_one_group(E, N):
+    gh.ensure_built()
+    logits = mixed_logits(N, E, seed=E + N)
+    idx_or, w_or = oracle.gate_topk(logits, 8)
+    idx, w = run_gate(E, N, logits)
+    np.testing.assert_array_equal(idx, idx_or)
+    gh.assert_weights_close(w, w_or)
+
+
+@pytest.mark.parametrize("E", [128, 256])
+def test_unaligned_logits_take_the_generic_kernel(E):
+    gh.ensure_built()
+    N = 1030
+    logits = mixed_logits(N, E, seed=3 * E)
+    idx_or, w_or = oracle.gate_topk(logits, 8)
+    idx_a, w_a = run_gate(E, N, logits, offset_floats=0)
+    idx_u, w_u = run_gate(E, N, logits, offset_floats=1)
+    np.testing.assert_array_equal(idx_a, idx_or)
+    np.testing.assert_array_equal(idx_u, idx_or)
+    gh.assert_weights_close(w_a, w_or)
+    gh.assert_weights_close(w_u, w_or)
+    np.testing.assert_array_equal(w_a, w_u)
+
+
+def test_all_rows_equal_pick_the_lowest_ids():
+    gh.ensure_built()
+    N, E = 37, 256
+    logits = np.zeros((N, E), dtype=np.float32)
+    logits[1::3] = -0.0
+    idx, w = run_gate(E, N, logits)
+    assert (idx == np.arange(8)).all()
+    assert (w == np.float32(1.0 / 8)).all()
