@@ -362,8 +362,9 @@ def run_row(args, w):
     ue_build.build()
     dev = torch.device("cuda", 0)
     gen = torch.Generator(device=dev).manual_seed(0)
-    L = ue.Layer(w.R, w.T, w.E, w.K, w.S, w.d if args.row == "backward" else 8, device=0,
-                 with_rows=False)
+    rows_d = w.d if args.row in ("backward", "permute_patterns") else 8
+    L = ue.Layer(w.R, w.T, w.E, w.K, w.S, rows_d, device=0,
+                 with_rows=args.row == "permute_patterns")
     L.logits.copy_(torch.from_numpy(synth_logits(w)))
     L.run_routing()
     torch.cuda.synchronize(dev)
@@ -395,6 +396,34 @@ def run_row(args, w):
         kernels["combine_backward"] = (t1, 4 * N * d + 2 * Q * d + 8 * Q + 2 * Q * d + 4 * Q)
         kernels["permute_backward"] = (t2, 2 * Q * d + 4 * Q + 4 * N * d)
         workload = dict(workload=w.name, N=N, K=K, d=d, pairs=Q)
+    elif args.row == "permute_patterns":
+        # the permute's traffic (2Nd read, 2Qd written) under three row
+        # layouts, beside write-only and 1:1-copy traffic of torch's own
+        # kernels: where the routed layout stands between the best and the
+        # worst placement of the same bytes
+        N, K, d, Q = w.N, w.K, w.d, w.Q
+        L.hidden.copy_(torch.randint(-30000, 30000, (N, d), dtype=torch.int16, device=dev,
+                                     generator=gen).view(torch.bfloat16))
+        ident = torch.arange(Q, dtype=torch.int32, device=dev).view(N, K)
+        rand = torch.randperm(Q, device=dev, generator=gen).to(torch.int32).view(N, K)
+        pbytes = 2 * N * d + 2 * Q * d + 4 * Q
+        kernels["permute_routed"] = (timed(lambda: L.permute(st)), pbytes)
+        kernels["permute_contiguous_rows"] = (
+            timed(lambda: ue.ue_permute(L.ctx, L.hidden, ident, L.dispatch, st)), pbytes)
+        kernels["permute_random_rows"] = (
+            timed(lambda: ue.ue_permute(L.ctx, L.hidden, rand, L.dispatch, st)), pbytes)
+        flat = L.dispatch.view(-1)
+        half = flat.numel() // 2
+        flat64 = flat[:flat.numel() // 4 * 4].view(torch.int64)
+        kernels["torch_fill_write_only"] = (timed(lambda: flat64.fill_(0x3F803F803F803F80)),
+                                            8 * flat64.numel())
+        kernels["torch_copy_1to1"] = (timed(lambda: flat[half:2 * half].copy_(flat[:half])),
+                                      4 * half)
+        del ident, rand
+        workload = dict(workload=w.name, N=N, K=K, d=d, pairs=Q,
+                        routed=("dest_row of the path's reroute: per-slot runs, 4*P regions "
+                                "written at once"),
+                        contiguous="dest_row = n*K + k", random="a random permutation of [0, Q)")
     else:
         plan = L.plan_arrays()
         se = plan["slot_expert"]
@@ -427,7 +456,8 @@ def run_row(args, w):
     for k, (t, by) in kernels.items():
         gbs = by / t / 1e9
         out[k] = {"us": t * 1e6, "algorithmic_bytes": by, "gbs": gbs, "frac_of_peak": gbs / peak}
-    dom = max(out, key=lambda k: out[k]["us"])
+    dom = ("permute_routed" if args.row == "permute_patterns"
+           else max(out, key=lambda k: out[k]["us"]))
     line = {"row": args.row, "config": workload, "steps": args.steps, "kernels": out,
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": out[dom]["gbs"], "peak": peak,
                          "unit": "GB/s", "frac": out[dom]["frac_of_peak"],
@@ -458,6 +488,15 @@ def row_oracle_baseline(args, w, slot_expert):
         by = (4 * n * d + 2 * n * K * d + 8 * n * K + 2 * n * K * d + 4 * n * K) + \
              (2 * n * K * d + 4 * n * K + 4 * n * d)
         sample = f"{n} tokens x K={K} x d={d}: combine backward + permute backward"
+    elif args.row == "permute_patterns":
+        n, K, d = 8192, w.K, w.d
+        dest = np.random.default_rng(0).permutation(n * K).astype(np.int32).reshape(n, K)
+        hidden = synth.bf16_normal(n, d, 0, 63)
+        t0 = time.perf_counter()
+        oracle.permute(hidden, K, dest)
+        secs = time.perf_counter() - t0
+        by = 2 * n * d + 2 * n * K * d + 4 * n * K
+        sample = f"{n} tokens x K={K} x d={d}: permute with random rows"
     else:
         numel = expert_numel(args)
         used = [g for g in range(len(slot_expert)) if slot_expert[g] >= 0][:8]
@@ -630,7 +669,8 @@ def main():
                     help="the 48 x 8 non-stationary sweep, CUDA-graph captured")
     ap.add_argument("--planner", choices=("greedy", "bisect"), default="greedy",
                     help="planner of the sweep (greedy: the path's rule)")
-    ap.add_argument("--row", choices=("backward", "weight_sync", "grad_reduce", "planner"),
+    ap.add_argument("--row", choices=("backward", "weight_sync", "grad_reduce", "planner",
+                                      "permute_patterns"),
                     default=None, help="measure one of the rows beside the forward path "
                     "(planner: the planner variants, on pages_ep64_e256_t8k by default)")
     args = ap.parse_args()

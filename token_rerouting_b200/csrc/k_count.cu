@@ -9,10 +9,11 @@
 // them in shared memory, one private histogram per warp so that a hot expert
 // contends only within a warp; shared-memory atomics resolve the rest. Each
 // CTA then adds its non-zero bins to the outputs (zeroed on the stream
-// first) with one global atomic per bin. Chunks are large (16384 pairs), so
-// few CTAs contend for each bin of load_e. Every thread issues all its loads
-// before it counts. Integer sums are exact, so the result does not depend on
-// the order of the additions.
+// first) with one global atomic per bin. Chunks of 4096 pairs give a few
+// CTAs per SM (512 on the Qwen3-shaped layer), so the kernel's length is a
+// few load and atomic latencies; each bin of load_e takes one atomic per
+// CTA. Every thread issues all its loads before it counts. Integer sums are
+// exact, so the result does not depend on the order of the additions.
 #include "ue_internal.cuh"
 
 namespace ue {
@@ -20,7 +21,7 @@ namespace {
 
 constexpr int kCountThreads = 512;
 constexpr int kCountWarps = kCountThreads / 32;
-constexpr int kCountChunk = 16384;  // pairs per CTA (few CTAs add into each bin)
+constexpr int kCountChunk = 4096;  // pairs per CTA
 
 template <bool VEC>
 __global__ void __launch_bounds__(kCountThreads)
