@@ -723,6 +723,12 @@ def main():
     L = ue.Layer(w.R, w.T, w.E, w.K, w.S, w.d, device=local)
     L.logits.copy_(torch.from_numpy(logits_h))
     L.hidden.copy_(torch.from_numpy(hidden_h.view(np.int16)).to(dev).view(torch.bfloat16))
+    # a second layer instance (the next microbatch): the timed steps alternate
+    # between the two, so that one instance's routing runs while the other
+    # permutes and combines
+    LB = ue.Layer(w.R, w.T, w.E, w.K, w.S, w.d, device=local)
+    LB.logits.copy_(torch.from_numpy(synth.logits(w, mb=rank + world)))
+    LB.hidden.copy_(L.hidden)
     stream = torch.cuda.current_stream(dev)
 
     steps_fn = [L.gate, L.count, L.plan_step, L.reroute, L.permute, L.combine]
@@ -731,12 +737,42 @@ def main():
         for f in steps_fn:
             f(stream=stream)
 
+    # Pipelined steps: step i runs on instance i % 2. Its routing (gate,
+    # count, plan, reroute) goes on a side stream once step i-2's combine has
+    # released the instance; its permute and combine go on the main stream
+    # once its routing is done. So step i+1's routing overlaps step i's
+    # permute and combine, as the pages' asynchronous update_placement and
+    # reroute (events, current_stream_wait) allow; the first step's routing
+    # overlaps nothing.
+    insts = [L, LB]
+    side = torch.cuda.Stream(dev)
+    ev_routed = [torch.cuda.Event() for _ in insts]
+    ev_done = [torch.cuda.Event() for _ in insts]
+
+    def pipelined_steps(n):
+        for x in range(2):
+            ev_done[x].record(stream)
+        for i in range(n):
+            x = i % 2
+            I = insts[x]
+            side.wait_event(ev_done[x])
+            for f in (I.gate, I.count, I.plan_step, I.reroute):
+                f(stream=side)
+            ev_routed[x].record(side)
+            stream.wait_event(ev_routed[x])
+            I.permute(stream=stream)
+            I.combine(stream=stream)
+            ev_done[x].record(stream)
+
     for _ in range(args.warmup):
         step()
+    pipelined_steps(max(4, args.warmup))
     torch.cuda.synchronize(dev)
-    rc = L.error(stream)
+    rc = L.error(stream) or LB.error(stream)
     if rc != 0:
         raise SystemExit(f"device error after warm-up: {ue.STATUS.get(rc, rc)}")
+    step()
+    torch.cuda.synchronize(dev)
     plan0 = L.plan_arrays()
 
     # the step as one CUDA graph of the six kernels (captured once, outside
@@ -764,16 +800,31 @@ def main():
     torch.cuda.synchronize(dev)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for s in range(args.steps):
-        graph.replay()
+    pipelined_steps(args.steps)
     end.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     total_ms = start.elapsed_time(end)
-    rc = L.error(stream)
+    rc = L.error(stream) or LB.error(stream)
     if rc != 0:
         raise SystemExit(f"device error in the timed region: {ue.STATUS.get(rc, rc)}")
+
+    # the same steps one after another, each one graph replay of the six
+    # kernels on one instance (reported beside the value)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    sa, sb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sa.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    sb.record(stream)
+    torch.cuda.synchronize(dev)
+    serial_ms = max_over_ranks(sa.elapsed_time(sb) / args.steps, world, dev)
+    rc = L.error(stream)
+    if rc != 0:
+        raise SystemExit(f"device error in the serial steps: {ue.STATUS.get(rc, rc)}")
 
     # per-kernel breakdown from eager launches bracketed by events (not part
     # of the value): ev[s][k] .. ev[s][k+1] brackets kernel k of step s
@@ -824,8 +875,13 @@ def main():
     gate_to_permute = sum(per_kernel_ms[k] for k in KERNELS[:5])
     cfg.update(us_per_layer_gate_to_permute=1e3 * gate_to_permute,
                us_per_layer_incl_combine=1e3 * sum(per_kernel_ms.values()),
-               timing="each timed step replays one CUDA graph of the six kernels; per-kernel "
-                      "times from eager launches bracketed by CUDA events",
+               timing="exactly `steps` steps, each the six kernels over one batch; two layer "
+                      "instances alternate, and step i+1's routing (gate, count, plan, reroute) "
+                      "runs on a second stream during step i's permute and combine (events "
+                      "order each instance's uses); per-kernel times from eager launches "
+                      "bracketed by CUDA events",
+               ms_per_step_serial=serial_ms,
+               serial="the same steps one after another, one CUDA graph replay each",
                parallelism=f"replicas: {world} independent layer instance(s), one per GPU")
 
     # end to end through the public API with host buffers. Every step copies
@@ -839,7 +895,7 @@ def main():
     if not args.no_e2e:
         lg_pin = torch.from_numpy(logits_h).pin_memory()
         hd_pin = torch.from_numpy(hidden_h.view(np.int16)).pin_memory()
-        L2 = ue.Layer(w.R, w.T, w.E, w.K, w.S, w.d, device=local)
+        L2 = LB
         bufs = [L, L2]
         outs = [torch.empty(L.out.shape, dtype=torch.float32).pin_memory() for _ in bufs]
         stats_pin = [torch.empty(4 + w.R, dtype=torch.int32).pin_memory() for _ in bufs]
@@ -885,7 +941,6 @@ def main():
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(a.elapsed_time(b_) / args.e2e_steps, world, dev)
         rc2 = L2.error(s_run) or L.error(s_run)
-        L2.close()
         if rc2 != 0:
             raise SystemExit(f"device error in the end-to-end steps: {ue.STATUS.get(rc2, rc2)}")
         h2d = lg_pin.numel() * 4 + hd_pin.numel() * 2
@@ -921,6 +976,7 @@ def main():
         }
         print(json.dumps(line), flush=True)
     L.close()
+    LB.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
