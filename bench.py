@@ -47,8 +47,8 @@ FALLBACK_HBM_GBS = 6650.0
 # prefix of the kernel source it was taken on; a kernel changed since then
 # reports null.
 TRAFFIC = {
-    "gate_topk": {"bytes_per_launch": 134480000, "source_sha": "f9c2f7be091df85a"},
-    "count": {"bytes_per_launch": 8824000, "source_sha": "df378f26704dc1a3"},
+    "gate_topk": {"bytes_per_launch": 134520000, "source_sha": "f9c2f7be091df85a"},
+    "count": {"bytes_per_launch": 8728000, "source_sha": "dda54be050ff39f0"},
     "plan": {"bytes_per_launch": 29000, "source_sha": "2edfc203d9880067"},
     "reroute": {"bytes_per_launch": 8968000, "source_sha": "237f5cbb848c661f"},
     "permute": {"bytes_per_launch": 18890168000, "source_sha": "07222823ab0e9db7"},
