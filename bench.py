@@ -745,7 +745,10 @@ def main():
     # reroute (events, current_stream_wait) allow; the first step's routing
     # overlaps nothing.
     insts = [L, LB]
-    side = torch.cuda.Stream(dev)
+    # the routing's stream has the higher priority: its few CTAs are placed
+    # ahead of the permute's pending ones, so it holds SM slots for a shorter
+    # time (measured: 6.353 against 6.375 ms per step at equal priority)
+    side = torch.cuda.Stream(dev, priority=-5)
     ev_routed = [torch.cuda.Event() for _ in insts]
     ev_done = [torch.cuda.Event() for _ in insts]
 
