@@ -21,6 +21,7 @@ struct ue_ctx {
     uint32_t* d_sync;       // [4] reroute ticket, finished CTAs, epoch
     int32_t* d_first;       // [R][P] locality order: first occurrence index
     int32_t* d_rowb;        // [R][P] locality order: row base
+    uint16_t* d_zrow;       // [d] zeros: the combine reads it for a row out of range
     int64_t tiles;
     int64_t spin_limit;
     int drop_first;
@@ -112,12 +113,14 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
         cudaMalloc(&ctx->d_status, status_words * sizeof(unsigned long long)) != cudaSuccess ||
         cudaMalloc(&ctx->d_sync, 4 * sizeof(uint32_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_first, table_words * sizeof(int32_t)) != cudaSuccess ||
-        cudaMalloc(&ctx->d_rowb, table_words * sizeof(int32_t)) != cudaSuccess) {
+        cudaMalloc(&ctx->d_rowb, table_words * sizeof(int32_t)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_zrow, (size_t)ctx->z.d * sizeof(uint16_t)) != cudaSuccess) {
         cudaFree(ctx->d_err);
         cudaFree(ctx->d_status);
         cudaFree(ctx->d_sync);
         cudaFree(ctx->d_first);
         cudaFree(ctx->d_rowb);
+        cudaFree(ctx->d_zrow);
         delete ctx;
         cudaGetLastError();
         return UE_ERR_NOMEM;
@@ -125,12 +128,14 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
     if (cudaMemset(ctx->d_err, 0, 2 * sizeof(int)) != cudaSuccess ||
         cudaMemset(ctx->d_status, 0, status_words * sizeof(unsigned long long)) != cudaSuccess ||
         cudaMemset(ctx->d_sync, 0, 4 * sizeof(uint32_t)) != cudaSuccess ||
+        cudaMemset(ctx->d_zrow, 0, (size_t)ctx->z.d * sizeof(uint16_t)) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess) {
         cudaFree(ctx->d_err);
         cudaFree(ctx->d_status);
         cudaFree(ctx->d_sync);
         cudaFree(ctx->d_first);
         cudaFree(ctx->d_rowb);
+        cudaFree(ctx->d_zrow);
         delete ctx;
         return UE_ERR_CUDA;
     }
@@ -150,6 +155,7 @@ ue_status ue_destroy(ue_ctx* ctx)
     cudaFree(ctx->d_sync);
     cudaFree(ctx->d_first);
     cudaFree(ctx->d_rowb);
+    cudaFree(ctx->d_zrow);
     ctx->magic = 0;
     delete ctx;
     return st;
@@ -289,8 +295,8 @@ ue_status ue_combine(ue_ctx* ctx, const uint16_t* y, const int32_t* dest_row, co
         !aligned(out, 16))
         return UE_ERR_INVALID_ARG;
     if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
-    return from_cuda(ue::launch_combine(ctx->z, ctx->comb, y, dest_row, w, out, ctx->d_err,
-                                        as_stream(stream)));
+    return from_cuda(ue::launch_combine(ctx->z, ctx->comb, y, dest_row, w, out, ctx->d_zrow,
+                                        ctx->d_err, as_stream(stream)));
 }
 
 ue_status ue_combine_backward(ue_ctx* ctx, const float* dout, const uint16_t* y,
@@ -314,7 +320,7 @@ ue_status ue_permute_backward(ue_ctx* ctx, const uint16_t* ddispatch, const int3
     if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
     // the combine with every weight equal to 1
     return from_cuda(ue::launch_combine(ctx->z, ctx->comb, ddispatch, dest_row, nullptr, dhidden,
-                                        ctx->d_err, as_stream(stream)));
+                                        ctx->d_zrow, ctx->d_err, as_stream(stream)));
 }
 
 ue_status ue_weight_sync(ue_ctx* ctx, const ue_placement* plan, const void* master,

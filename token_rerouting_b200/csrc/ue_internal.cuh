@@ -110,6 +110,7 @@ struct PermuteShape {
 };
 struct CombineShape {
     int grid, tpt;
+    int token;  // 1: one token per CTA, one chunk per thread (K = 4 or 8, 1024 <= d <= 8192)
 };
 cudaError_t plan_permute_shape(const Sizes& z, int num_sms, PermuteShape* out);
 cudaError_t plan_combine_shape(const Sizes& z, int num_sms, CombineShape* out);
@@ -117,9 +118,10 @@ cudaError_t plan_combine_shape(const Sizes& z, int num_sms, CombineShape* out);
 cudaError_t launch_permute(const Sizes& z, const PermuteShape& sh, const uint16_t* hidden,
                            const int32_t* dest_row, uint16_t* dispatch, int* err,
                            cudaStream_t st);
+// zrow: d zero bf16 values (16-byte aligned), read in place of a row out of range
 cudaError_t launch_combine(const Sizes& z, const CombineShape& sh, const uint16_t* y,
-                           const int32_t* dest_row, const float* w, float* out, int* err,
-                           cudaStream_t st);
+                           const int32_t* dest_row, const float* w, float* out,
+                           const uint16_t* zrow, int* err, cudaStream_t st);
 
 int gate_topk_grid(const Sizes& z, int num_sms);
 
