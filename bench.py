@@ -362,9 +362,9 @@ def run_row(args, w):
     ue_build.build()
     dev = torch.device("cuda", 0)
     gen = torch.Generator(device=dev).manual_seed(0)
-    rows_d = w.d if args.row in ("backward", "permute_patterns") else 8
+    rows_d = w.d if args.row in ("backward", "layouts") else 8
     L = ue.Layer(w.R, w.T, w.E, w.K, w.S, rows_d, device=0,
-                 with_rows=args.row == "permute_patterns")
+                 with_rows=args.row == "layouts")
     L.logits.copy_(torch.from_numpy(synth_logits(w)))
     L.run_routing()
     torch.cuda.synchronize(dev)
@@ -396,7 +396,7 @@ def run_row(args, w):
         kernels["combine_backward"] = (t1, 4 * N * d + 2 * Q * d + 8 * Q + 2 * Q * d + 4 * Q)
         kernels["permute_backward"] = (t2, 2 * Q * d + 4 * Q + 4 * N * d)
         workload = dict(workload=w.name, N=N, K=K, d=d, pairs=Q)
-    elif args.row == "permute_patterns":
+    elif args.row == "layouts":
         # the permute's traffic (2Nd read, 2Qd written) under three row
         # layouts, beside write-only and 1:1-copy traffic of torch's own
         # kernels: where the routed layout stands between the best and the
@@ -419,6 +419,18 @@ def run_row(args, w):
                                             8 * flat64.numel())
         kernels["torch_copy_1to1"] = (timed(lambda: flat[half:2 * half].copy_(flat[:half])),
                                       4 * half)
+        # the combine's gather (2Qd read, 4Nd written) under the same layouts,
+        # reading the dispatch buffer as the expert outputs, beside torch's
+        # read-only sum of the same 17.2 GB
+        cbytes = 2 * Q * d + 8 * Q + 4 * N * d
+        kernels["combine_routed"] = (timed(lambda: L.combine(stream=st)), cbytes)
+        kernels["combine_contiguous_rows"] = (
+            timed(lambda: ue.ue_combine(L.ctx, L.dispatch, ident, L.w, L.out, st)), cbytes)
+        kernels["combine_random_rows"] = (
+            timed(lambda: ue.ue_combine(L.ctx, L.dispatch, rand, L.w, L.out, st)), cbytes)
+        acc = torch.empty((), dtype=torch.int64, device=dev)
+        kernels["torch_sum_read_only"] = (timed(lambda: torch.sum(flat64, dim=0, out=acc)),
+                                          8 * flat64.numel())
         del ident, rand
         workload = dict(workload=w.name, N=N, K=K, d=d, pairs=Q,
                         routed=("dest_row of the path's reroute: per-slot runs, 4*P regions "
@@ -456,7 +468,7 @@ def run_row(args, w):
     for k, (t, by) in kernels.items():
         gbs = by / t / 1e9
         out[k] = {"us": t * 1e6, "algorithmic_bytes": by, "gbs": gbs, "frac_of_peak": gbs / peak}
-    dom = ("permute_routed" if args.row == "permute_patterns"
+    dom = ("permute_routed" if args.row == "layouts"
            else max(out, key=lambda k: out[k]["us"]))
     line = {"row": args.row, "config": workload, "steps": args.steps, "kernels": out,
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": out[dom]["gbs"], "peak": peak,
@@ -488,7 +500,7 @@ def row_oracle_baseline(args, w, slot_expert):
         by = (4 * n * d + 2 * n * K * d + 8 * n * K + 2 * n * K * d + 4 * n * K) + \
              (2 * n * K * d + 4 * n * K + 4 * n * d)
         sample = f"{n} tokens x K={K} x d={d}: combine backward + permute backward"
-    elif args.row == "permute_patterns":
+    elif args.row == "layouts":
         n, K, d = 8192, w.K, w.d
         dest = np.random.default_rng(0).permutation(n * K).astype(np.int32).reshape(n, K)
         hidden = synth.bf16_normal(n, d, 0, 63)
@@ -670,7 +682,7 @@ def main():
     ap.add_argument("--planner", choices=("greedy", "bisect"), default="greedy",
                     help="planner of the sweep (greedy: the path's rule)")
     ap.add_argument("--row", choices=("backward", "weight_sync", "grad_reduce", "planner",
-                                      "permute_patterns"),
+                                      "layouts"),
                     default=None, help="measure one of the rows beside the forward path "
                     "(planner: the planner variants, on pages_ep64_e256_t8k by default)")
     args = ap.parse_args()
