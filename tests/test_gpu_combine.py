@@ -5,7 +5,9 @@ the same kernel with unit weights.
 Cases: both K, the narrowest and the widest rows the kernel takes (d = 1024
 and d = 8192), rows out of range (they contribute nothing and set
 UE_ERR_DEVICE_BOUNDS), and a dest_row buffer that is not 16-byte aligned,
-which takes the persistent kernel and must give the same bits.
+which takes the persistent kernel and must give the same bits. The combine's
+backward, which loads a token's indices and weights as vectors only when
+both buffers are 16-byte aligned, must also give the same bits either way.
 
 Tolerance (the combine's, from its arithmetic): K fused multiply-adds into
 an fp32 sum starting from 0, k ascending, and the rounding of each w_k to
@@ -111,3 +113,35 @@ def test_unaligned_rows_take_the_persistent_kernel(K):
     assert rc_a == ue.UE_OK and rc_u == ue.UE_OK
     np.testing.assert_array_equal(out_a.view(np.uint32), out_u.view(np.uint32))
     np.testing.assert_array_equal(dh_a.view(np.uint32), dh_u.view(np.uint32))
+
+
+@pytest.mark.parametrize("K", [4, 8])
+def test_combine_backward_unaligned_rows_give_the_same_bits(K):
+    """The combine's backward loads a token's indices and weights as vectors
+    when dest_row and w are 16-byte aligned, one by one otherwise."""
+    gh.ensure_built()
+    N, d = 150, 2048
+    dest, w, y = inputs(N, K, d, seed=500 + K)
+    dout = synth.normal_f32(N * d, 7, 44).reshape(N, d)
+    L = gh.make_layer(1, N, K, K, 1, d, with_rows=False)
+    try:
+        dev = L.device
+        y_t = gh.bf16_to_device(y, dev)
+        dout_t = torch.from_numpy(dout).to(dev)
+        res = []
+        for off in (0, 1):
+            dbuf = torch.zeros(N * K + off, dtype=torch.int32, device=dev)
+            wbuf = torch.zeros(N * K + off, dtype=torch.float32, device=dev)
+            dest_t = dbuf[off:].view(N, K)
+            w_t = wbuf[off:].view(N, K)
+            dest_t.copy_(torch.from_numpy(dest))
+            w_t.copy_(torch.from_numpy(w))
+            dy = torch.zeros_like(y_t)
+            dw = torch.zeros((N, K), dtype=torch.float32, device=dev)
+            ue.ue_combine_backward(L.ctx, dout_t, y_t, dest_t, w_t, dy, dw)
+            assert L.error() == ue.UE_OK
+            res.append((gh.bf16_to_host_u16(dy), dw.cpu().numpy()))
+        np.testing.assert_array_equal(res[0][0], res[1][0])
+        np.testing.assert_array_equal(res[0][1].view(np.uint32), res[1][1].view(np.uint32))
+    finally:
+        L.close()

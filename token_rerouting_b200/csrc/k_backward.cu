@@ -64,9 +64,12 @@ __device__ __forceinline__ float dot_bf16(float part, const float (&g)[8], uint4
 }
 
 // One chunk per thread, K known at compile time (4 or 8), d <= 8192: one
-// token per CTA, blockDim = cw = the row's chunks rounded up to whole warps. A row out of range is only masked: its loads read row 0, which is
-// in range, it stores nothing, and the error is recorded after the work.
-template <int K>
+// token per CTA, blockDim = cw = the row's chunks rounded up to whole warps.
+// A row out of range is only masked: its loads read row 0, which is in range,
+// it stores nothing, and the error is recorded after the work. VEC: dest_row
+// and w are 16-byte aligned, and the token's K indices and weights arrive as
+// K/4 vector loads each.
+template <int K, bool VEC>
 __global__ void __launch_bounds__(1024)
 combine_bwd_chunk_kernel(const float* __restrict__ dout, const uint16_t* __restrict__ y,
                          const int32_t* __restrict__ dest_row, const float* __restrict__ w,
@@ -84,13 +87,37 @@ combine_bwd_chunk_kernel(const float* __restrict__ dout, const uint16_t* __restr
     int rows[K];
     float wk[K], part[K];
     unsigned valid = 0u;  // pairs with a row in range
+    if (VEC) {
+#pragma unroll
+        for (int h = 0; h < K / 4; ++h) {
+            int4 r4 = make_int4(0, 0, 0, 0);
+            float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (live) {
+                r4 = __ldg(reinterpret_cast<const int4*>(dest_row + n * K) + h);
+                w4 = __ldg(reinterpret_cast<const float4*>(w + n * K) + h);
+            }
+            rows[4 * h] = r4.x;
+            rows[4 * h + 1] = r4.y;
+            rows[4 * h + 2] = r4.z;
+            rows[4 * h + 3] = r4.w;
+            wk[4 * h] = w4.x;
+            wk[4 * h + 1] = w4.y;
+            wk[4 * h + 2] = w4.z;
+            wk[4 * h + 3] = w4.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            rows[k] = live ? __ldg(dest_row + n * K + k) : 0;
+            wk[k] = live ? __ldg(w + n * K + k) : 0.0f;
+        }
+    }
 #pragma unroll
     for (int k = 0; k < K; ++k) {
-        const int r = live ? __ldg(dest_row + n * K + k) : 0;
+        const int r = rows[k];
         const bool ok = (unsigned long long)(unsigned)r < (unsigned long long)Q;  // r >= 0 && r < Q
         rows[k] = ok ? r : 0;
         valid |= ok ? (1u << k) : 0u;
-        wk[k] = live ? __ldg(w + n * K + k) : 0.0f;
         part[k] = 0.0f;
     }
     if (live && c < C) {
@@ -250,12 +277,16 @@ cudaError_t launch_combine_backward(const Sizes& z, const BwdShape& sh, const fl
 {
     if (z.N == 0) return cudaSuccess;
     if (sh.single) {
-        if (z.K == 8)
-            combine_bwd_chunk_kernel<8><<<sh.grid, sh.cw, 0, st>>>(
-                dout, y, dest_row, w, dy, dw, z.N, z.d, sh.cw, z.Q, err);
-        else
-            combine_bwd_chunk_kernel<4><<<sh.grid, sh.cw, 0, st>>>(
-                dout, y, dest_row, w, dy, dw, z.N, z.d, sh.cw, z.Q, err);
+        const bool vec = ((reinterpret_cast<uintptr_t>(dest_row) |
+                           reinterpret_cast<uintptr_t>(w)) & 15u) == 0;
+#define UE_BWD_CHUNK(KK, V)                                                                      \
+    combine_bwd_chunk_kernel<KK, V><<<sh.grid, sh.cw, 0, st>>>(dout, y, dest_row, w, dy, dw, z.N, \
+                                                              z.d, sh.cw, z.Q, err)
+        if (z.K == 8 && vec) UE_BWD_CHUNK(8, true);
+        else if (z.K == 8) UE_BWD_CHUNK(8, false);
+        else if (vec) UE_BWD_CHUNK(4, true);
+        else UE_BWD_CHUNK(4, false);
+#undef UE_BWD_CHUNK
         return cudaGetLastError();
     }
 #define UE_BWD(KM)                                                                               \
