@@ -7,7 +7,9 @@
 * Gradient reduction: against the fp64 oracle within c 2^-24 sum |terms|
   (c = the expert's replica count, one fp32 rounding per addition); the same
   bits on a second run; and at full expert size bit-exact against a plain
-  fp32 PyTorch reference that adds the replicas in ascending slot order.
+  fp32 PyTorch reference that adds the replicas in ascending slot order;
+  hand placements (no replica at all, more replicas than experts, an id out
+  of range) bit-exact against the same ordered fp32 sum.
 """
 import numpy as np
 import pytest
@@ -131,5 +133,40 @@ def test_grad_reduce_qwen3_expert_size_matches_ordered_fp32():
         ue.ue_grad_reduce(L.ctx, plc, reps, master, NUMEL)
         assert L.error() == 0
         assert torch.equal(master, ref)
+    finally:
+        L.close()
+
+
+@pytest.mark.parametrize("se_list", [
+    [-1] * 16,                                            # no replica anywhere
+    [3, 3, 3, 3, 0, 1, -1, 3, 2, 2, 5, 3, -1, 7, 7, 3],   # G = 16 > E = 8, expert 3 seven times
+    [6, -1, 6, 9, 1, -1, -1, -1, -1, -1, -1, -1, 1, -1, 6, -1],  # an id out of range (9 >= E)
+])
+def test_grad_reduce_hand_placements(se_list):
+    """Hand placements: the reduction's list of replicated experts may be
+    empty, longer than E replicas for one expert, or hold an id out of range
+    (that slot is skipped and UE_ERR_DEVICE_BOUNDS set). The result is the
+    master plus the replicas added in ascending g in fp32, bit for bit; 1100
+    float4 per expert make a ragged last piece."""
+    R, T, E, K, S, d = 8, 4, 8, 2, 2, 8
+    G = R * S
+    numel = 4 * 1100
+    L = gh.make_layer(R, T, E, K, S, d, with_rows=False)
+    dev = L.device
+    try:
+        se = torch.tensor(se_list, dtype=torch.int32, device=dev)
+        dummy = torch.zeros(max(E, 4), dtype=torch.int32, device=dev)
+        plc = ue.placement(se, dummy, dummy, dummy, dummy, dummy)
+        master = torch.from_numpy(synth.normal_f32(E * numel, 1, 53).reshape(E, numel))
+        reps = torch.from_numpy(synth.normal_f32(G * numel, 1, 54).reshape(G, numel))
+        m_t = master.to(dev)
+        ue.ue_grad_reduce(L.ctx, plc, reps.to(dev), m_t, numel)
+        bad = any(e >= E for e in se_list)
+        assert L.error() == (ue.UE_ERR_DEVICE_BOUNDS if bad else ue.UE_OK)
+        ref = master.clone()
+        for g, e in enumerate(se_list):
+            if 0 <= e < E:
+                ref[e] = ref[e] + reps[g]
+        np.testing.assert_array_equal(m_t.cpu().numpy().view(np.uint32), ref.numpy().view(np.uint32))
     finally:
         L.close()

@@ -22,6 +22,7 @@ struct ue_ctx {
     int32_t* d_first;       // [R][P] locality order: first occurrence index
     int32_t* d_rowb;        // [R][P] locality order: row base
     uint16_t* d_zrow;       // [d] zeros: the combine reads it for a row out of range
+    int32_t* d_grtab;       // [kGrTableWords] gradient reduction: replicated experts, their slots
     int64_t tiles;
     int64_t spin_limit;
     int drop_first;
@@ -114,13 +115,15 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
         cudaMalloc(&ctx->d_sync, 4 * sizeof(uint32_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_first, table_words * sizeof(int32_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_rowb, table_words * sizeof(int32_t)) != cudaSuccess ||
-        cudaMalloc(&ctx->d_zrow, (size_t)ctx->z.d * sizeof(uint16_t)) != cudaSuccess) {
+        cudaMalloc(&ctx->d_zrow, (size_t)ctx->z.d * sizeof(uint16_t)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_grtab, ue::kGrTableWords * sizeof(int32_t)) != cudaSuccess) {
         cudaFree(ctx->d_err);
         cudaFree(ctx->d_status);
         cudaFree(ctx->d_sync);
         cudaFree(ctx->d_first);
         cudaFree(ctx->d_rowb);
         cudaFree(ctx->d_zrow);
+        cudaFree(ctx->d_grtab);
         delete ctx;
         cudaGetLastError();
         return UE_ERR_NOMEM;
@@ -136,6 +139,7 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
         cudaFree(ctx->d_first);
         cudaFree(ctx->d_rowb);
         cudaFree(ctx->d_zrow);
+        cudaFree(ctx->d_grtab);
         delete ctx;
         return UE_ERR_CUDA;
     }
@@ -156,6 +160,7 @@ ue_status ue_destroy(ue_ctx* ctx)
     cudaFree(ctx->d_first);
     cudaFree(ctx->d_rowb);
     cudaFree(ctx->d_zrow);
+    cudaFree(ctx->d_grtab);
     ctx->magic = 0;
     delete ctx;
     return st;
@@ -347,7 +352,7 @@ ue_status ue_grad_reduce(ue_ctx* ctx, const ue_placement* plan, const float* rep
         return UE_ERR_INVALID_ARG;
     if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
     return from_cuda(ue::launch_grad_reduce(ctx->z, plan->slot_expert, replica_grads,
-                                            master_grads, numel_per_expert, ctx->num_sms,
+                                            master_grads, numel_per_expert, ctx->d_grtab,
                                             ctx->d_err, as_stream(stream)));
 }
 

@@ -138,8 +138,11 @@ cudaError_t launch_combine_backward(const Sizes& z, const BwdShape& sh, const fl
 cudaError_t launch_weight_sync(const Sizes& z, const int32_t* slot_expert, const void* master,
                                void* replicas, int64_t bytes_per_expert, int num_sms, int* err,
                                cudaStream_t st);
+// tables: context scratch of kGrTableWords int32 (the reduction's list of
+// replicated experts and their replica slots, rebuilt by every call)
+constexpr int kGrTableWords = 3 * kMaxE + kMaxG + 1;
 cudaError_t launch_grad_reduce(const Sizes& z, const int32_t* slot_expert, const float* replicas,
-                               float* master, int64_t numel_per_expert, int num_sms, int* err,
+                               float* master, int64_t numel_per_expert, int32_t* tables, int* err,
                                cudaStream_t st);
 
 }  // namespace ue
