@@ -52,7 +52,7 @@ TRAFFIC = {
     "plan": {"bytes_per_launch": 29000, "source_sha": "2edfc203d9880067"},
     "reroute": {"bytes_per_launch": 8968000, "source_sha": "237f5cbb848c661f"},
     "permute": {"bytes_per_launch": 18890168000, "source_sha": "07222823ab0e9db7"},
-    "combine": {"bytes_per_launch": 21243824000, "source_sha": "0ebcc3caa2094612"},
+    "combine": {"bytes_per_launch": 21242032000, "source_sha": "c0631738399ffc37"},
 }
 
 def sha_of(path):
