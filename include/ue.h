@@ -97,8 +97,11 @@ typedef struct ue_ctx ue_ctx; /* opaque */
 
 /* Create a context for `cfg` on CUDA device `device` (made current) and
  * allocate its scratch once: the error word, the reroute's look-back status
- * words (ceil(Q/8192)*E 64-bit words plus a ticket, a counter and an epoch)
- * and the locality order's two int32 [R][P] tables. Nothing is allocated
+ * words (ceil(Q/8192)*E 64-bit words plus a ticket, a counter and an epoch),
+ * the locality order's two int32 [R][P] tables, a row of d zero bf16 values
+ * (the combine reads it in place of a row out of range) and the gradient
+ * reduction's int32 lists of replicated experts and their slots (at most
+ * 3*256 + 256 + 1 words). Nothing is allocated
  * after this call ("Interface / 1. Initialization": buffers reserved up
  * front, no dynamic allocation at runtime).
  * Returns UE_ERR_INVALID_ARG for a null `out` or a config outside the
