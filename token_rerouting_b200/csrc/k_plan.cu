@@ -36,8 +36,10 @@
 //  - warp 0 (rank side) keeps the rank loads and the redundant slots in
 //    registers (lane l owns ranks l, l+32, ... and their slots, so every
 //    load change lands in the lane that owns the rank). Per iteration: the
-//    stop test and the least loaded rank with a free slot (three `redux`
-//    reductions, with the pick's ready flag loaded before them), the
+//    stop test and the least loaded rank with a free slot (two `redux`
+//    reductions, max load and min of (load << 7 | r), when Q < 2^25; three
+//    otherwise), with the pick's ready flag and the pick itself loaded before
+//    them, the
 //    placement in r*'s lowest free slot, and the new quotas of e*'s copies: the
 //    master's goes from ceil(L/(c-1)) to ceil(L/c); a first replica takes
 //    floor(L/2); later replicas are found by ballots in ascending slot order.
@@ -85,6 +87,7 @@ struct Pick {
     unsigned qb;   // floor(L / c)
     unsigned rem;  // L mod c
     unsigned dq0;  // master quota change: ceil(L/c) - ceil(L/(c-1)) (two's complement)
+    int rm;        // the master's rank, e / M
 };
 
 template <int NJE, int NJR, int SM>
@@ -161,7 +164,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
             if (hi == 0u && lo == 0u) {
                 // no expert may take another copy: end marker
                 if (lane == 0) {
-                    sPick[t] = Pick{-1, 0u, 0u, 0u, 0u};
+                    sPick[t] = Pick{-1, 0u, 0u, 0u, 0u, 0};
                     __threadfence_block();
                     sReady[t] = 1;
                 }
@@ -193,7 +196,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
                 const unsigned rem = Le - qb * ce;
                 const unsigned q0_new = qb + (rem > 0u ? 1u : 0u);
                 const unsigned q0_old = div_by(Le + ce - 2u, ce - 1u, sRecip);
-                sPick[t] = Pick{estar, ce, qb, rem, q0_new - q0_old};
+                sPick[t] = Pick{estar, ce, qb, rem, q0_new - q0_old, estar / M};
                 __threadfence_block();
                 sReady[t] = 1;
             }
@@ -218,29 +221,57 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
         }
         int iters = 0;
         unsigned max_before = 0u;
+        // with every rank load below 2^25 (Q < 2^25), a rank's load and its
+        // index (< 128) pack into one 32-bit key, and the least loaded rank
+        // with a free slot (ties to the lowest r) is one reduction
+        const bool packed = Q < (1LL << 25);
         for (;;) {
-            // this iteration's pick: its flag is read first, so that the load
-            // overlaps the reductions below (acquire orders the pick read)
+            // this iteration's pick: its flag is read first and the pick
+            // right after it (acquire orders the read), so that both loads
+            // overlap the reductions below; a pick read before its flag was
+            // set is read again after the wait
+            // (iters reaches G only when every slot is used and the loop is
+            // about to stop; the index is clamped so that these early reads
+            // stay inside the arrays)
+            const int it0 = iters < kMaxG ? iters : kMaxG - 1;
             int ready = 0;
             asm volatile("ld.acquire.cta.shared.u32 %0, [%1];"
                          : "=r"(ready)
-                         : "r"((unsigned)__cvta_generic_to_shared((const void*)&sReady[iters]))
+                         : "r"((unsigned)__cvta_generic_to_shared((const void*)&sReady[it0]))
                          : "memory");
+            const int ready0 = ready;
+            const Pick pk_early = sPick[it0];
             unsigned maxl = 0u, bestl = 0xffffffffu, bestr = 0xffffffffu;
+            int rstar;
+            if (packed) {
+                unsigned key = 0xffffffffu;
 #pragma unroll
-            for (int j = 0; j < NJR; ++j) {
-                maxl = max(maxl, load[j]);
-                if (used[j] < S && load[j] < bestl) {
-                    bestl = load[j];
-                    bestr = (unsigned)(lane + 32 * j);
+                for (int j = 0; j < NJR; ++j) {
+                    maxl = max(maxl, load[j]);
+                    if (used[j] < S) key = min(key, (load[j] << 7) | (unsigned)(lane + 32 * j));
                 }
+                maxl = __reduce_max_sync(kFull, maxl);
+                key = __reduce_min_sync(kFull, key);
+                if (iters == 0) max_before = maxl;
+                if (50LL * R * (long long)maxl <= stop_rhs) break;
+                if (key == 0xffffffffu) break;  // no free slot anywhere
+                rstar = (int)(key & 127u);
+            } else {
+#pragma unroll
+                for (int j = 0; j < NJR; ++j) {
+                    maxl = max(maxl, load[j]);
+                    if (used[j] < S && load[j] < bestl) {
+                        bestl = load[j];
+                        bestr = (unsigned)(lane + 32 * j);
+                    }
+                }
+                maxl = __reduce_max_sync(kFull, maxl);
+                const unsigned ml = __reduce_min_sync(kFull, bestl);
+                if (iters == 0) max_before = maxl;
+                if (50LL * R * (long long)maxl <= stop_rhs) break;
+                if (ml == 0xffffffffu) break;  // no free slot anywhere
+                rstar = (int)__reduce_min_sync(kFull, bestl == ml ? bestr : 0xffffffffu);
             }
-            maxl = __reduce_max_sync(kFull, maxl);
-            const unsigned ml = __reduce_min_sync(kFull, bestl);
-            if (iters == 0) max_before = maxl;
-            if (50LL * R * (long long)maxl <= stop_rhs) break;
-            if (ml == 0xffffffffu) break;  // no free slot anywhere
-            const int rstar = (int)__reduce_min_sync(kFull, bestl == ml ? bestr : 0xffffffffu);
 
             // the pick is normally ready long before: the expert side needs
             // far fewer instructions per step. The wait is bounded.
@@ -254,7 +285,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
                 if (lane == 0) raise_error(err, UE_ERR_TIMEOUT, iters);
                 break;
             }
-            const Pick pk = sPick[iters];
+            const Pick pk = ready0 ? pk_early : sPick[iters];
             if (pk.e < 0) break;  // no expert may take another copy
             const int estar = pk.e;
             const int rj = rstar >> 5;
@@ -278,7 +309,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
                     }
             }
             // master quota change, on the master rank's owner
-            const int rm = estar / M;
+            const int rm = pk.rm;
             if (lane == (rm & 31)) {
 #pragma unroll
                 for (int j = 0; j < NJR; ++j)
