@@ -79,6 +79,22 @@ def algorithmic_bytes(w):
     }
 
 
+def row_bytes(N=0, K=0, d=0, used=0, replicated=0, bytes_per_expert=0, numel=0):
+    """Bytes each row beside the path must move (reads + writes of its operands).
+    combine backward: dout fp32 and the K bf16 rows y in, dest + w in, the K
+    bf16 rows dy and the fp32 dw out; permute backward: the K bf16 rows and
+    dest in, one fp32 row out; weight sync: every used slot's expert read and
+    written once; gradient reduction: each replicated master read and written,
+    each used replica slot read (fp32)."""
+    Q = N * K
+    return {
+        "combine_backward": 4 * N * d + 2 * Q * d + 8 * Q + 2 * Q * d + 4 * Q,
+        "permute_backward": 2 * Q * d + 4 * Q + 4 * N * d,
+        "weight_sync": 2 * used * bytes_per_expert,
+        "grad_reduce": 4 * numel * (2 * replicated + used),
+    }
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -393,8 +409,9 @@ def run_row(args, w):
         dh = torch.empty((N, d), dtype=torch.float32, device=dev)
         t1 = timed(lambda: ue.ue_combine_backward(L.ctx, dout, y, L.dest_row, L.w, dy, dw, st))
         t2 = timed(lambda: ue.ue_permute_backward(L.ctx, y, L.dest_row, dh, st))
-        kernels["combine_backward"] = (t1, 4 * N * d + 2 * Q * d + 8 * Q + 2 * Q * d + 4 * Q)
-        kernels["permute_backward"] = (t2, 2 * Q * d + 4 * Q + 4 * N * d)
+        rb = row_bytes(N=N, K=K, d=d)
+        kernels["combine_backward"] = (t1, rb["combine_backward"])
+        kernels["permute_backward"] = (t2, rb["permute_backward"])
         workload = dict(workload=w.name, N=N, K=K, d=d, pairs=Q)
     elif args.row == "layouts":
         # the permute's traffic (2Nd read, 2Qd written) under three row
@@ -448,13 +465,14 @@ def run_row(args, w):
                                    device=dev, generator=gen)
             reps = torch.empty((w.G, numel), dtype=torch.int16, device=dev)
             t = timed(lambda: ue.ue_weight_sync(L.ctx, L.plan, master, reps, bpe, st))
-            kernels["weight_sync"] = (t, 2 * used * bpe)
+            kernels["weight_sync"] = (t, row_bytes(used=used, bytes_per_expert=bpe)["weight_sync"])
         else:
             master = torch.randn((w.E, numel), dtype=torch.float32, device=dev, generator=gen)
             reps = torch.randn((w.G, numel), dtype=torch.float32, device=dev, generator=gen)
             t = timed(lambda: ue.ue_grad_reduce(L.ctx, L.plan, reps, master, numel, st))
             nrep = int((cnt > 0).sum())
-            kernels["grad_reduce"] = (t, 4 * numel * (2 * nrep + used))
+            kernels["grad_reduce"] = (t, row_bytes(used=used, replicated=nrep,
+                                                   numel=numel)["grad_reduce"])
         workload = dict(workload=w.name, expert_numel=numel, replicas=used,
                         replicated_experts=int((cnt > 0).sum()),
                         expert_shape=("Qwen3-235B expert: fc1 2*4096*1536 + fc2 4096*1536"

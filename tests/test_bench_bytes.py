@@ -44,3 +44,26 @@ def test_per_step_counts_on_a_small_case():
         "permute": 2 * N * d + K * 2 * N * d,
         "combine": K * 2 * N * d + 4 * Q + 4 * Q + 4 * N * d,
     }
+
+
+def test_row_bytes_on_the_qwen3_layer():
+    """The rows beside the path on the Qwen3-shaped layer with Qwen3-235B-sized
+    experts (18,874,368 elements: fc1 2*4096*1536 + fc2 4096*1536) and the
+    layer's greedy plan: 128 used replica slots over 107 replicated experts."""
+    w = synth.WORKLOADS["qwen3_layer_r64_e128"]
+    numel = 2 * 4096 * 1536 + 4096 * 1536
+    assert numel == bench.EXPERT_NUMEL
+    b = bench.row_bytes(N=w.N, K=w.K, d=w.d, used=128, replicated=107,
+                        bytes_per_expert=2 * numel, numel=numel)
+    assert abs(b["combine_backward"] / 1e9 - 38.68) < 0.005
+    assert abs(b["permute_backward"] / 1e9 - 21.48) < 0.005
+    assert abs(b["weight_sync"] / 1e9 - 9.66) < 0.005
+    assert abs(b["grad_reduce"] / 1e9 - 25.82) < 0.005
+    # per-operand form on a small case
+    N, K, d = 10, 4, 16
+    Q = N * K
+    b = bench.row_bytes(N=N, K=K, d=d, used=3, replicated=2, bytes_per_expert=32, numel=8)
+    assert b["combine_backward"] == 4 * N * d + K * 2 * N * d + 4 * Q + 4 * Q + K * 2 * N * d + 4 * Q
+    assert b["permute_backward"] == K * 2 * N * d + 4 * Q + 4 * N * d
+    assert b["weight_sync"] == 3 * 32 * 2
+    assert b["grad_reduce"] == 4 * 8 * (2 + 2 + 3)
