@@ -4,9 +4,11 @@
 One step = one layer instance through the whole path on the device:
 gate top-k -> exact histogram -> replication plan -> reroute -> permute ->
 gate-weighted combine (identity experts: the combine reads the dispatch
-buffer), on the Qwen3-235B-shaped layer (R=64 simulated EP ranks x 4096
-tokens, E=128, K=8, S=2, d=4096) with synthetic skewed routing (pre-balance
-max/mean rank load 2.5).
+buffer). The default workload is the largest layer that fits one GPU, the
+EP40 prefill layer (R=40 simulated EP ranks x 8192 tokens, E=160, K=8, S=1,
+d=5120, 2.6 M pairs) with synthetic per-source-rank Zipf skew; --workload
+selects another (the Qwen3-235B-shaped layer, the DeepSeek-V3-shaped layer,
+the small R=8 layer).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ue|reference]
 
@@ -35,24 +37,26 @@ if ROOT not in sys.path:
 METRIC = ("routed token-expert pairs/s and µs/layer (gate→plan→permute), "
           "% of HBM roofline")
 UNIT = "pairs/s"
-DEFAULT_WORKLOAD = "qwen3_layer_r64_e128"
+DEFAULT_WORKLOAD = "prefill_ep40_e160"
 KERNELS = ("gate_topk", "count", "plan", "reroute", "permute", "combine")
 FALLBACK_HBM_GBS = 6650.0
 
-# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# one ncu --set full capture of the same workload at 512 tokens per rank,
-# scaled by 8 to the full 4096 tokens per rank (the traffic of every kernel
-# but the plan grows in proportion to the tokens; the plan's, a few KB of
-# loads and outputs, does not and is taken as measured), with the SHA-256
-# prefix of the kernel source it was taken on; a kernel changed since then
-# reports null.
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+# each workload's kernels, from one ncu capture of the same workload at a
+# fraction of its tokens per rank, scaled up by the token ratio (the traffic
+# of every kernel but the plan grows in proportion to the tokens; the
+# plan's, a few KB of loads and outputs, does not and is taken as measured),
+# with the SHA-256 prefix of the kernel source it was taken on; a kernel
+# changed since then reports null.
 TRAFFIC = {
-    "gate_topk": {"bytes_per_launch": 134520000, "source_sha": "f9c2f7be091df85a"},
-    "count": {"bytes_per_launch": 8728000, "source_sha": "dda54be050ff39f0"},
-    "plan": {"bytes_per_launch": 29000, "source_sha": "2edfc203d9880067"},
-    "reroute": {"bytes_per_launch": 8968000, "source_sha": "237f5cbb848c661f"},
-    "permute": {"bytes_per_launch": 18890168000, "source_sha": "07222823ab0e9db7"},
-    "combine": {"bytes_per_launch": 21242032000, "source_sha": "c0631738399ffc37"},
+    "qwen3_layer_r64_e128": {
+        "gate_topk": {"bytes_per_launch": 134520000, "source_sha": "f9c2f7be091df85a"},
+        "count": {"bytes_per_launch": 8728000, "source_sha": "dda54be050ff39f0"},
+        "plan": {"bytes_per_launch": 29000, "source_sha": "2edfc203d9880067"},
+        "reroute": {"bytes_per_launch": 8968000, "source_sha": "237f5cbb848c661f"},
+        "permute": {"bytes_per_launch": 18890168000, "source_sha": "07222823ab0e9db7"},
+        "combine": {"bytes_per_launch": 21242032000, "source_sha": "c0631738399ffc37"},
+    },
 }
 
 def sha_of(path):
@@ -220,6 +224,128 @@ def oracle_slices(w, logits, hidden, tokens_per_rank, budget_s, max_slices):
     return pairs, elapsed, done
 
 
+def host_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def threaded_oracle_slice(w, lg, hd, t, threads, bufs=None):
+    """One slice (t tokens per rank, every rank) through the oracle's own C
+    functions with the data-parallel steps split over host threads by token
+    range: top-k and the weights, the counts (by source-rank range), the
+    permute (by dispatch-row range) and the combine (by token range); the
+    plan and the reroute stay sequential. The oracle's C calls release the
+    interpreter lock, so the ranges run in parallel. bufs: optional
+    preallocated (dispatch uint16 [Q][d], out float64 [N][d]), reused across
+    slices so that first-touch page faults stay out of the timing. Returns
+    the outputs."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+
+    import oracle
+    R, E, K, d = w.R, w.E, w.K, w.d
+    N, Q = R * t, R * t * K
+    nt = max(1, threads)
+
+    def ranges(n, parts):
+        b = np.linspace(0, n, min(parts, n) + 1).astype(np.int64)
+        return [(int(b[j]), int(b[j + 1])) for j in range(len(b) - 1) if b[j + 1] > b[j]]
+
+    idx = np.empty((N, K), dtype=np.int32)
+    wts = np.empty((N, K), dtype=np.float64)
+    load_re = np.empty((R, E), dtype=np.int32)
+    if bufs is None:
+        dispatch = np.empty((Q, d), dtype=np.uint16)
+        out = np.empty((N, d), dtype=np.float64)
+    else:
+        dispatch, out = bufs
+    with ThreadPoolExecutor(nt) as ex:
+        def gate(ab):
+            a, b = ab
+            idx[a:b], wts[a:b] = oracle.gate_topk(lg[a:b], K)
+        list(ex.map(gate, ranges(N, nt)))
+
+        def count(rr):
+            r0, r1 = rr
+            load_re[r0:r1], _ = oracle.count(idx[r0 * t:r1 * t], r1 - r0, t, E)
+        list(ex.map(count, ranges(R, nt)))
+        load_e = load_re.sum(axis=0, dtype=np.int64).astype(np.int32)
+        pl = oracle.plan(load_e, R, w.S)
+        phys, dest = oracle.reroute(idx, R, E, w.S, pl)
+
+        def permute(ab):
+            a, b = ab
+            oracle.permute_rows(hd, K, dest, np.arange(a, b, dtype=np.int64), out=dispatch[a:b])
+        list(ex.map(permute, ranges(Q, nt)))
+
+        def combine(ab):
+            a, b = ab
+            oracle.combine(dispatch, N, K, dest, wts, tokens=np.arange(a, b, dtype=np.int64),
+                           out=out[a:b])
+        list(ex.map(combine, ranges(N, nt)))
+    return dict(idx=idx, w=wts, load_re=load_re, load_e=load_e, plan=pl, phys_slot=phys,
+                dest_row=dest, dispatch=dispatch, out=out)
+
+
+def check_threaded_slice(w, lg, hd, t, res):
+    """The threaded slice's outputs against the single-threaded oracle's on
+    the same slice: every array equal (the same C functions on the same
+    data; only the split differs)."""
+    import numpy as np
+
+    import oracle
+    o = oracle.run_path(lg, w.R, t, w.S, w.K)
+    for k in ("idx", "w", "load_re", "load_e", "phys_slot", "dest_row"):
+        if not np.array_equal(res[k], o[k]):
+            raise SystemExit(f"threaded CPU baseline differs from the oracle in {k}")
+    for f in ("slot_expert", "n_copies", "slot_quota", "slot_offset", "rank_load", "stats"):
+        if not np.array_equal(getattr(res["plan"], f), getattr(o["plan"], f)):
+            raise SystemExit(f"threaded CPU baseline differs from the oracle in the plan ({f})")
+    disp = oracle.permute(hd, w.K, o["dest_row"])
+    if not np.array_equal(res["dispatch"], disp):
+        raise SystemExit("threaded CPU baseline differs from the oracle in the dispatch rows")
+    out = oracle.combine(disp, w.R * t, w.K, o["dest_row"], o["w"])
+    if not np.array_equal(res["out"], out):
+        raise SystemExit("threaded CPU baseline differs from the oracle in the combine")
+
+
+def threaded_oracle_slices(w, logits, hidden, tokens_per_rank, budget_s, max_slices,
+                           threads):
+    """oracle_slices with the threaded split (threaded_oracle_slice). Before
+    the timing, the threaded split is checked against the single-threaded
+    oracle on a 64-token-per-rank slice of the same workload. Returns
+    (pairs, seconds, slices)."""
+    import numpy as np
+    t = tokens_per_rank
+    pairs, elapsed, done = 0, 0.0, 0
+    nsl = max(1, w.T // t)
+    lg3 = logits.reshape(w.R, w.T, w.E)
+    hd3 = hidden.reshape(w.R, w.T, w.d)
+    tc = min(64, w.T)
+    lgc = lg3[:, :tc].reshape(-1, w.E).copy()
+    hdc = hd3[:, :tc].reshape(-1, w.d).copy()
+    check_threaded_slice(w, lgc, hdc, tc, threaded_oracle_slice(w, lgc, hdc, tc, threads))
+    bufs = (np.empty((w.R * t * w.K, w.d), dtype=np.uint16),
+            np.empty((w.R * t, w.d), dtype=np.float64))
+    for b in bufs:
+        b.fill(0)  # touch every page before the timing
+    for j in range(min(nsl, max_slices)):
+        lg = lg3[:, j * t:(j + 1) * t].reshape(-1, w.E).copy()
+        hd = hd3[:, j * t:(j + 1) * t].reshape(-1, w.d).copy()
+        t0 = time.perf_counter()
+        res = threaded_oracle_slice(w, lg, hd, t, threads, bufs)
+        elapsed += time.perf_counter() - t0
+        pairs += w.R * t * w.K
+        done += 1
+        del res
+        if elapsed >= budget_s:
+            break
+    return pairs, elapsed, done
+
+
 def run_reference(args, w):
     world, rank, _ = dist_setup(args.gpus)
     if rank != 0:
@@ -256,12 +382,33 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+ROUTING_TEXT = {
+    "small_r8_e64": "Zipf(s=1.2) log-weight bias in a seeded expert permutation",
+    "qwen3_layer_r64_e128": "Zipf(s=1.0) log-weight bias scaled so that the masters-only "
+                            "max/mean rank load is 2.5",
+    "dsv3_layer_r64_e256": "Zipf(s=1.3) log-weight bias plus two seeded hotspot experts "
+                           "boosted to draw 8% of pairs each",
+    "prefill_ep40_e160": "per-source-rank Zipf bias, s_r ~ U[0.8, 1.5] for each rank over one "
+                         "shared expert permutation (skew differs by source rank)",
+    "pages_ep64_e256_t8k": "Zipf(s=1.0) log-weight bias scaled to the pages' runtime-test "
+                           "imbalance 2.01",
+}
+L2_BYTES = 126 * 2 ** 20
+
+
 def workload_config(w):
+    base = w.name.split("_t")[0] if w.name not in ROUTING_TEXT else w.name
+    routing = ("logits N(0,1) + " + ROUTING_TEXT.get(base, f"{w.recipe} bias")
+               + ", seed 0 (microbatch = rank)")
+    lb, hb, db = 4 * w.N * w.E, 2 * w.N * w.d, 2 * w.Q * w.d
+    def size(b):
+        return f"{b / 1e9:.2f} GB" if b >= 1e9 else f"{b / 1e6:.1f} MB"
+
+    sizes = f"logits {size(lb)}, hidden {size(hb)}, dispatch {size(db)}"
+    l2 = (f"inputs larger than L2 ({sizes}); no flush needed" if db > 2 * L2_BYTES
+          else f"inputs L2-resident ({sizes}); not flushed between steps")
     return {"workload": w.name, "R": w.R, "T": w.T, "N": w.N, "E": w.E, "K": w.K, "S": w.S,
-            "d": w.d, "pairs_per_step": w.Q,
-            "routing": "logits N(0,1) + Zipf(s=1.0) log-weight bias scaled to a masters-only "
-                       "max/mean rank load of 2.5, seed 0 (microbatch = rank)",
-            "l2": "inputs larger than L2 (logits 134 MB, hidden 2.1 GB, dispatch 17.2 GB)",
+            "d": w.d, "pairs_per_step": w.Q, "routing": routing, "l2": l2,
             "experts": "identity (combine reads the dispatch buffer)"}
 
 
@@ -889,10 +1036,9 @@ def main():
     dom = max(("permute", "combine", "gate_topk", "reroute"), key=lambda k: per_kernel_ms[k])
     peak, peak_kind = load_peaks()
     achieved = abytes[dom] / (per_kernel_ms[dom] / 1e3) / 1e9
-    tr = TRAFFIC.get(dom)
+    tr = TRAFFIC.get(w.name, {}).get(dom)
     src = os.path.join(ROOT, "token_rerouting_b200", "csrc", KERNEL_SRC[dom])
-    traffic = (tr["bytes_per_launch"] if tr and tr.get("source_sha") == sha_of(src)
-               and w.name == DEFAULT_WORKLOAD else None)
+    traffic = (tr["bytes_per_launch"] if tr and tr.get("source_sha") == sha_of(src) else None)
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "peak_kind": f"of {peak_kind}",
                 "traffic": traffic, "algorithmic_bytes": abytes[dom]}
@@ -992,6 +1138,15 @@ def main():
                "sample": f"{nsl} slice(s) of 512 tokens per rank x {w.R} ranks "
                          f"({pairs} pairs, {secs:.1f} s), each a whole layer instance "
                          f"through the single-threaded C oracle incl. permute and combine"}
+        nthr = host_threads()
+        tp, ts, tn = threaded_oracle_slices(w, logits_h, hidden_h, 512, 10.0, 16, nthr)
+        cpu["threaded"] = {
+            "value": tp / ts, "unit": UNIT, "cores": nthr,
+            "kind": "oracle split over host threads by token range (top-k, counts, permute, "
+                    "combine); plan and reroute sequential",
+            "sample": f"{tn} slice(s) of 512 tokens per rank x {w.R} ranks ({tp} pairs, "
+                      f"{ts:.1f} s)",
+            "checked": "first slice's outputs equal to the single-threaded oracle's"}
 
     if rank == 0:
         line = {

@@ -353,17 +353,26 @@ ue_status ue_grad_reduce(ue_ctx* ctx, const ue_placement* plan, const float* rep
  * few words, held on every GPU that loads the library until the process
  * exits): sizes with ceil(R*T*K / 8192) * E > 262144 are rejected with
  * UE_ERR_UNSUPPORTED before anything is launched. The first call made with
- * a given device current looks up that array's device address
+ * a given device current checks that the device is an sm_100 part
+ * (UE_ERR_UNSUPPORTED otherwise), looks up that array's device address
  * (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture. Every call shares the array and it is never cleared: its
- * status words carry the call's epoch, so words left by an earlier call read
- * as unpublished, and each call's last CTA resets the tile ticket. Calls
- * that overlap on the GPU (other streams, other threads) race and give
- * wrong results. Calls no cudaMalloc or cudaFree.
+ * stream capture. cudaDeviceReset makes the cached address stale: do not
+ * call this entry point again in a process that has reset the device.
+ * Every call shares the array and it is never cleared: its status words
+ * carry the call's epoch, so words left by an earlier call read as
+ * unpublished, and each call's last CTA resets the tile ticket, also after
+ * a call that ended in a device-side error. Calls that overlap on the GPU
+ * (other streams, other threads) race and give wrong results. Calls no
+ * cudaMalloc or cudaFree.
  *   cfg, idx, plan, phys_slot, dest_row, stream: as for ue_init + ue_reroute
- *   (cfg is a host pointer, read during the call).
- *   error: device int32[2], zeroed by the caller; a device-side error writes
- *   {code, detail} into it (the first one only). NULL: errors are dropped.
+ *   (cfg is a host pointer, read during the call). idx, phys_slot,
+ *   dest_row, error and the plan arrays must be memory of the current
+ *   device (UE_ERR_INVALID_ARG otherwise, before any launch).
+ *   error: device int32[2], zeroed by the caller, required (NULL is
+ *   UE_ERR_INVALID_ARG): a device-side error writes {code, detail} into it
+ *   (the first one only). After a device-side error (an expert id out of
+ *   range, a look-back wait that ran out) the outputs are not valid: a pair
+ *   with a bad id gets -1, and a timed-out call writes nothing.
  * Host-side errors are returned at once, as for ue_reroute. */
 ue_status ue_reroute_noalloc(const ue_config* cfg, const int32_t* idx,
                              const ue_placement* plan, int32_t* phys_slot,

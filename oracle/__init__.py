@@ -252,13 +252,16 @@ def permute(hidden_u16: np.ndarray, K: int, dest_row: np.ndarray):
 
 
 def permute_rows(hidden_u16: np.ndarray, K: int, dest_row: np.ndarray,
-                 rows: np.ndarray):
-    """The permute's result at the given dispatch rows only."""
+                 rows: np.ndarray, out: np.ndarray | None = None):
+    """The permute's result at the given dispatch rows only (written into
+    ``out`` if given: a C-contiguous uint16 [len(rows), d] array)."""
     hidden_u16 = np.ascontiguousarray(hidden_u16, dtype=np.uint16)
     N, d = hidden_u16.shape
     dest_row = np.ascontiguousarray(dest_row, dtype=np.int32)
     rows = np.ascontiguousarray(rows, dtype=np.int64)
-    out = np.empty((rows.size, d), dtype=np.uint16)
+    if out is None:
+        out = np.empty((rows.size, d), dtype=np.uint16)
+    assert out.dtype == np.uint16 and out.shape == (rows.size, d)
     _check(_load().or_permute_rows(_ptr(hidden_u16), N, d, K, _ptr(dest_row),
                                    _ptr(rows), rows.size, _ptr(out)),
            "permute_rows")
@@ -266,20 +269,24 @@ def permute_rows(hidden_u16: np.ndarray, K: int, dest_row: np.ndarray,
 
 
 def combine(y_u16: np.ndarray, N: int, K: int, dest_row: np.ndarray,
-            w: np.ndarray, tokens: np.ndarray | None = None):
+            w: np.ndarray, tokens: np.ndarray | None = None,
+            out: np.ndarray | None = None):
     """fp64 out[n] = sum_k w[n, k] * y[dest_row[n, k]] (all tokens, or the
-    listed ones)."""
+    listed ones; written into ``out`` if given: a C-contiguous float64 array
+    with one row per evaluated token)."""
     y_u16 = np.ascontiguousarray(y_u16, dtype=np.uint16)
     d = y_u16.shape[1]
     dest_row = np.ascontiguousarray(dest_row, dtype=np.int32)
     w = np.ascontiguousarray(w, dtype=np.float64)
     if tokens is not None:
         tokens = np.ascontiguousarray(tokens, dtype=np.int64)
-        out = np.empty((tokens.size, d), dtype=np.float64)
         nt = tokens.size
     else:
-        out = np.empty((N, d), dtype=np.float64)
         nt = 0
+    rows_out = tokens.size if tokens is not None else N
+    if out is None:
+        out = np.empty((rows_out, d), dtype=np.float64)
+    assert out.dtype == np.float64 and out.shape == (rows_out, d) and out.flags["C_CONTIGUOUS"]
     _check(_load().or_combine(_ptr(y_u16), N, d, K, _ptr(dest_row), _ptr(w),
                               _ptr(tokens), nt, _ptr(out)), "combine")
     return out

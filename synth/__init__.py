@@ -248,6 +248,15 @@ def expert_outputs(w: Workload, seed: int = 0) -> np.ndarray:
     return bf16_normal(w.Q, w.d, seed, _TAG_Y, w.cid)
 
 
+def expert_output_rows(w: Workload, seed: int = 0) -> np.ndarray:
+    """Seeded source rows sigma [Q] int64 in [0, N) for a cheaper stand-in for
+    expert outputs at full size: y[r] = hidden[sigma[r]]. Each dispatch row
+    gets its own randomly chosen N(0,1) bf16 row, independent of the routing,
+    so a row read from the wrong place differs from the right one unless two
+    draws coincide (probability 1/N per pair of rows)."""
+    return _stream(seed, _TAG_Y, w.cid, 1).integers(0, w.N, size=w.Q, dtype=np.int64)
+
+
 def custom(R, T, E, K, S, d, name="custom", cid=99, recipe="zipf", zipf_s=1.2):
     """A workload of arbitrary sizes (tests: ragged and edge cases)."""
     return Workload(name, cid, R=R, T=T, E=E, K=K, S=S, d=d, recipe=recipe,
@@ -259,6 +268,6 @@ def describe(w: Workload) -> str:
             f"S={w.S} d={w.d} Q={w.Q} recipe={w.recipe}")
 
 
-__all__ = ["Workload", "WORKLOADS", "logits", "hidden", "expert_outputs",
+__all__ = ["Workload", "WORKLOADS", "logits", "hidden", "expert_outputs", "expert_output_rows",
            "bf16_normal", "normal_f32", "f32_to_bf16_bits", "bf16_bits_to_f32",
            "logit_bias", "custom", "describe"]

@@ -97,3 +97,89 @@ def assert_combine_close(out_gpu, out_or, scale):
     bad = err > bound
     assert not bad.any(), (f"{bad.sum()} combine elements out of tolerance; worst ratio "
                            f"{(err / bound).max():.3e}")
+
+
+def _workers():
+    import os
+    return max(1, min(16, os.cpu_count() or 1))
+
+
+def assert_dispatch_all_rows(layer, hidden_u16, K, dest_row_or, chunk_rows=1 << 15):
+    """Every dispatch row of the device against the oracle's permute (built
+    from the oracle's own dest_row), chunk by chunk so that the rows are
+    never all on the host at once. The oracle calls and the comparisons run
+    in threads (both release the interpreter lock)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+    Q = layer.Q
+
+    def job(r0):
+        r1 = min(Q, r0 + chunk_rows)
+        got = bf16_to_host_u16(layer.dispatch[r0:r1])
+        exp = oracle.permute_rows(hidden_u16, K, dest_row_or, np.arange(r0, r1, dtype=np.int64))
+        if np.array_equal(got, exp):
+            return None
+        bad = np.nonzero((got != exp).any(axis=1))[0]
+        return (r0 + bad[:4]).tolist(), int(bad.size)
+
+    with ThreadPoolExecutor(_workers()) as ex:
+        res = [r for r in ex.map(job, range(0, Q, chunk_rows)) if r is not None]
+    assert not res, (f"{sum(n for _, n in res)} dispatch rows differ from the oracle's permute; "
+                     f"first {res[0][0]}")
+
+
+def expert_outputs_on_device(layer, hidden_u16, sigma):
+    """Write the stand-in expert outputs y[r] = hidden[sigma[r]] into the
+    layer's dispatch buffer (input construction for the combine check)."""
+    import torch
+    sig = torch.from_numpy(np.ascontiguousarray(sigma, dtype=np.int64)).to(layer.device)
+    step = 1 << 18
+    for r0 in range(0, layer.Q, step):
+        r1 = min(layer.Q, r0 + step)
+        torch.index_select(layer.hidden, 0, sig[r0:r1], out=layer.dispatch[r0:r1])
+    torch.cuda.synchronize(layer.device)
+
+
+def assert_combine_all_tokens(layer, hidden_u16, sigma, K, dest_row_or, w_or,
+                              tokens=None, chunk_tokens=2048):
+    """Every element of the device's combine output (or those of the listed
+    tokens) against the oracle's fp64 combine of the same expert outputs
+    y[r] = hidden[sigma[r]] at the oracle's dest_row with the oracle's
+    weights, within the normwise tolerance. For each chunk of tokens the
+    oracle is given the chunk's K rows per token, gathered on the host, with
+    dest_row renumbered to them; the tolerance scale sum_k |w_k y_k| is the
+    oracle's combine of |y| with |w|."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+    N = layer.N
+    toks = np.arange(N, dtype=np.int64) if tokens is None else np.asarray(tokens, np.int64)
+    out_dev = layer.out
+
+    def job(c0):
+        t = toks[c0:c0 + chunk_tokens]
+        n = t.size
+        if tokens is None:
+            got = out_dev[int(t[0]):int(t[-1]) + 1].cpu().numpy()
+        else:
+            import torch
+            got = out_dev[torch.from_numpy(t).to(layer.device)].cpu().numpy()
+        rows = dest_row_or[t].ravel()
+        ych = np.ascontiguousarray(hidden_u16[sigma[rows]])
+        dloc = np.arange(n * K, dtype=np.int32).reshape(n, K)
+        wt = np.ascontiguousarray(w_or[t], dtype=np.float64)
+        exp = oracle.combine(ych, n, K, dloc, wt)
+        np.bitwise_and(ych, np.uint16(0x7FFF), out=ych)
+        scale = oracle.combine(ych, n, K, dloc, np.abs(wt))
+        err = np.abs(got.astype(np.float64) - exp)
+        bound = COMBINE_RTOL * scale + COMBINE_ATOL
+        bad = err > bound
+        if not bad.any():
+            return None
+        return int(bad.sum()), float((err / bound).max()), int(t[np.argwhere(bad)[0][0]])
+
+    with ThreadPoolExecutor(_workers()) as ex:
+        res = [r for r in ex.map(job, range(0, toks.size, chunk_tokens)) if r is not None]
+    assert not res, (f"{sum(r[0] for r in res)} combine elements out of tolerance; worst ratio "
+                     f"{max(r[1] for r in res):.3e}; first token {res[0][2]}")

@@ -67,3 +67,17 @@ def test_row_bytes_on_the_qwen3_layer():
     assert b["permute_backward"] == K * 2 * N * d + 4 * Q + 4 * N * d
     assert b["weight_sync"] == 3 * 32 * 2
     assert b["grad_reduce"] == 4 * 8 * (2 + 2 + 3)
+
+
+def test_threaded_cpu_baseline_equals_the_oracle():
+    """The threaded CPU baseline (the oracle's own C functions split over host
+    threads by token range) gives exactly the single-threaded oracle's
+    outputs on a small workload, for several thread counts."""
+    import synth
+    w = synth.WORKLOADS["small_r8_e64"]
+    lg, hd = synth.logits(w), synth.hidden(w)
+    for threads in (1, 3, 8):
+        res = bench.threaded_oracle_slice(w, lg, hd, w.T, threads)
+        bench.check_threaded_slice(w, lg, hd, w.T, res)
+    pairs, secs, n = bench.threaded_oracle_slices(w, lg, hd, 128, 0.0, 2, 4)
+    assert pairs == w.R * 128 * w.K and n == 1 and secs > 0

@@ -5,11 +5,18 @@ and hot set redrawn per instance, with a uniform instance (0,0) and a
 graph over fixed buffers; each instance's logits are staged into the input
 buffer and the graph is replayed.
 
-Every instance is checked on the device by properties that hold at any size
-(dest_row is a permutation of the pairs; each slot receives exactly its
-quota; each pair lands on a copy of its own expert; rank loads sum to the
-pairs). Eight instances, the two special ones included, are compared with
-the oracle element by element on the routing and on sampled dispatch rows.
+Every instance's routing (top-k ids, counts, every plan array, phys_slot,
+dest_row) is compared with the oracle's, byte for byte, through a SHA-256
+digest the oracle wrote for that instance (tests/golden/sweep_digests.py);
+on a mismatch the oracle is run on the instance to name the array that
+differs. Every instance's gate weights are compared with the oracle's on a
+sample of rows, and every instance is also checked on the device by
+properties (dest_row is a permutation of the pairs; each slot receives
+exactly its quota; each pair lands on a copy of its own expert; rank loads
+sum to the pairs). Eight instances, the two special ones included, are also
+compared with the oracle element by element on the routing, on sampled
+dispatch rows, and on the combine with independent expert outputs (every
+token under the greedy plan, a token sample under the capacity planner).
 
 The sweep runs twice: with the path's greedy plan, and with the capacity
 planner at the pages' defaults ("UltraEP" README, "Performance Tuning /
@@ -18,6 +25,9 @@ replica), whose every instance is also checked against its own guarantees
 (rank loads within the chosen capacity C(k) = floor(k Q / (100 R)), every
 replica at least 1024 pairs).
 """
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -25,6 +35,10 @@ import torch
 import oracle
 import synth
 from tests import gpu_helpers as gh
+from tests.routing_digest import flatten_oracle, routing_digest
+
+DIGESTS = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                       "sweep_digests.json")
 
 pytestmark = pytest.mark.gpu
 
@@ -61,8 +75,23 @@ def test_sweep_graph_captured(planner):
         L.permute(st)
         L.combine(stream=st)
 
+    with open(DIGESTS) as f:
+        digests = json.load(f)["digests"][planner]
+    assert len(digests) == w.layers * w.microbatches
+
+    def oracle_path(logits):
+        if opts is None:
+            return oracle.run_path(logits, w.R, w.T, w.S, w.K)
+        idx, wts = oracle.gate_topk(logits, w.K)
+        load_re, load_e = oracle.count(idx, w.R, w.T, w.E)
+        pl = oracle.plan_bisect(load_e, w.R, w.S)
+        phys, dest = oracle.reroute(idx, w.R, w.E, w.S, pl)
+        return dict(idx=idx, w=wts, load_re=load_re, load_e=load_e, plan=pl,
+                    phys_slot=phys, dest_row=dest)
+
     try:
         hidden = synth.hidden(w)
+        sigma = synth.expert_output_rows(w)
         L.hidden.copy_(gh.bf16_to_device(hidden, dev))
         L.logits.copy_(torch.from_numpy(synth.logits(w, 0, 0)))
         s = torch.cuda.Stream(device=dev)
@@ -108,21 +137,33 @@ def test_sweep_graph_captured(planner):
                     if bool(used.any()):
                         rep_q = L.slot_quota.view(w.R, w.M + w.S)[:, w.M:].flatten()[used]
                         assert int(rep_q.min()) >= 1024, (layer, mb)
+                # every instance: the routing against the oracle's digest
+                g = gh.routing_results(L)
+                inst = layer * w.microbatches + mb
+                if routing_digest(g) != digests[inst] or (layer, mb) in exact:
+                    o = oracle_path(logits)
+                    gh.assert_routing_equal(g, o)
+                    assert routing_digest(flatten_oracle(o)) == digests[inst], (
+                        "stored digest differs from the oracle's routing", layer, mb)
+                # every instance: gate weights on a row sample
+                wrows = np.sort(rng.choice(w.N, 1024, replace=False))
+                _, w_or = oracle.gate_topk(logits[wrows], w.K)
+                gh.assert_weights_close(g["w"][wrows], w_or)
                 if (layer, mb) in exact:
-                    if opts is None:
-                        o = oracle.run_path(logits, w.R, w.T, w.S, w.K)
-                    else:
-                        idx, wts = oracle.gate_topk(logits, w.K)
-                        load_re, load_e = oracle.count(idx, w.R, w.T, w.E)
-                        pl = oracle.plan_bisect(load_e, w.R, w.S)
-                        phys, dest = oracle.reroute(idx, w.R, w.E, w.S, pl)
-                        o = dict(idx=idx, w=wts, load_re=load_re, load_e=load_e, plan=pl,
-                                 phys_slot=phys, dest_row=dest)
-                    gh.assert_routing_equal(gh.routing_results(L), o)
-                    rows = np.sort(rng.choice(w.Q, 2048, replace=False))
+                    rows = np.sort(np.concatenate([
+                        rng.choice(w.Q, 16384, replace=False),
+                        o["plan"].slot_offset[np.nonzero(o["plan"].slot_quota)[0]]]))
+                    rows = np.unique(rows)
                     got = gh.bf16_to_host_u16(L.dispatch[torch.from_numpy(rows).to(dev)])
                     np.testing.assert_array_equal(
                         got, oracle.permute_rows(hidden, w.K, o["dest_row"], rows))
+                    # combine with independent expert outputs
+                    gh.expert_outputs_on_device(L, hidden, sigma)
+                    L.combine()
+                    toks = (None if opts is None
+                            else np.sort(rng.choice(w.N, 16384, replace=False)))
+                    gh.assert_combine_all_tokens(L, hidden, sigma, w.K, o["dest_row"], o["w"],
+                                                 tokens=toks)
         assert L.error() == 0
         # the sweep spans balanced and heavily skewed instances
         assert min(skew_before) < 1.1 and max(skew_before) > 2.0

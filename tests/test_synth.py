@@ -98,3 +98,22 @@ def test_prefill_per_rank_exponents_differ():
     assert bias.shape == (40, 160)
     assert info["s_r"].min() >= 0.8 and info["s_r"].max() <= 1.5
     assert len(np.unique(np.round(info["s_r"], 6))) == 40
+
+
+@pytest.mark.slow_cpu
+def test_stored_sweep_digests_are_the_oracles():
+    """The stored digests of the sweep (written by tests/golden/sweep_digests.py
+    from the oracle) match the oracle recomputed here on the uniform
+    instance, the 30%-single-expert instance and one Zipf instance."""
+    import json
+    import os
+
+    from tests.routing_digest import flatten_oracle, routing_digest
+    path = os.path.join(os.path.dirname(__file__), "golden", "sweep_digests.json")
+    with open(path) as f:
+        doc = json.load(f)
+    w = synth.WORKLOADS[doc["workload"]]
+    for layer, mb in [(0, 0), (0, 1), (17, 3)]:
+        o = oracle.run_path(synth.logits(w, layer, mb), w.R, w.T, w.S, w.K)
+        assert routing_digest(flatten_oracle(o)) == \
+            doc["digests"]["greedy"][layer * w.microbatches + mb], (layer, mb)

@@ -33,19 +33,6 @@ namespace {
 
 constexpr uint32_t kMagic = 0x75656331u;  // "uec1"
 
-bool config_ok(const ue_config& c)
-{
-    if (c.R < 1 || c.R > ue::kMaxR) return false;
-    if (c.E < 1 || c.E > ue::kMaxE || c.E % c.R != 0) return false;
-    if (c.K < 1 || c.K > ue::kMaxK || c.K > c.E) return false;
-    if (c.S < 0 || c.S > ue::kMaxS || c.R * c.S > ue::kMaxG) return false;
-    if (c.T < 1) return false;
-    if (c.d < 8 || c.d % 8 != 0 || c.d > ue::kMaxD) return false;
-    const int64_t Q = (int64_t)c.R * c.T * c.K;
-    if (Q >= (int64_t(1) << 30)) return false;
-    return true;
-}
-
 bool ctx_ok(const ue_ctx* ctx) { return ctx != nullptr && ctx->magic == kMagic; }
 
 bool aligned(const void* p, size_t a) { return p != nullptr && ((uintptr_t)p % a) == 0; }
@@ -79,7 +66,7 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
 {
     if (out == nullptr) return UE_ERR_INVALID_ARG;
     *out = nullptr;
-    if (cfg == nullptr || !config_ok(*cfg)) return UE_ERR_INVALID_ARG;
+    if (cfg == nullptr || !ue::config_ok(*cfg)) return UE_ERR_INVALID_ARG;
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess) return UE_ERR_CUDA;
     if (device < 0 || device >= ndev) return UE_ERR_INVALID_ARG;

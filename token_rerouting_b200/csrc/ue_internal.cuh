@@ -51,6 +51,20 @@ struct Sizes {
     int64_t N, Q;
 };
 
+// The config limits every entry point checks on the host (ue.h, ue_config).
+inline bool config_ok(const ue_config& c)
+{
+    if (c.R < 1 || c.R > kMaxR) return false;
+    if (c.E < 1 || c.E > kMaxE || c.E % c.R != 0) return false;
+    if (c.K < 1 || c.K > kMaxK || c.K > c.E) return false;
+    if (c.S < 0 || c.S > kMaxS || c.R * c.S > kMaxG) return false;
+    if (c.T < 1) return false;
+    if (c.d < 8 || c.d % 8 != 0 || c.d > kMaxD) return false;
+    const int64_t Q = (int64_t)c.R * c.T * c.K;
+    if (Q >= (int64_t(1) << 30)) return false;
+    return true;
+}
+
 inline Sizes make_sizes(const ue_config& c)
 {
     Sizes s;

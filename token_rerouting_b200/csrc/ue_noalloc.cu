@@ -17,7 +17,10 @@
 // The array's name, used in host code, is only a host-side stand-in for the
 // symbol, not a device address. The device address is fetched once per
 // device with cudaGetSymbolAddress (on the first call made with that device
-// current) and passed to the kernel.
+// current, which also checks that the device is an sm_100 part) and passed
+// to the kernel. cudaDeviceReset unloads the module and makes the cached
+// address stale, so this entry point must not be used after a reset in the
+// same process.
 #include <mutex>
 
 #include "ue_internal.cuh"
@@ -26,23 +29,32 @@ namespace {
 
 constexpr size_t kStatusWords = size_t(1) << 18;  // 2 MiB of 64-bit look-back words
 constexpr size_t kSyncWord = kStatusWords;        // ticket, counter, epoch (as 32-bit)
-constexpr size_t kErrWord = kStatusWords + 16;    // error word when none is given
-constexpr size_t kScratchWords = kStatusWords + 32;
+constexpr size_t kScratchWords = kStatusWords + 16;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned long long g_reroute_scratch[kScratchWords];
 
 std::mutex g_mutex;
 unsigned long long* g_scratch_addr[kMaxDevices] = {};
+ue_status g_device_status[kMaxDevices] = {};  // first lookup's outcome per device
 
 // device address of g_reroute_scratch on the current device, looked up once
-ue_status scratch_address(unsigned long long** out)
+ue_status scratch_address(int dev, unsigned long long** out)
 {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return UE_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return UE_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_mutex);
     if (g_scratch_addr[dev] == nullptr) {
+        if (g_device_status[dev] == UE_ERR_UNSUPPORTED) return UE_ERR_UNSUPPORTED;
+        int major = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return UE_ERR_CUDA;
+        }
+        if (major != 10) {
+            g_device_status[dev] = UE_ERR_UNSUPPORTED;
+            return UE_ERR_UNSUPPORTED;
+        }
         void* p = nullptr;
         const cudaError_t ce = cudaGetSymbolAddress(&p, g_reroute_scratch);
         if (ce != cudaSuccess || p == nullptr) {
@@ -57,37 +69,48 @@ ue_status scratch_address(unsigned long long** out)
 
 bool aligned4(const void* p) { return p != nullptr && ((uintptr_t)p % 4) == 0; }
 
+// true when p is device (or managed) memory that device dev can address as
+// its own; host memory and another GPU's memory are refused
+bool on_device(const void* p, int dev)
+{
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (a.type == cudaMemoryTypeManaged) return true;
+    return a.type == cudaMemoryTypeDevice && a.device == dev;
+}
+
 }  // namespace
 
 extern "C" ue_status ue_reroute_noalloc(const ue_config* cfg, const int32_t* idx,
                                         const ue_placement* plan, int32_t* phys_slot,
                                         int32_t* dest_row, int32_t* error, void* stream)
 {
-    if (cfg == nullptr || plan == nullptr) return UE_ERR_INVALID_ARG;
-    const ue_config& c = *cfg;
-    if (c.R < 1 || c.R > ue::kMaxR || c.E < 1 || c.E > ue::kMaxE || c.E % c.R != 0 ||
-        c.K < 1 || c.K > ue::kMaxK || c.K > c.E || c.S < 0 || c.S > ue::kMaxS ||
-        c.R * c.S > ue::kMaxG || c.T < 1 || c.d < 8 || c.d % 8 != 0 || c.d > ue::kMaxD ||
-        (int64_t)c.R * c.T * c.K >= (int64_t(1) << 30))
-        return UE_ERR_INVALID_ARG;
-    const ue::Sizes z = ue::make_sizes(c);
+    if (cfg == nullptr || plan == nullptr || !ue::config_ok(*cfg)) return UE_ERR_INVALID_ARG;
+    const ue::Sizes z = ue::make_sizes(*cfg);
     if ((z.G > 0 && !aligned4(plan->slot_expert)) || !aligned4(plan->n_copies) ||
         !aligned4(plan->slot_quota) || !aligned4(plan->slot_offset) ||
         !aligned4(plan->rank_load) || !aligned4(plan->stats) || !aligned4(idx) ||
-        !aligned4(phys_slot) || !aligned4(dest_row) ||
-        (error != nullptr && !aligned4(error)))
+        !aligned4(phys_slot) || !aligned4(dest_row) || !aligned4(error))
         return UE_ERR_INVALID_ARG;
     const int64_t tiles = (z.Q + ue::kRerouteTile - 1) / ue::kRerouteTile;
     if ((size_t)tiles * (size_t)z.E > kStatusWords) return UE_ERR_UNSUPPORTED;
 
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return UE_ERR_CUDA;
     unsigned long long* base = nullptr;
-    const ue_status st = scratch_address(&base);
+    const ue_status st = scratch_address(dev, &base);
     if (st != UE_OK) return st;
-    int* err = error != nullptr ? reinterpret_cast<int*>(error)
-                                : reinterpret_cast<int*>(base + kErrWord);
+    // every buffer the kernel touches must live on the current device
+    if (!on_device(idx, dev) || !on_device(phys_slot, dev) || !on_device(dest_row, dev) ||
+        !on_device(error, dev) || !on_device(plan->slot_offset, dev) ||
+        !on_device(plan->slot_quota, dev) || (z.G > 0 && !on_device(plan->slot_expert, dev)))
+        return UE_ERR_INVALID_ARG;
     uint32_t* sync = reinterpret_cast<uint32_t*>(base + kSyncWord);
     const cudaError_t ce = ue::launch_reroute(z, idx, *plan, phys_slot, dest_row, base, sync,
-                                              int64_t(1) << 22, 0, err,
+                                              int64_t(1) << 22, 0, reinterpret_cast<int*>(error),
                                               reinterpret_cast<cudaStream_t>(stream));
     return ce == cudaSuccess ? UE_OK : UE_ERR_CUDA;
 }
