@@ -38,7 +38,7 @@ METRIC = ("routed token-expert pairs/s and µs/layer (gate→plan→permute), "
           "% of HBM roofline")
 UNIT = "pairs/s"
 DEFAULT_WORKLOAD = "prefill_ep40_e160"
-KERNELS = ("gate_topk", "count", "plan", "reroute", "permute", "combine")
+KERNELS = ("gate_count", "plan", "reroute", "permute", "combine")
 FALLBACK_HBM_GBS = 6650.0
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
@@ -49,9 +49,15 @@ FALLBACK_HBM_GBS = 6650.0
 # with the SHA-256 prefix of the kernel source it was taken on; a kernel
 # changed since then reports null.
 TRAFFIC = {
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum at 1024 tokens
+    # per rank (6 launches each), times 8
+    "prefill_ep40_e160": {
+        "permute": {"bytes_per_launch": 29715613013, "source_sha": "07222823ab0e9db7"},
+        "combine": {"bytes_per_launch": 33329068032, "source_sha": "c0631738399ffc37"},
+    },
+    # ncu --set full at 512 tokens per rank, times 8
     "qwen3_layer_r64_e128": {
-        "gate_topk": {"bytes_per_launch": 134520000, "source_sha": "f9c2f7be091df85a"},
-        "count": {"bytes_per_launch": 8728000, "source_sha": "dda54be050ff39f0"},
+        "gate_count": {"bytes_per_launch": 134520000, "source_sha": "f9c2f7be091df85a"},
         "plan": {"bytes_per_launch": 29000, "source_sha": "2edfc203d9880067"},
         "reroute": {"bytes_per_launch": 8968000, "source_sha": "237f5cbb848c661f"},
         "permute": {"bytes_per_launch": 18890168000, "source_sha": "07222823ab0e9db7"},
@@ -65,17 +71,19 @@ def sha_of(path):
 
 
 KERNEL_SRC = {
-    "gate_topk": "k_gate.cu", "count": "k_count.cu", "plan": "k_plan.cu",
+    "gate_count": "k_gate.cu", "plan": "k_plan.cu",
     "reroute": "k_reroute.cu", "permute": "k_permute.cu", "combine": "k_combine.cu",
 }
 
 
 def algorithmic_bytes(w):
-    """Bytes each step must move per kernel (reads + writes of its operands)."""
+    """Bytes each step must move per kernel (reads + writes of its operands).
+    The histogram is taken inside the gate kernel (gate_count), so it adds no
+    bytes there; "count" is the separate count kernel's, for reference."""
     N, E, K, d, Q = w.N, w.E, w.K, w.d, w.Q
     return {
-        "gate_topk": 4 * N * E + 8 * Q,          # logits in; idx + w out
-        "count": 4 * Q,                          # idx in (counts are tiny)
+        "gate_count": 4 * N * E + 8 * Q,         # logits in; idx + w out (counts are tiny)
+        "count": 4 * Q,                          # idx in (the separate kernel)
         "plan": 0,                               # latency bound: reported in us
         "reroute": 4 * Q + 8 * Q,                # idx in; phys_slot + dest_row out
         "permute": 2 * N * d + 2 * Q * d,        # each row read once, written K times
@@ -97,6 +105,19 @@ def row_bytes(N=0, K=0, d=0, used=0, replicated=0, bytes_per_expert=0, numel=0):
         "weight_sync": 2 * used * bytes_per_expert,
         "grad_reduce": 4 * numel * (2 * replicated + used),
     }
+
+
+def kernels_per_step(w, num_sms=148):
+    """Kernel launches of one step: the gate with the count fused in (K = 8, E
+    a multiple of 32 from 64 to 256, each gate CTA's rows within four source
+    ranks), else the gate kernel plus the count kernel; then plan, reroute,
+    permute and combine. Mirrors the library's gate launch shape."""
+    fused = w.K == 8 and w.E % 32 == 0 and 64 <= w.E <= 256
+    if fused:
+        target = num_sms * 4
+        rpc = max(4, ((w.N + target - 1) // target + 3) // 4 * 4)
+        fused = (rpc + w.T - 1) // w.T + 1 <= 4
+    return 5 if fused else 6
 
 
 def load_peaks():
@@ -436,8 +457,7 @@ def run_sweep(args):
     opts = ue.plan_opts(ue.UE_SOLVER_BISECT) if args.planner == "bisect" else None
 
     def run_once(st):
-        L.gate(st)
-        L.count(st)
+        L.gate_count(st)
         if opts is None:
             L.plan_step(st)
         else:
@@ -500,7 +520,7 @@ def run_sweep(args):
                    "l2": "inputs larger than L2"},
         "us_per_layer": dist(times), "max_over_mean_before": dist(before),
         "max_over_mean_after": dist(after), "copies": dist(copies), "clocks": clk,
-        "gpu_launches": len(KERNELS) * len(times),
+        "gpu_launches": kernels_per_step(w) * len(times),
     }
     print(json.dumps(line), flush=True)
 
@@ -760,8 +780,7 @@ def run_planner(args, w):
                "bisect": ue.plan_opts(ue.UE_SOLVER_BISECT)}
     for target, alpha in instances:
         L.logits.copy_(torch.from_numpy(synth.logits(w, alpha=alpha)))
-        L.gate()
-        L.count()
+        L.gate_count()
         torch.cuda.synchronize(dev)
         load_e = L.load_e.cpu().numpy()
         before = float(load_e.reshape(w.R, M).sum(axis=1).max() / mean)
@@ -908,7 +927,7 @@ def main():
     LB.hidden.copy_(L.hidden)
     stream = torch.cuda.current_stream(dev)
 
-    steps_fn = [L.gate, L.count, L.plan_step, L.reroute, L.permute, L.combine]
+    steps_fn = [L.gate_count, L.plan_step, L.reroute, L.permute, L.combine]
 
     def step():
         for f in steps_fn:
@@ -936,7 +955,7 @@ def main():
             x = i % 2
             I = insts[x]
             side.wait_event(ev_done[x])
-            for f in (I.gate, I.count, I.plan_step, I.reroute):
+            for f in (I.gate_count, I.plan_step, I.reroute):
                 f(stream=side)
             ev_routed[x].record(side)
             stream.wait_event(ev_routed[x])
@@ -955,7 +974,7 @@ def main():
     torch.cuda.synchronize(dev)
     plan0 = L.plan_arrays()
 
-    # the step as one CUDA graph of the six kernels (captured once, outside
+    # the step as one CUDA graph of the path's kernels (captured once, outside
     # the timed region), so that the timed steps carry no launch gaps
     gstream = torch.cuda.Stream(dev)
     gstream.wait_stream(stream)
@@ -990,7 +1009,7 @@ def main():
     if rc != 0:
         raise SystemExit(f"device error in the timed region: {ue.STATUS.get(rc, rc)}")
 
-    # the same steps one after another, each one graph replay of the six
+    # the same steps one after another, each one graph replay of the path's
     # kernels on one instance (reported beside the value)
     torch.cuda.synchronize(dev)
     if world > 1:
@@ -1006,34 +1025,48 @@ def main():
     if rc != 0:
         raise SystemExit(f"device error in the serial steps: {ue.STATUS.get(rc, rc)}")
 
-    # per-kernel breakdown from eager launches bracketed by events (not part
-    # of the value): ev[s][k] .. ev[s][k+1] brackets kernel k of step s
-    nk = min(args.steps, 50)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(steps_fn) + 1)]
-           for _ in range(nk)]
-    for s in range(nk):
-        ev = evs[s]
-        ev[0].record(stream)
-        for k, f in enumerate(steps_fn):
-            f(stream=stream)
-            ev[k + 1].record(stream)
-    torch.cuda.synchronize(dev)
+    # per-kernel breakdown (not part of the value): each kernel alone, as
+    # replays of a CUDA graph of back-to-back launches on gstream (every
+    # kernel is idempotent on the instance's current buffers), timed with
+    # CUDA events on gstream; per launch = elapsed / launches
+    per_kernel_ms = {}
+    for name, f in zip(KERNELS, steps_fn):
+        reps = 4 if name in ("permute", "combine") else 20
+        gstream.wait_stream(stream)
+        with torch.cuda.stream(gstream):
+            f(stream=gstream)
+        torch.cuda.synchronize(dev)
+        kg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(kg, stream=gstream):
+            for _ in range(reps):
+                f(stream=gstream)
+        with torch.cuda.stream(gstream):
+            for _ in range(2):
+                kg.replay()
+        torch.cuda.synchronize(dev)
+        nrep = 3
+        ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(gstream):  # replay() launches on the current stream
+            ka.record(gstream)
+            for _ in range(nrep):
+                kg.replay()
+            kb.record(gstream)
+        torch.cuda.synchronize(dev)
+        per_kernel_ms[name] = ka.elapsed_time(kb) / (nrep * reps)
+        del kg
     clk = clocks.stop()
     rc = L.error(stream)
     if rc != 0:
         raise SystemExit(f"device error in the breakdown steps: {ue.STATUS.get(rc, rc)}")
     del graph
 
-    per_kernel_ms = {name: statistics.fmean(evs[s][k].elapsed_time(evs[s][k + 1])
-                                            for s in range(nk))
-                     for k, name in enumerate(KERNELS)}
     ms_step_local = total_ms / args.steps
     ms_step = max_over_ranks(ms_step_local, world, dev)
     value = world * w.Q / (ms_step / 1e3)
 
     # dominant kernel and its roofline
     abytes = algorithmic_bytes(w)
-    dom = max(("permute", "combine", "gate_topk", "reroute"), key=lambda k: per_kernel_ms[k])
+    dom = max(("permute", "combine", "gate_count", "reroute"), key=lambda k: per_kernel_ms[k])
     peak, peak_kind = load_peaks()
     achieved = abytes[dom] / (per_kernel_ms[dom] / 1e3) / 1e9
     tr = TRAFFIC.get(w.name, {}).get(dom)
@@ -1051,14 +1084,16 @@ def main():
             kernels[k].update(gbs=gbs, frac_of_peak=gbs / peak)
 
     cfg = workload_config(w)
-    gate_to_permute = sum(per_kernel_ms[k] for k in KERNELS[:5])
+    gate_to_permute = sum(per_kernel_ms[k] for k in KERNELS[:4])
     cfg.update(us_per_layer_gate_to_permute=1e3 * gate_to_permute,
                us_per_layer_incl_combine=1e3 * sum(per_kernel_ms.values()),
-               timing="exactly `steps` steps, each the six kernels over one batch; two layer "
-                      "instances alternate, and step i+1's routing (gate, count, plan, reroute) "
+               timing="exactly `steps` steps, each the path's five calls (gate with the count "
+                      "fused, plan, reroute, permute, combine) over one batch; two layer "
+                      "instances alternate, and step i+1's routing (gate and count, plan, reroute) "
                       "runs on a second stream during step i's permute and combine (events "
-                      "order each instance's uses); per-kernel times from eager launches "
-                      "bracketed by CUDA events",
+                      "order each instance's uses); per-kernel times: each kernel alone as CUDA "
+                      "graph replays of back-to-back launches (20, or 4 for permute and "
+                      "combine), CUDA events on the replay stream",
                ms_per_step_serial=serial_ms,
                serial="the same steps one after another, one CUDA graph replay each",
                parallelism=f"replicas: {world} independent layer instance(s), one per GPU")
@@ -1097,7 +1132,7 @@ def main():
             ev_in[b].record(s_in)
             s_run.wait_event(ev_in[b])
             s_run.wait_event(ev_out[b])          # its previous result has been read out
-            for f in [Lb.gate, Lb.count, Lb.plan_step, Lb.reroute, Lb.permute, Lb.combine]:
+            for f in [Lb.gate_count, Lb.plan_step, Lb.reroute, Lb.permute, Lb.combine]:
                 f(stream=s_run)
             ev_run[b].record(s_run)
             s_out.wait_event(ev_run[b])
@@ -1126,7 +1161,7 @@ def main():
         d2h = outs[0].numel() * 4 + stats_pin[0].numel() * 4
         e2e = {"value": world * w.Q / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "what": "every step: pinned host logits + hidden -> device, the six kernels, "
+               "what": "every step: pinned host logits + hidden -> device, the path's kernels, "
                        "fp32 combine output + plan stats -> pinned host; consecutive steps "
                        "pipelined over two buffer sets and three streams (upload, kernels, "
                        "readback overlap)"}
@@ -1155,7 +1190,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic", "config": cfg,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": len(steps_fn) * args.steps,
+            "gpu_launches": kernels_per_step(w) * args.steps,
             "clocks": clk, "kernels": kernels,
             "imbalance": {"max_over_mean_before": float(plan0["stats"][1]) / (w.Q / w.R),
                           "max_over_mean_after": float(plan0["stats"][2]) / (w.Q / w.R),

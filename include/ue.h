@@ -142,6 +142,17 @@ ue_status ue_gate_topk(ue_ctx* ctx, const float* logits, int32_t* idx,
 ue_status ue_count(ue_ctx* ctx, const int32_t* idx, int32_t* load_re,
                    int32_t* load_e, void* stream);
 
+/* ue_gate_topk and ue_count in one call: the same idx, w, load_re and load_e
+ * as the two calls in sequence (same arguments, same layouts, the same
+ * errors). For K = 8 and E a multiple of 32 from 64 to 256 the histogram is
+ * taken inside the gate kernel (each CTA adds its picks to a shared
+ * histogram per source rank and its bins to the outputs at the end), so
+ * idx is not read back; other shapes run the two kernels. Uses context
+ * scratch (a ticket, a counter, an epoch and a flag), so calls on one
+ * context must not overlap on the GPU. */
+ue_status ue_gate_count(ue_ctx* ctx, const float* logits, int32_t* idx, float* w,
+                        int32_t* load_re, int32_t* load_e, void* stream);
+
 /* Quota-driven replication plan ("How balancing in 300 microseconds works";
  * "Interface / 2. Forward and backward": update_placement).
  *   load_e int32 [E] exact per-expert pair counts, Q = sum(load_e).

@@ -25,7 +25,7 @@ import synth
 def test_totals_per_workload(name, gate_to_permute_gb, combine_gb):
     w = synth.WORKLOADS[name]
     b = bench.algorithmic_bytes(w)
-    g2p = sum(b[k] for k in ("gate_topk", "plan", "reroute", "permute"))
+    g2p = sum(b[k] for k in ("gate_count", "plan", "reroute", "permute"))
     assert abs(g2p / 1e9 - gate_to_permute_gb) < 0.005
     assert b["count"] == 4 * w.Q
     assert abs(b["combine"] / 1e9 - combine_gb) < 0.005
@@ -37,7 +37,7 @@ def test_per_step_counts_on_a_small_case():
     Q = N * K
     b = bench.algorithmic_bytes(w)
     assert b == {
-        "gate_topk": 4 * N * E + 4 * Q + 4 * Q,
+        "gate_count": 4 * N * E + 4 * Q + 4 * Q,
         "count": 4 * Q,
         "plan": 0,
         "reroute": 4 * Q + 4 * Q + 4 * Q,

@@ -3,7 +3,9 @@ benchmark times (Qwen3-shaped layer, DeepSeek-V3-shaped layer, EP40
 prefill), every output element against the oracle:
 
 * the routing half (top-k ids and weights, counts, every plan array, the
-  reroute): every element, bit-exact (weights within one ulp);
+  reroute): every element, bit-exact (weights within one ulp), through the
+  fused gate and count; the separate gate and count calls must give the
+  same bits;
 * the permute: every dispatch row against the oracle's permute, byte for
   byte;
 * the combine: every output element against the oracle's fp64 combine
@@ -42,6 +44,12 @@ def test_full_size_workload(name):
         assert L.error() == 0
         g = gh.routing_results(L)
         gh.assert_routing_equal(g, o)
+        # the separate gate and count calls give the same ids, weights and counts
+        fused = [t.clone() for t in (L.idx, L.w, L.load_re, L.load_e)]
+        L.gate()
+        L.count()
+        assert L.error() == 0
+        assert all(torch.equal(a, b) for a, b in zip(fused, (L.idx, L.w, L.load_re, L.load_e)))
 
         # every dispatch row
         gh.assert_dispatch_all_rows(L, hidden, w.K, o["dest_row"])

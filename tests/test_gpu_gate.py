@@ -1,4 +1,5 @@
-"""GPU parity of the gate's two selection paths for K = 8 and E = 128 or 256.
+"""GPU parity of the gate's two selection paths for K = 8 and E a multiple of
+32 from 64 to 256, and of the gate with the exact histogram fused in.
 
 The fast path ranks packed keys (an order key whose low log2(E) bits carry
 the expert id) and re-selects, with full keys and the lower-id tie rule, every
@@ -9,6 +10,12 @@ values a few fp32 ulps apart (both re-selected), with a ragged last group.
 Both paths must give the oracle's ids bit for bit and its weights within one
 fp32 ulp; a logits buffer that is not 16-byte aligned takes the generic
 kernel, which must agree as well.
+
+ue_gate_count must give the same ids and weights and the oracle's counts
+bit for bit, on shapes whose CTAs cover one to three source ranks (the
+histogram inside the gate kernel) and on one where they cover more (the
+gate kernel, then the count kernel), on calls in a row and on replays of a
+captured CUDA graph (the fused kernel's scratch is left ready by each launch).
 
 "UltraEP" README, "Interface / 2. Forward and backward" (probs, routing_map
 from the router); "What Happened" (routing from the exact probabilities).
@@ -64,7 +71,7 @@ def run_gate(E, N, logits, offset_floats=0):
         ue.ue_destroy(ctx)
 
 
-@pytest.mark.parametrize("E", [128, 256])
+@pytest.mark.parametrize("E", [64, 96, 128, 160, 192, 224, 256])
 @pytest.mark.parametrize("N", [2002, 4099])
 def test_packed_and_exact_rows_in_one_group(E, N):
     gh.ensure_built()
@@ -98,3 +105,60 @@ def test_all_rows_equal_pick_the_lowest_ids():
     idx, w = run_gate(E, N, logits)
     assert (idx == np.arange(8)).all()
     assert (w == np.float32(1.0 / 8)).all()
+
+
+def run_gate_count(R, T, E, logits_list, graph=False):
+    """ue_gate_count over each logits array in turn (eagerly, or as replays of
+    one captured graph); returns the outputs of every call."""
+    N, K = R * T, 8
+    dev = torch.device("cuda", 0)
+    cfg = ue.make_config(R, T, E, K, 1, 8)
+    ctx = ue.ue_init(cfg, 0)
+    try:
+        lg = torch.empty((N, E), dtype=torch.float32, device=dev)
+        idx = torch.full((N, K), -7, dtype=torch.int32, device=dev)
+        w = torch.full((N, K), -1.0, dtype=torch.float32, device=dev)
+        load_re = torch.full((R, E), 12345, dtype=torch.int32, device=dev)
+        load_e = torch.full((E,), 12345, dtype=torch.int32, device=dev)
+        s = torch.cuda.Stream(device=dev)
+        g = None
+        if graph:
+            lg.copy_(torch.from_numpy(logits_list[0]))
+            with torch.cuda.stream(s):
+                ue.ue_gate_count(ctx, lg, idx, w, load_re, load_e, s)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                ue.ue_gate_count(ctx, lg, idx, w, load_re, load_e, s)
+            torch.cuda.synchronize()
+        res = []
+        for logits in logits_list:
+            lg.copy_(torch.from_numpy(logits))
+            torch.cuda.synchronize()
+            if g is not None:
+                g.replay()
+            else:
+                ue.ue_gate_count(ctx, lg, idx, w, load_re, load_e)
+            assert ue.ue_get_error(ctx, s if g is not None else None) == ue.UE_OK
+            torch.cuda.synchronize()
+            res.append((idx.cpu().numpy(), w.cpu().numpy(), load_re.cpu().numpy(),
+                        load_e.cpu().numpy()))
+        return res
+    finally:
+        ue.ue_destroy(ctx)
+
+
+@pytest.mark.parametrize("R,T,E", [(2, 2049, 128), (128, 2, 128), (64, 3, 192), (40, 1001, 160),
+                                   (32, 777, 224), (32, 33, 96), (64, 65, 64), (8, 4099, 256),
+                                   (128, 1, 256)])
+@pytest.mark.parametrize("graph", [False, True])
+def test_gate_count_matches_the_oracle(R, T, E, graph):
+    gh.ensure_built()
+    lgs = [mixed_logits(R * T, E, seed=R * 1000 + T + s) for s in range(3)]
+    for logits, (idx, w, load_re, load_e) in zip(lgs, run_gate_count(R, T, E, lgs, graph)):
+        idx_or, w_or = oracle.gate_topk(logits, 8)
+        np.testing.assert_array_equal(idx, idx_or)
+        gh.assert_weights_close(w, w_or)
+        lre_or, le_or = oracle.count(idx_or, R, T, E)
+        np.testing.assert_array_equal(load_re, lre_or)
+        np.testing.assert_array_equal(load_e, le_or)

@@ -65,8 +65,7 @@ def test_sweep_graph_captured(planner):
     opts = ue.plan_opts(ue.UE_SOLVER_BISECT) if planner == "bisect" else None
 
     def run_once(st):
-        L.gate(st)
-        L.count(st)
+        L.gate_count(st)
         if opts is None:
             L.plan_step(st)
         else:

@@ -33,7 +33,7 @@ UE_OK, UE_ERR_INVALID_ARG, UE_ERR_CUDA, UE_ERR_NOMEM = 0, 1, 2, 3
 UE_ERR_DEVICE_BOUNDS, UE_ERR_TIMEOUT, UE_ERR_UNSUPPORTED = 4, 5, 6
 
 # every symbol include/ue.h declares
-EXPORTS = ("ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count",
+EXPORTS = ("ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count", "ue_gate_count",
            "ue_plan", "ue_plan_ex", "ue_reroute", "ue_reroute_ex", "ue_locality_split",
            "ue_reroute_local", "ue_permute", "ue_combine", "ue_combine_backward",
            "ue_permute_backward", "ue_weight_sync", "ue_grad_reduce", "ue_reroute_noalloc",
@@ -96,6 +96,7 @@ def load_library(path: str | None = None):
     lib.ue_destroy.argtypes = [vp]
     lib.ue_get_error.argtypes = [vp, vp]
     lib.ue_gate_topk.argtypes = [vp, vp, vp, vp, vp]
+    lib.ue_gate_count.argtypes = [vp, vp, vp, vp, vp, vp, vp]
     lib.ue_count.argtypes = [vp, vp, vp, vp, vp]
     lib.ue_plan.argtypes = [vp, vp, ctypes.POINTER(ue_placement), vp]
     lib.ue_plan_ex.argtypes = [vp, vp, ctypes.POINTER(ue_plan_opts), ctypes.POINTER(ue_placement),
@@ -169,6 +170,12 @@ def ue_get_error(ctx, stream=None) -> int:
 def ue_gate_topk(ctx, logits, idx, w, stream=None):
     _ok("ue_gate_topk", load_library().ue_gate_topk(ctx, _ptr(logits), _ptr(idx), _ptr(w),
                                                     _stream(stream)))
+
+
+def ue_gate_count(ctx, logits, idx, w, load_re, load_e, stream=None):
+    _ok("ue_gate_count", load_library().ue_gate_count(ctx, _ptr(logits), _ptr(idx), _ptr(w),
+                                                      _ptr(load_re), _ptr(load_e),
+                                                      _stream(stream)))
 
 
 def ue_count(ctx, idx, load_re, load_e, stream=None):
@@ -275,7 +282,7 @@ def ue_debug_drop_first_publish(ctx, enable: bool):
 
 from .layer import Layer  # noqa: E402  (buffers + one call per step)
 
-__all__ = ["ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count", "ue_plan",
+__all__ = ["ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count", "ue_gate_count", "ue_plan",
            "ue_plan_ex", "ue_reroute_ex", "ue_locality_split", "ue_reroute_local",
            "ue_plan_opts", "plan_opts", "UE_SOLVER_GREEDY", "UE_SOLVER_BISECT",
            "UE_ORDER_PREFIX", "UE_ORDER_INTERLEAVE",

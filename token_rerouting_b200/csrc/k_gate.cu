@@ -161,29 +161,55 @@ gate_topk_kernel(const float* __restrict__ logits, int64_t N, int E, int Krt,
 }
 
 // ---------------------------------------------------------------------------
-// Fast path for K = 8 and E = 32 * VPL, VPL in {4, 8} (E = 128 or 256).
+// Fast path for K = 8 and E = 128 * NCH4 + 32 * NT (a multiple of 32, 64 to
+// 256), optionally with the exact histogram fused in.
 //
 // Each logit's order key keeps its high bits and carries (E-1-e) in its low
-// log2(E) bits, so keys are unique within a row and a round of the selection
-// is one `redux` max and a pop. The packed order is the exact order (larger
-// value first, lower id first among equal values) wherever the values differ
-// above the dropped bits. A (K+1)-th round checks exactly that: if the first
-// K+1 packed picks of a row differ pairwise in their high parts (adjacent
-// ones suffice: they are sorted), every unpicked key lies strictly below the
-// K-th pick, and the picks are in exact order. Rows that fail the check (two
-// of the leading values within 2^-16 relative of each other, or exact ties)
-// are selected again with full keys and the id tie rule from the copy of the
-// row staged in shared memory. The results are identical to the generic
-// kernel's in every case.
+// LOB bits (7 for E <= 128, 8 above), so keys are unique within a row and a
+// round of the selection is one `redux` max and a pop. The packed order is
+// the exact order (larger value first, lower id first among equal values)
+// wherever the values differ above the dropped bits. A (K+1)-th round checks
+// exactly that: if the first K+1 packed picks of a row differ pairwise in
+// their high parts (adjacent ones suffice: they are sorted), every unpicked
+// key lies strictly below the K-th pick, and the picks are in exact order.
+// Rows that fail the check (two of the leading values within 2^-16 relative
+// of each other, or exact ties) are selected again with full keys and the
+// id tie rule, from the row read again (an L1 hit: the loads allocate in
+// L1). The results are identical to the generic kernel's in every case.
 //
-// Lane l holds experts e = 128 c + 4 l + j (chunk c < VPL/4, j < 4): one
-// 16-byte load per chunk, ids ascending along the lane's list.
+// Lane l holds experts e = 128 c + 4 l + j (chunk c < NCH4, j < 4: one
+// 16-byte load per chunk) and then 128 NCH4 + 32 t + l (t < NT: one 4-byte
+// load each), ids ascending along the lane's list.
+//
+// Each CTA owns a contiguous block of rows, so with the count fused it
+// touches only a few source ranks: each pick is added to a shared histogram
+// per source rank, and the CTA adds its non-zero bins to load_re and load_e
+// at the end. The outputs are zeroed by the first CTA to take a ticket
+// (which waits for nothing, so it always runs), which then sets a flag;
+// every CTA waits for that flag (bounded) before its global atomics. The
+// flag carries the launch epoch, and the last CTA to finish resets the
+// ticket and advances the epoch, so nothing is cleared between launches.
 constexpr int kFastK = 8;
 constexpr int kFastRows = 32 / kFastK;  // rows per warp group
 constexpr int kGateWarps = kGateThreads / 32;
+constexpr int kGateHist = 4;            // source ranks one CTA may touch (fused count)
+constexpr long long kGateWaitLimit = 1LL << 22;
 
-// Order key of a finite float with -0.0 made +0.0 first (the sum -0 + +0 is
-// +0 under round-to-nearest; finite inputs are otherwise unchanged).
+// packed key: order key of the finite float v (-0.0 made +0.0 first; the sum
+// -0 + +0 is +0 under round-to-nearest) with its low bits replaced by lo:
+// x = u ^ (s & 0x7fffffff) ^ 0x80000000 with s the sign mask (lop3 0x1e),
+// then (x & khi) | lo (lop3 0xea)
+__device__ __forceinline__ uint32_t packed_key(float v, uint32_t lo, uint32_t khi)
+{
+    const uint32_t u = __float_as_uint(__fadd_rn(v, 0.0f));
+    const uint32_t sgn = (uint32_t)((int32_t)u >> 31);
+    uint32_t x, k;
+    asm("lop3.b32 %0, %1, %2, %3, 0x1e;" : "=r"(x) : "r"(u), "r"(sgn), "r"(0x80000000u));
+    asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(k) : "r"(x), "r"(khi), "r"(lo));
+    return k;
+}
+
+// full order key of a finite float (-0.0 made +0.0 first)
 __device__ __forceinline__ uint32_t order_key_finite(float v)
 {
     const uint32_t u = __float_as_uint(__fadd_rn(v, 0.0f));
@@ -197,16 +223,36 @@ __device__ __forceinline__ void cas_desc(uint32_t& a, uint32_t& b)
     b = lo;
 }
 
-// descending sort of distinct keys by a sorting network (5 or 19 comparators)
+// descending sort of distinct keys by a sorting network
 template <int VPL>
 __device__ __forceinline__ void sort_desc(uint32_t (&k)[VPL])
 {
-    if constexpr (VPL == 4) {
+    if constexpr (VPL == 2) {
+        cas_desc(k[0], k[1]);
+    } else if constexpr (VPL == 3) {
+        cas_desc(k[0], k[1]); cas_desc(k[1], k[2]); cas_desc(k[0], k[1]);
+    } else if constexpr (VPL == 4) {
         cas_desc(k[0], k[1]); cas_desc(k[2], k[3]);
         cas_desc(k[0], k[2]); cas_desc(k[1], k[3]);
         cas_desc(k[1], k[2]);
+    } else if constexpr (VPL == 5) {
+        cas_desc(k[0], k[1]); cas_desc(k[3], k[4]); cas_desc(k[2], k[4]);
+        cas_desc(k[2], k[3]); cas_desc(k[0], k[3]); cas_desc(k[0], k[2]);
+        cas_desc(k[1], k[4]); cas_desc(k[1], k[3]); cas_desc(k[1], k[2]);
+    } else if constexpr (VPL == 6) {
+        cas_desc(k[1], k[2]); cas_desc(k[4], k[5]); cas_desc(k[0], k[2]);
+        cas_desc(k[3], k[5]); cas_desc(k[0], k[1]); cas_desc(k[3], k[4]);
+        cas_desc(k[2], k[5]); cas_desc(k[0], k[3]); cas_desc(k[1], k[4]);
+        cas_desc(k[2], k[4]); cas_desc(k[1], k[3]); cas_desc(k[2], k[3]);
+    } else if constexpr (VPL == 7) {
+        cas_desc(k[1], k[2]); cas_desc(k[3], k[4]); cas_desc(k[5], k[6]);
+        cas_desc(k[0], k[2]); cas_desc(k[3], k[5]); cas_desc(k[4], k[6]);
+        cas_desc(k[0], k[1]); cas_desc(k[4], k[5]); cas_desc(k[2], k[6]);
+        cas_desc(k[0], k[4]); cas_desc(k[1], k[5]); cas_desc(k[0], k[3]);
+        cas_desc(k[2], k[5]); cas_desc(k[1], k[3]); cas_desc(k[2], k[4]);
+        cas_desc(k[2], k[3]);
     } else {
-        static_assert(VPL == 8, "fast gate path: VPL 4 or 8");
+        static_assert(VPL == 8, "fast gate path: 2 to 8 values per lane");
         cas_desc(k[0], k[1]); cas_desc(k[2], k[3]); cas_desc(k[4], k[5]); cas_desc(k[6], k[7]);
         cas_desc(k[0], k[2]); cas_desc(k[1], k[3]); cas_desc(k[4], k[6]); cas_desc(k[5], k[7]);
         cas_desc(k[1], k[2]); cas_desc(k[5], k[6]);
@@ -216,21 +262,49 @@ __device__ __forceinline__ void sort_desc(uint32_t (&k)[VPL])
     }
 }
 
+template <int NCH4, int NT>
+struct FastRow {
+    static constexpr int VPL = 4 * NCH4 + NT;
+    float4 c4[NCH4 > 0 ? NCH4 : 1];
+    float t1[NT > 0 ? NT : 1];
+
+    __device__ __forceinline__ void load(const float* row, int lane, bool ok)
+    {
+#pragma unroll
+        for (int c = 0; c < NCH4; ++c)
+            c4[c] = ok ? __ldg(reinterpret_cast<const float4*>(row) + c * 32 + lane)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) t1[t] = ok ? __ldg(row + 128 * NCH4 + 32 * t + lane) : 0.f;
+    }
+    __device__ __forceinline__ float at(int i) const
+    {
+        if (i < 4 * NCH4) {
+            const float4 x = c4[i >> 2];
+            const int j = i & 3;
+            return j == 0 ? x.x : j == 1 ? x.y : j == 2 ? x.z : x.w;
+        }
+        return t1[i - 4 * NCH4];
+    }
+};
+
+// expert id held in position i of lane `lane`'s list
+template <int NCH4>
+__device__ __forceinline__ int fast_expert(int i, int lane)
+{
+    return i < 4 * NCH4 ? 128 * (i >> 2) + 4 * lane + (i & 3) : 128 * NCH4 + 32 * (i - 4 * NCH4) + lane;
+}
+
 // The K+1 packed picks of one row into win[0..K]; lane 0 writes them.
-template <int VPL>
-__device__ __forceinline__ void select_packed(const float4 (&v)[VPL / 4], const uint32_t (&lo)[VPL],
+template <int NCH4, int NT>
+__device__ __forceinline__ void select_packed(const FastRow<NCH4, NT>& v,
+                                              const uint32_t (&lo)[4 * NCH4 + NT], uint32_t khi,
                                               uint32_t* win, bool writer)
 {
-    constexpr int LOB = VPL == 4 ? 7 : 8;
-    constexpr uint32_t kHi = ~((1u << LOB) - 1u);
+    constexpr int VPL = 4 * NCH4 + NT;
     uint32_t key[VPL];
 #pragma unroll
-    for (int c = 0; c < VPL / 4; ++c) {
-        key[4 * c + 0] = (order_key_finite(v[c].x) & kHi) | lo[4 * c + 0];
-        key[4 * c + 1] = (order_key_finite(v[c].y) & kHi) | lo[4 * c + 1];
-        key[4 * c + 2] = (order_key_finite(v[c].z) & kHi) | lo[4 * c + 2];
-        key[4 * c + 3] = (order_key_finite(v[c].w) & kHi) | lo[4 * c + 3];
-    }
+    for (int i = 0; i < VPL; ++i) key[i] = packed_key(v.at(i), lo[i], khi);
     sort_desc<VPL>(key);
 #pragma unroll
     for (int k = 0; k < kFastK; ++k) {
@@ -245,22 +319,21 @@ __device__ __forceinline__ void select_packed(const float4 (&v)[VPL / 4], const 
     if (writer) win[kFastK] = m;
 }
 
-// Exact selection of one staged row: full keys, equal keys to the lower id.
-// win[k] = E-1-e_k, which decodes like a packed pick.
-template <int VPL>
-__device__ __forceinline__ void select_exact_staged(const float4* row, int lane, uint32_t* win)
+// Exact selection of one row read again from global memory: full keys,
+// equal keys to the lower id. win[k] = E-1-e_k, which decodes like a packed
+// pick.
+template <int NCH4, int NT>
+__device__ __forceinline__ void select_exact_row(const float* row, int lane, uint32_t* win)
 {
-    constexpr int E = 32 * VPL;
+    constexpr int VPL = 4 * NCH4 + NT;
+    constexpr int E = 128 * NCH4 + 32 * NT;
+    FastRow<NCH4, NT> v;
+    v.load(row, lane, true);
     uint32_t key[VPL], ke[VPL];
 #pragma unroll
-    for (int c = 0; c < VPL / 4; ++c) {
-        const float4 x = row[c * 32 + lane];
-        const float xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            key[4 * c + j] = order_key_finite(xs[j]);
-            ke[4 * c + j] = (uint32_t)(128 * c + 4 * lane + j);
-        }
+    for (int i = 0; i < VPL; ++i) {
+        key[i] = order_key_finite(v.at(i));
+        ke[i] = (uint32_t)fast_expert<NCH4>(i, lane);
     }
     // stable descending bubble sort: equal keys keep the lower id first
 #pragma unroll
@@ -293,54 +366,77 @@ __device__ __forceinline__ void select_exact_staged(const float4* row, int lane,
     }
 }
 
-template <int VPL>
-__global__ void __launch_bounds__(kGateThreads, 4)
-gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int32_t* __restrict__ idx,
-                      float* __restrict__ w)
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p)
 {
-    constexpr int E = 32 * VPL;
-    constexpr int NCH = VPL / 4;
-    constexpr int LOB = VPL == 4 ? 7 : 8;
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+template <int NCH4, int NT, bool COUNT>
+__global__ void __launch_bounds__(kGateThreads, 4)
+gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_per_cta,
+                      int32_t* __restrict__ idx, float* __restrict__ w, GateCount cnt)
+{
+    constexpr int VPL = 4 * NCH4 + NT;
+    constexpr int E = 128 * NCH4 + 32 * NT;
+    constexpr int LOB = E <= 128 ? 7 : 8;
     constexpr uint32_t kLo = (1u << LOB) - 1u;
-    __shared__ float4 s_row[kGateWarps][kFastRows][E / 4];
+    constexpr uint32_t kHi = ~kLo;
+    constexpr int HE = COUNT ? E : 1;
     __shared__ uint32_t s_win[kGateWarps][kFastRows][kFastK + 1];
+    __shared__ int s_hist[COUNT ? kGateHist : 1][HE];
+    __shared__ uint32_t s_epoch, s_ticket, s_ok;
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int64_t gwarp = (int64_t)blockIdx.x * kGateWarps + warp;
-    const int64_t nwarps = (int64_t)gridDim.x * kGateWarps;
-    const int64_t ngroups = (N + kFastRows - 1) / kFastRows;
+    const int64_t row_beg = (int64_t)blockIdx.x * rows_per_cta;
+    const int64_t row_end = min(N, row_beg + rows_per_cta);
+    int64_t rank0 = 0;
+    if constexpr (COUNT) {
+        for (int x = threadIdx.x; x < kGateHist * E; x += blockDim.x) (&s_hist[0][0])[x] = 0;
+        if (threadIdx.x == 0) {
+            s_epoch = *reinterpret_cast<volatile uint32_t*>(cnt.sync + 2);
+            s_ticket = atomicAdd(cnt.sync, 1u);
+        }
+        __syncthreads();
+        if (s_ticket == 0u) {
+            // the first CTA zeroes the outputs, then sets the flag
+            const int re = cnt.R * E;
+            for (int x = threadIdx.x; x < re; x += blockDim.x) cnt.load_re[x] = 0;
+            for (int x = threadIdx.x; x < E; x += blockDim.x) cnt.load_e[x] = 0;
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) st_release_gpu(cnt.sync + 3, s_epoch + 1u);
+        }
+        rank0 = row_beg / cnt.T;
+    }
+
     uint32_t lo[VPL];
 #pragma unroll
-    for (int c = 0; c < NCH; ++c)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) lo[4 * c + j] = (uint32_t)(E - 1 - (128 * c + 4 * lane + j));
+    for (int i = 0; i < VPL; ++i) lo[i] = (uint32_t)(E - 1 - fast_expert<NCH4>(i, lane));
     const int r = lane / kFastK;   // this lane's row of the group in the epilogue
     const int k = lane % kFastK;   // and its rank among the row's picks
 
-    for (int64_t grp = gwarp; grp < ngroups; grp += nwarps) {
-        const int64_t row0 = grp * kFastRows;
-        const int rows = (int)min((int64_t)kFastRows, N - row0);
-        float4 v[kFastRows][NCH];
+    for (int64_t row0 = row_beg + (int64_t)warp * kFastRows; row0 < row_end;
+         row0 += (int64_t)kGateWarps * kFastRows) {
+        const int rows = (int)min((int64_t)kFastRows, row_end - row0);
+        FastRow<NCH4, NT> v[kFastRows];
 #pragma unroll
-        for (int b = 0; b < kFastRows; ++b) {
-            const float4* src = reinterpret_cast<const float4*>(logits + (row0 + b) * (int64_t)E);
-#pragma unroll
-            for (int c = 0; c < NCH; ++c)
-                v[b][c] = b < rows ? __ldcs(src + c * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int b = 0; b < kFastRows; ++b)
-#pragma unroll
-            for (int c = 0; c < NCH; ++c) s_row[warp][b][c * 32 + lane] = v[b][c];
+        for (int b = 0; b < kFastRows; ++b) v[b].load(logits + (row0 + b) * (int64_t)E, lane, b < rows);
         if (rows == kFastRows) {
 #pragma unroll
             for (int b = 0; b < kFastRows; ++b)
-                select_packed<VPL>(v[b], lo, s_win[warp][b], lane == 0);
+                select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0);
         } else {
 #pragma unroll
             for (int b = 0; b < kFastRows; ++b)
-                if (b < rows) select_packed<VPL>(v[b], lo, s_win[warp][b], lane == 0);
+                if (b < rows) select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0);
         }
         __syncwarp();
         // rows whose leading picks agree above the dropped bits: exact again
@@ -350,13 +446,15 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int32_t* __re
         unsigned redo = __ballot_sync(kFull, act && (a >> LOB) == (nx >> LOB));
         while (redo) {
             const int rr = (__ffs(redo) - 1) / kFastK;
-            select_exact_staged<VPL>(s_row[warp][rr], lane, s_win[warp][rr]);
+            select_exact_row<NCH4, NT>(logits + (row0 + rr) * (int64_t)E, lane, s_win[warp][rr]);
             redo &= ~(0xffu << (rr * kFastK));
         }
         __syncwarp();
         // gate weights of the whole group at once, fp64
-        const uint32_t e = (uint32_t)(E - 1) - (s_win[warp][r][k] & kLo);
-        const float vf = reinterpret_cast<const float*>(s_row[warp][r])[e];
+        // (lanes of rows past the end hold stale picks: they read nothing)
+        const int e = act ? (E - 1) - (int)(s_win[warp][r][k] & kLo) : 0;
+        const int64_t row = row0 + (act ? r : 0);
+        const float vf = act ? __ldg(logits + row * (int64_t)E + e) : 0.0f;
         const int lead = act ? r * kFastK : 0;
         const double v_own = (double)vf;
         const double v0 = __shfl_sync(kFull, v_own, lead);
@@ -365,12 +463,72 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int32_t* __re
 #pragma unroll
         for (int kk = 0; kk < kFastK; ++kk) z += __shfl_sync(kFull, x, act ? lead + kk : 0);
         if (act) {
-            const int64_t pos = (row0 + r) * (int64_t)kFastK + k;
+            const int64_t pos = row * (int64_t)kFastK + k;
             idx[pos] = (int32_t)e;
             w[pos] = (float)(x / z);
+            if constexpr (COUNT) {
+                // source rank of the row, relative to the CTA's first rank
+                const int64_t rel = row - rank0 * cnt.T;
+                int hs = 0;
+#pragma unroll
+                for (int q = 1; q < kGateHist; ++q) hs += rel >= (int64_t)q * cnt.T ? 1 : 0;
+                atomicAdd(&s_hist[hs][e], 1);
+            }
         }
-        __syncwarp();  // the staged rows and picks are rewritten by the next group
+        __syncwarp();  // the picks are rewritten by the next group
     }
+
+    if constexpr (COUNT) {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t ok = 0u;
+            for (long long spin = 0; spin < kGateWaitLimit; ++spin) {
+                if (ld_acquire_gpu(cnt.sync + 3) == s_epoch + 1u) {
+                    ok = 1u;
+                    break;
+                }
+                __nanosleep(64);
+            }
+            if (!ok) raise_error(cnt.err, UE_ERR_TIMEOUT, (int)blockIdx.x);
+            s_ok = ok;
+        }
+        __syncthreads();
+        if (s_ok) {
+            for (int x = threadIdx.x; x < kGateHist * E; x += blockDim.x) {
+                const int h = (&s_hist[0][0])[x];
+                if (h) {
+                    const int hs = x / E, ex = x - hs * E;
+                    atomicAdd(&cnt.load_re[(rank0 + hs) * E + ex], h);
+                    atomicAdd(&cnt.load_e[ex], h);
+                }
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            const uint32_t done = atomicAdd(cnt.sync + 1, 1u);
+            if (done == gridDim.x - 1) {
+                // last CTA: ready for the next launch
+                cnt.sync[0] = 0u;
+                cnt.sync[1] = 0u;
+                __threadfence();
+                cnt.sync[2] = s_epoch + 1u;
+            }
+        }
+    }
+}
+
+template <int NCH4, int NT>
+cudaError_t launch_fast(const Sizes& z, const GateShape& sh, const float* logits, int32_t* idx,
+                        float* w, const GateCount* cnt, cudaStream_t st)
+{
+    if (cnt != nullptr)
+        gate_topk_fast_kernel<NCH4, NT, true><<<sh.grid, kGateThreads, 0, st>>>(
+            logits, z.N, sh.rows_per_cta, idx, w, *cnt);
+    else
+        gate_topk_fast_kernel<NCH4, NT, false><<<sh.grid, kGateThreads, 0, st>>>(
+            logits, z.N, sh.rows_per_cta, idx, w, GateCount{});
+    return cudaGetLastError();
 }
 
 template <int VPL>
@@ -388,40 +546,72 @@ cudaError_t launch_vpl(const Sizes& z, const float* logits, int32_t* idx,
 
 }  // namespace
 
-int gate_topk_grid(const Sizes& z, int num_sms)
+bool gate_fast_shape(const Sizes& z)
 {
+    return z.K == kFastK && z.E % 32 == 0 && z.E >= 64 && z.E <= 256;
+}
+
+GateShape plan_gate_shape(const Sizes& z, int num_sms)
+{
+    GateShape sh;
+    // generic kernel: grid-stride over warp groups, at most 4 CTAs per SM
     const int rpg = 32 / z.K;
     const int64_t groups = (z.N + rpg - 1) / rpg;
     const int64_t blocks_needed = (groups + (kGateThreads / 32) - 1) / (kGateThreads / 32);
-    const int64_t cap = (int64_t)num_sms * 4;
-    return (int)std::max<int64_t>(1, std::min(blocks_needed, cap));
+    sh.grid = (int)std::max<int64_t>(1, std::min(blocks_needed, (int64_t)num_sms * 4));
+    sh.rows_per_cta = 0;
+    sh.fast = gate_fast_shape(z) ? 1 : 0;
+    sh.fused = 0;
+    if (sh.fast) {
+        // contiguous blocks of whole warp groups, one wave of at most 4 CTAs per SM
+        const int64_t target = std::max<int64_t>(1, (int64_t)num_sms * 4);
+        int64_t rpc = (z.N + target - 1) / target;
+        rpc = std::max<int64_t>(kFastRows, (rpc + kFastRows - 1) / kFastRows * kFastRows);
+        sh.rows_per_cta = rpc;
+        sh.grid = (int)std::max<int64_t>(1, (z.N + rpc - 1) / rpc);
+        // the fused count needs every CTA's rows within kGateHist source ranks
+        const int64_t spans = (rpc + z.T - 1) / z.T + 1;
+        sh.fused = spans <= kGateHist ? 1 : 0;
+    }
+    return sh;
 }
 
-cudaError_t launch_gate_topk(const Sizes& z, const float* logits, int32_t* idx,
-                             float* w, int grid, cudaStream_t st)
+cudaError_t launch_gate_topk(const Sizes& z, const GateShape& sh, const float* logits,
+                             int32_t* idx, float* w, const GateCount* cnt, cudaStream_t st)
 {
-    if (z.N == 0) return cudaSuccess;
-    if (z.K == kFastK && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0) {
-        if (z.E == 128) {
-            gate_topk_fast_kernel<4><<<grid, kGateThreads, 0, st>>>(logits, z.N, idx, w);
-            return cudaGetLastError();
-        }
-        if (z.E == 256) {
-            gate_topk_fast_kernel<8><<<grid, kGateThreads, 0, st>>>(logits, z.N, idx, w);
-            return cudaGetLastError();
-        }
+    if (z.N == 0) {
+        if (cnt == nullptr) return cudaSuccess;
+        return launch_count(z, idx, cnt->load_re, cnt->load_e, cnt->err, st);
     }
+    if (sh.fast && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0) {
+        const GateCount* fc = (cnt != nullptr && sh.fused) ? cnt : nullptr;
+        cudaError_t ce;
+        switch (z.E) {
+        case 64: ce = launch_fast<0, 2>(z, sh, logits, idx, w, fc, st); break;
+        case 96: ce = launch_fast<0, 3>(z, sh, logits, idx, w, fc, st); break;
+        case 128: ce = launch_fast<1, 0>(z, sh, logits, idx, w, fc, st); break;
+        case 160: ce = launch_fast<1, 1>(z, sh, logits, idx, w, fc, st); break;
+        case 192: ce = launch_fast<1, 2>(z, sh, logits, idx, w, fc, st); break;
+        case 224: ce = launch_fast<1, 3>(z, sh, logits, idx, w, fc, st); break;
+        default: ce = launch_fast<2, 0>(z, sh, logits, idx, w, fc, st); break;
+        }
+        if (ce != cudaSuccess || cnt == nullptr || fc != nullptr) return ce;
+        return launch_count(z, idx, cnt->load_re, cnt->load_e, cnt->err, st);
+    }
+    cudaError_t ce;
     switch ((z.E + 31) / 32) {
-    case 1: return launch_vpl<1>(z, logits, idx, w, grid, st);
-    case 2: return launch_vpl<2>(z, logits, idx, w, grid, st);
-    case 3: return launch_vpl<3>(z, logits, idx, w, grid, st);
-    case 4: return launch_vpl<4>(z, logits, idx, w, grid, st);
-    case 5: return launch_vpl<5>(z, logits, idx, w, grid, st);
-    case 6: return launch_vpl<6>(z, logits, idx, w, grid, st);
-    case 7: return launch_vpl<7>(z, logits, idx, w, grid, st);
-    case 8: return launch_vpl<8>(z, logits, idx, w, grid, st);
+    case 1: ce = launch_vpl<1>(z, logits, idx, w, sh.grid, st); break;
+    case 2: ce = launch_vpl<2>(z, logits, idx, w, sh.grid, st); break;
+    case 3: ce = launch_vpl<3>(z, logits, idx, w, sh.grid, st); break;
+    case 4: ce = launch_vpl<4>(z, logits, idx, w, sh.grid, st); break;
+    case 5: ce = launch_vpl<5>(z, logits, idx, w, sh.grid, st); break;
+    case 6: ce = launch_vpl<6>(z, logits, idx, w, sh.grid, st); break;
+    case 7: ce = launch_vpl<7>(z, logits, idx, w, sh.grid, st); break;
+    case 8: ce = launch_vpl<8>(z, logits, idx, w, sh.grid, st); break;
     default: return cudaErrorInvalidValue;
     }
+    if (ce != cudaSuccess || cnt == nullptr) return ce;
+    return launch_count(z, idx, cnt->load_re, cnt->load_e, cnt->err, st);
 }
 
 }  // namespace ue

@@ -20,65 +20,50 @@
 //
 // Design (B200): the greedy is serial, so its speed is the latency of one
 // iteration. The choice of e* depends only on the copy counts, never on the
-// ranks: the sequence of experts the greedy picks is fixed by the loads
-// alone (a highest-ratio apportionment). So two warps of one CTA run it as a
-// pipeline:
-//  - warp 1 (expert side) produces the picks in order: e*, its new copy
-//    count and the quota parameters of that step, pushed into a shared-memory
-//    queue with a ready flag per entry. L/c is compared through the integer
-//    key floor(L*2^24/c), one 64-bit multiply-high with a table of
-//    ceil(2^64/c); for c <= 257 and L < 2^30 the map is exact and order
-//    preserving (two different ratios differ by more than 1/66049, i.e. by
-//    more than 250 after scaling; equal ratios give equal keys). The expert id
-//    sits below the key, so the argmax with ties to the lowest e is two warp
-//    `redux` max reductions. An expert that may not grow has key 0; when
-//    every key is 0 the expert side pushes an end marker (e = -1).
-//  - warp 0 (rank side) keeps the rank loads and the redundant slots in
-//    registers (lane l owns ranks l, l+32, ... and their slots, so every
-//    load change lands in the lane that owns the rank). Per iteration: the
-//    stop test and the least loaded rank with a free slot (two `redux`
-//    reductions, max load and min of (load << 7 | r), when Q < 2^25; three
-//    otherwise), with the pick's ready flag and the pick itself loaded before
-//    them, the
-//    placement in r*'s lowest free slot, and the new quotas of e*'s copies: the
-//    master's goes from ceil(L/(c-1)) to ceil(L/c); a first replica takes
-//    floor(L/2); later replicas are found by ballots in ascending slot order.
-//    The count of co-located copies does not depend on the order of
-//    placement and is taken from the final slots.
-// Warp 1 needs far fewer instructions per step, so warp 0 rarely waits; its
-// wait on a queue entry is bounded. The rest of the CTA writes the outputs
-// and scans the slot offsets at the end.
+// ranks: the experts the greedy picks, in order, are fixed by the loads
+// alone. Each step takes the largest current ratio L_e/c_e (ties to the
+// lowest e) and then moves e to L_e/(c_e+1), so the picks are the keys
+// (L_e/c, e), c = 1, 2, ..., in descending order of ratio (equal ratios:
+// lower e first), truncated where an expert may not grow. One CTA therefore
+// computes the whole pick sequence in parallel before the serial part:
+//  - candidates: with Q > 0 every key of ratio >= Q/(G+E) is kept, c <= min(G,
+//    floor(L_e (G+E) / Q)) per expert. That is at least G + 1 keys when no
+//    expert is capped (sum floor(x_e) > sum x_e - E = G) and at most G + E,
+//    so the top G keys are among them. With a minimum per replica some
+//    experts are capped (c <= floor(L_e/m) - 1); while the candidates are
+//    fewer than G and some expert is cut by the threshold, the threshold is
+//    halved (at most 2G + E candidates);
+//  - each candidate is one 64-bit key: floor(L_e 2^17 / c) (exact and order
+//    preserving for c <= 257: two different ratios differ by more than
+//    2^-17), then 255 - e, then c - 1; a bitonic sort in shared memory puts
+//    them in pick order, and each pick's quota parameters follow in
+//    parallel (fewer than G picks end with an end marker).
+// Then one warp runs the rank side alone, with the picks already in shared
+// memory: it keeps the rank loads and the redundant slots in registers (lane
+// l owns ranks l, l+32, ... and their slots, so every load change lands in
+// the lane that owns the rank). Per iteration: the stop test and the least
+// loaded rank with a free slot (two `redux` reductions, max load and min of
+// (load << 7 | r), when Q < 2^25; three otherwise), the placement in r*'s
+// lowest free slot, and the new quotas of e*'s copies: the master's goes
+// from ceil(L/(c-1)) to ceil(L/c); a first replica takes floor(L/2); later
+// replicas are found by ballots in ascending slot order. The count of
+// co-located copies does not depend on the order of placement and is taken
+// from the final slots. The rest of the CTA writes the outputs and scans the
+// slot offsets at the end.
 #include "ue_internal.cuh"
 
 namespace ue {
 namespace {
 
-constexpr int kPlanThreads = 256;
+constexpr int kPlanThreads = 512;
 constexpr int kPlanWarps = kPlanThreads / 32;
-constexpr int kKeyShift = 24;
-constexpr long long kPickWaitLimit = 1LL << 24;
+constexpr int kRatioShift = 17;
+constexpr int kCandMax = 1024;  // candidate keys: at most 2G + E <= 768
 
 __device__ __forceinline__ unsigned div_by(unsigned x, unsigned c, const unsigned long long* recip)
 {
     // floor(x / c) for x < 2^40, c <= 257: exact with ceil(2^64 / c)
     return c == 1u ? x : (unsigned)__umul64hi((unsigned long long)x, recip[c]);
-}
-
-// floor(L * 2^24 / c) with the expert id below it: larger ratio first, then
-// lower id
-__device__ __forceinline__ unsigned long long packed_key(unsigned L, unsigned c, int e,
-                                                         const unsigned long long* recip)
-{
-    const unsigned long long x = (unsigned long long)L << kKeyShift;
-    const unsigned long long k = c == 1u ? x : __umul64hi(x, recip[c]);
-    return (k << 9) | (unsigned long long)(511 - e);
-}
-
-// may an expert with load L and c copies take copy c+1 and keep at least m
-// pairs on each?
-__device__ __forceinline__ bool may_grow(unsigned L, unsigned c, unsigned m)
-{
-    return (unsigned long long)m * (c + 1u) <= (unsigned long long)L;
 }
 
 struct Pick {
@@ -90,20 +75,35 @@ struct Pick {
     int rm;        // the master's rank, e / M
 };
 
-template <int NJE, int NJR, int SM>
+// block-wide sum of v over all threads (every thread gets the total)
+__device__ __forceinline__ long long block_sum(long long v, long long* scratch)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    __syncthreads();
+    if (lane == 0) scratch[warp] = v;
+    __syncthreads();
+    long long t = 0;
+    for (int w = 0; w < kPlanWarps; ++w) t += scratch[w];
+    return t;
+}
+
+template <int NJR, int SM>
 __global__ void __launch_bounds__(kPlanThreads, 1)
 plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned min_tokens,
             ue_placement out, int* err)
 {
     __shared__ unsigned long long sRecip[kMaxG + 2];  // ceil(2^64 / c), c = 2 .. G+1
     __shared__ int sL[kMaxE];       // exact load per expert
+    __shared__ int sCnt[kMaxE + 1]; // candidates per expert, then their exclusive scan
     __shared__ int sC[kMaxE];       // copies per expert (final)
     __shared__ int sRank[kMaxR];    // rank loads (initial, then final)
     __shared__ int sSlotE[kMaxG];   // expert of redundant slot g, -1 empty (final)
     __shared__ int sSlotQ[kMaxG];   // quota of redundant slot g (final)
-    __shared__ Pick sPick[kMaxG];   // the expert side's picks, in order
-    __shared__ volatile int sReady[kMaxG];
-    __shared__ volatile int sDone;  // the rank side has stopped
+    __shared__ unsigned long long sKey[kCandMax];
+    __shared__ Pick sPick[kMaxG + 1];  // the picks in order (then an end marker)
+    __shared__ long long sRed[kPlanWarps];
     __shared__ int sUsedPicks;
     __shared__ unsigned long long sQ;
     __shared__ int sStats[4];
@@ -114,15 +114,15 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
     const int G = R * S;
     const int P = R * (M + S);
     const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
 
     if (tid == 0) {
         sQ = 0ull;
         sUsedPicks = 0;
-        sDone = 0;
         sColoc = 0;
     }
     for (int r = tid; r < R; r += blockDim.x) sRank[r] = 0;
-    for (int g = tid; g < G; g += blockDim.x) sReady[g] = 0;
     for (int c = tid + 2; c <= G + 1; c += blockDim.x)
         sRecip[c] = (0xffffffffffffffffull / (unsigned long long)c) + 1ull;
     __syncthreads();
@@ -139,69 +139,112 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
     }
     if (part) atomicAdd(&sQ, part);
     __syncthreads();
+    const unsigned long long Qall = sQ;
 
-    const int warp = tid >> 5;
-    const int lane = tid & 31;
-    if (warp == 1) {
-        // ---- expert side: the greedy's picks, independent of the ranks ----
-        unsigned Lr[NJE], cr[NJE];
-        unsigned long long key[NJE];
-#pragma unroll
-        for (int j = 0; j < NJE; ++j) {
-            const int e = lane + 32 * j;
-            Lr[j] = e < E ? (unsigned)sL[e] : 0u;
-            cr[j] = 1u;
-            key[j] = (e < E && may_grow(Lr[j], 1u, min_tokens)) ? packed_key(Lr[j], 1u, e, sRecip)
-                                                                 : 0ull;
-        }
-        for (int t = 0; t < G; ++t) {
-            if (__any_sync(kFull, sDone != 0)) break;
-            unsigned long long best = 0ull;
-#pragma unroll
-            for (int j = 0; j < NJE; ++j) best = key[j] > best ? key[j] : best;
-            const unsigned hi = __reduce_max_sync(kFull, (unsigned)(best >> 32));
-            const unsigned lo = __reduce_max_sync(kFull, (unsigned)(best >> 32) == hi ? (unsigned)best : 0u);
-            if (hi == 0u && lo == 0u) {
-                // no expert may take another copy: end marker
-                if (lane == 0) {
-                    sPick[t] = Pick{-1, 0u, 0u, 0u, 0u, 0};
-                    __threadfence_block();
-                    sReady[t] = 1;
+    // ---- the pick sequence, in parallel ----
+    // candidates per expert at threshold Q/(G+E)/2^lvl (one thread per expert)
+    int total = 0;
+    if (Qall > 0ull && G > 0) {
+        for (int lvl = 0;; ++lvl) {
+            int cnt = 0, cut = 0;
+            if (tid < E) {
+                const long long L = sL[tid];
+                long long cap = G;
+                if (min_tokens > 0u) cap = min(cap, L / (long long)min_tokens - 1);
+                if (L > 0 && cap > 0) {
+                    const unsigned long long num = (unsigned long long)L * (unsigned)(G + E);
+                    const unsigned long long q = num / Qall, r = num - q * Qall;
+                    long long th;
+                    if (lvl >= 10 && q > 0ull) th = cap;  // q * 2^lvl >= 1024 > cap
+                    else th = (long long)((q << lvl) + ((r << lvl) / Qall));
+                    cnt = (int)min(cap, th);
+                    cut = th < cap;
                 }
-                break;
+                sCnt[tid] = cnt;
             }
-            const int estar = 511 - (int)(lo & 511u);
-            const int ej = estar >> 5;
-            unsigned Le = 0u, ce = 0u;
-#pragma unroll
-            for (int j = 0; j < NJE; ++j)
-                if (j == ej) {
-                    Le = Lr[j];
-                    ce = cr[j];
-                }
-            Le = __shfl_sync(kFull, Le, estar & 31);
-            ce = __shfl_sync(kFull, ce, estar & 31) + 1u;
-            const unsigned long long nk =
-                may_grow(Le, ce, min_tokens) ? packed_key(Le, ce, estar, sRecip) : 0ull;
-            if (lane == (estar & 31)) {
-#pragma unroll
-                for (int j = 0; j < NJE; ++j)
-                    if (j == ej) {
-                        cr[j] = ce;
-                        key[j] = nk;
-                    }
-            }
-            if (lane == 0) {
-                const unsigned qb = div_by(Le, ce, sRecip);
-                const unsigned rem = Le - qb * ce;
-                const unsigned q0_new = qb + (rem > 0u ? 1u : 0u);
-                const unsigned q0_old = div_by(Le + ce - 2u, ce - 1u, sRecip);
-                sPick[t] = Pick{estar, ce, qb, rem, q0_new - q0_old, estar / M};
-                __threadfence_block();
-                sReady[t] = 1;
-            }
+            const long long both = block_sum(((long long)cut << 32) | cnt, sRed);
+            total = (int)(both & 0xffffffffll);
+            if (total >= G || (both >> 32) == 0 || lvl >= 33) break;
         }
-    } else if (warp == 0) {
+    } else if (tid < E) {
+        sCnt[tid] = 0;
+    }
+    __syncthreads();
+    // exclusive scan of the counts (E <= 256 <= blockDim)
+    {
+        const int c = tid < E ? sCnt[tid] : 0;
+        int incl = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off) incl += o;
+        }
+        if (lane == 31) sWarpSum[warp] = incl;
+        __syncthreads();
+        int wofs = 0;
+        for (int w = 0; w < warp; ++w) wofs += sWarpSum[w];
+        __syncthreads();
+        if (tid < E) sCnt[tid] = wofs + incl - c;
+        if (tid == 0) sCnt[E] = total;
+    }
+    __syncthreads();
+    // the keys: position p belongs to the expert whose range holds it
+    int n = 2;
+    while (n < total) n <<= 1;
+    for (int p = tid; p < n; p += blockDim.x) {
+        unsigned long long key = 0ull;
+        if (p < total) {
+            int lo = 0, hi = E - 1;  // last e with sCnt[e] <= p
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (sCnt[mid] <= p) lo = mid;
+                else hi = mid - 1;
+            }
+            const int e = lo;
+            const unsigned c = (unsigned)(p - sCnt[e] + 1);
+            const unsigned long long x = (unsigned long long)sL[e] << kRatioShift;
+            const unsigned long long ratio = c == 1u ? x : __umul64hi(x, sRecip[c]);
+            key = (ratio << 16) | ((unsigned long long)(255 - e) << 8) | (c - 1u);
+        }
+        sKey[p] = key;
+    }
+    __syncthreads();
+    // bitonic sort, descending
+    for (int k = 2; k <= n; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int q = tid; q < (n >> 1); q += blockDim.x) {
+                const int i = (q / j) * 2 * j + (q % j);
+                const int ij = i + j;
+                const unsigned long long a = sKey[i], b = sKey[ij];
+                const bool desc = (i & k) == 0;
+                if (desc ? (a < b) : (a > b)) {
+                    sKey[i] = b;
+                    sKey[ij] = a;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    const int npicks = min(G, total);
+    for (int t = tid; t <= npicks && t < G + 1; t += blockDim.x) {
+        if (t == npicks) {
+            sPick[t] = Pick{-1, 0u, 0u, 0u, 0u, 0};
+        } else {
+            const unsigned long long key = sKey[t];
+            const int e = 255 - (int)((key >> 8) & 255ull);
+            const unsigned c = (unsigned)(key & 255ull) + 1u;  // copies before the pick
+            const unsigned ce = c + 1u;
+            const unsigned Le = (unsigned)sL[e];
+            const unsigned qb = div_by(Le, ce, sRecip);
+            const unsigned rem = Le - qb * ce;
+            const unsigned q0_new = qb + (rem > 0u ? 1u : 0u);
+            const unsigned q0_old = div_by(Le + c - 1u, c, sRecip);
+            sPick[t] = Pick{e, ce, qb, rem, q0_new - q0_old, e / M};
+        }
+    }
+    __syncthreads();
+
+    if (warp == 0) {
         // ---- rank side: stop test, least loaded free rank, bookkeeping ----
         const long long Q = (long long)sQ;
         const long long stop_rhs = 51LL * Q;
@@ -225,22 +268,12 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
         // index (< 128) pack into one 32-bit key, and the least loaded rank
         // with a free slot (ties to the lowest r) is one reduction
         const bool packed = Q < (1LL << 25);
+        Pick pk = sPick[0];
         for (;;) {
-            // this iteration's pick: its flag is read first and the pick
-            // right after it (acquire orders the read), so that both loads
-            // overlap the reductions below; a pick read before its flag was
-            // set is read again after the wait
-            // (iters reaches G only when every slot is used and the loop is
-            // about to stop; the index is clamped so that these early reads
-            // stay inside the arrays)
-            const int it0 = iters < kMaxG ? iters : kMaxG - 1;
-            int ready = 0;
-            asm volatile("ld.acquire.cta.shared.u32 %0, [%1];"
-                         : "=r"(ready)
-                         : "r"((unsigned)__cvta_generic_to_shared((const void*)&sReady[it0]))
-                         : "memory");
-            const int ready0 = ready;
-            const Pick pk_early = sPick[it0];
+            // the next pick is read now, so that its load overlaps the
+            // reductions (iters + 1 <= G always: the loop stops once every
+            // slot is used)
+            const Pick pk_next = sPick[min(iters + 1, kMaxG)];
             unsigned maxl = 0u, bestl = 0xffffffffu, bestr = 0xffffffffu;
             int rstar;
             if (packed) {
@@ -273,19 +306,6 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
                 rstar = (int)__reduce_min_sync(kFull, bestl == ml ? bestr : 0xffffffffu);
             }
 
-            // the pick is normally ready long before: the expert side needs
-            // far fewer instructions per step. The wait is bounded.
-            for (long long spin = 0; !ready && spin < kPickWaitLimit; ++spin)
-                asm volatile("ld.acquire.cta.shared.u32 %0, [%1];"
-                             : "=r"(ready)
-                             : "r"((unsigned)__cvta_generic_to_shared((const void*)&sReady[iters]))
-                             : "memory");
-            ready = __all_sync(kFull, ready);
-            if (!ready) {
-                if (lane == 0) raise_error(err, UE_ERR_TIMEOUT, iters);
-                break;
-            }
-            const Pick pk = ready0 ? pk_early : sPick[iters];
             if (pk.e < 0) break;  // no expert may take another copy
             const int estar = pk.e;
             const int rj = rstar >> 5;
@@ -336,12 +356,12 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
 #pragma unroll
                 for (int j = 0; j < NJR; ++j) {
                     unsigned lower = 0u;   // e* replicas in lower lanes of group j
-                    unsigned total = 0u;   // e* replicas in group j
+                    unsigned grp = 0u;     // e* replicas in group j
 #pragma unroll
                     for (int s = 0; s < SM; ++s) {
                         const unsigned msk = __ballot_sync(kFull, s < S && slotE[j][s] == estar);
                         lower += __popc(msk & lt);
-                        total += __popc(msk);
+                        grp += __popc(msk);
                     }
                     unsigned mine = 0u;  // e* replicas in this lane's lower slots
 #pragma unroll
@@ -354,10 +374,11 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
                             mine += 1u;
                         }
                     }
-                    before += total;
+                    before += grp;
                 }
             }
             iters += 1;
+            pk = pk_next;
         }
         unsigned mx = 0u;
 #pragma unroll
@@ -380,7 +401,6 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
             sStats[1] = (int)max_before;
             sStats[2] = (int)mx;
             sUsedPicks = iters;
-            sDone = 1;
         }
     }
     __syncthreads();
@@ -450,24 +470,15 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
     if (tid == 0) out.slot_offset[P] = (int)sQ;
 }
 
-template <int NJE, int NJR>
+template <int NJR>
 cudaError_t launch_s(const Sizes& z, const int32_t* load_e, unsigned m, const ue_placement& out,
                      int* err, cudaStream_t st)
 {
     if (z.S <= 2)
-        plan_kernel<NJE, NJR, 2><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, m, out, err);
+        plan_kernel<NJR, 2><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, m, out, err);
     else
-        plan_kernel<NJE, NJR, 8><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, m, out, err);
+        plan_kernel<NJR, 8><<<1, kPlanThreads, 0, st>>>(load_e, z.R, z.E, z.S, m, out, err);
     return cudaGetLastError();
-}
-
-template <int NJE>
-cudaError_t launch_r(const Sizes& z, const int32_t* load_e, unsigned m, const ue_placement& out,
-                     int* err, cudaStream_t st)
-{
-    if (z.R <= 32) return launch_s<NJE, 1>(z, load_e, m, out, err, st);
-    if (z.R <= 64) return launch_s<NJE, 2>(z, load_e, m, out, err, st);
-    return launch_s<NJE, 4>(z, load_e, m, out, err, st);
 }
 
 }  // namespace
@@ -476,10 +487,9 @@ cudaError_t launch_plan(const Sizes& z, const int32_t* load_e, int min_tokens,
                         const ue_placement& out, int* err, cudaStream_t st)
 {
     const unsigned m = (unsigned)min_tokens;
-    if (z.E <= 32) return launch_r<1>(z, load_e, m, out, err, st);
-    if (z.E <= 64) return launch_r<2>(z, load_e, m, out, err, st);
-    if (z.E <= 128) return launch_r<4>(z, load_e, m, out, err, st);
-    return launch_r<8>(z, load_e, m, out, err, st);
+    if (z.R <= 32) return launch_s<1>(z, load_e, m, out, err, st);
+    if (z.R <= 64) return launch_s<2>(z, load_e, m, out, err, st);
+    return launch_s<4>(z, load_e, m, out, err, st);
 }
 
 }  // namespace ue

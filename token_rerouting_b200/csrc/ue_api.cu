@@ -12,13 +12,14 @@ struct ue_ctx {
     ue::Sizes z;
     int device;
     int num_sms;
-    int gate_grid;
+    ue::GateShape gate;
     ue::PermuteShape perm;
     ue::CombineShape comb;
     ue::BwdShape bwd;       // combine backward launch shape
     int* d_err;             // [2] error code, detail
     unsigned long long* d_status;  // [tiles][E] reroute look-back words
     uint32_t* d_sync;       // [4] reroute ticket, finished CTAs, epoch
+    uint32_t* d_gsync;      // [4] fused gate count: ticket, finished CTAs, epoch, flag
     int32_t* d_first;       // [R][P] locality order: first occurrence index
     int32_t* d_rowb;        // [R][P] locality order: row base
     uint16_t* d_zrow;       // [d] zeros: the combine reads it for a row out of range
@@ -81,7 +82,7 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
     ctx->z = ue::make_sizes(*cfg);
     ctx->device = device;
     ctx->num_sms = prop.multiProcessorCount;
-    ctx->gate_grid = ue::gate_topk_grid(ctx->z, ctx->num_sms);
+    ctx->gate = ue::plan_gate_shape(ctx->z, ctx->num_sms);
     ctx->tiles = (ctx->z.Q + ue::kRerouteTile - 1) / ue::kRerouteTile;
     ctx->spin_limit = 1LL << 22;
     ctx->drop_first = 0;
@@ -100,6 +101,7 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
     if (cudaMalloc(&ctx->d_err, 2 * sizeof(int)) != cudaSuccess ||
         cudaMalloc(&ctx->d_status, status_words * sizeof(unsigned long long)) != cudaSuccess ||
         cudaMalloc(&ctx->d_sync, 4 * sizeof(uint32_t)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_gsync, 4 * sizeof(uint32_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_first, table_words * sizeof(int32_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_rowb, table_words * sizeof(int32_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_zrow, (size_t)ctx->z.d * sizeof(uint16_t)) != cudaSuccess ||
@@ -107,6 +109,7 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
         cudaFree(ctx->d_err);
         cudaFree(ctx->d_status);
         cudaFree(ctx->d_sync);
+        cudaFree(ctx->d_gsync);
         cudaFree(ctx->d_first);
         cudaFree(ctx->d_rowb);
         cudaFree(ctx->d_zrow);
@@ -118,11 +121,13 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
     if (cudaMemset(ctx->d_err, 0, 2 * sizeof(int)) != cudaSuccess ||
         cudaMemset(ctx->d_status, 0, status_words * sizeof(unsigned long long)) != cudaSuccess ||
         cudaMemset(ctx->d_sync, 0, 4 * sizeof(uint32_t)) != cudaSuccess ||
+        cudaMemset(ctx->d_gsync, 0, 4 * sizeof(uint32_t)) != cudaSuccess ||
         cudaMemset(ctx->d_zrow, 0, (size_t)ctx->z.d * sizeof(uint16_t)) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess) {
         cudaFree(ctx->d_err);
         cudaFree(ctx->d_status);
         cudaFree(ctx->d_sync);
+        cudaFree(ctx->d_gsync);
         cudaFree(ctx->d_first);
         cudaFree(ctx->d_rowb);
         cudaFree(ctx->d_zrow);
@@ -144,6 +149,7 @@ ue_status ue_destroy(ue_ctx* ctx)
     cudaFree(ctx->d_err);
     cudaFree(ctx->d_status);
     cudaFree(ctx->d_sync);
+    cudaFree(ctx->d_gsync);
     cudaFree(ctx->d_first);
     cudaFree(ctx->d_rowb);
     cudaFree(ctx->d_zrow);
@@ -172,7 +178,19 @@ ue_status ue_gate_topk(ue_ctx* ctx, const float* logits, int32_t* idx, float* w,
     if (!ctx_ok(ctx) || !aligned(logits, 4) || !aligned(idx, 4) || !aligned(w, 4))
         return UE_ERR_INVALID_ARG;
     if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
-    return from_cuda(ue::launch_gate_topk(ctx->z, logits, idx, w, ctx->gate_grid,
+    return from_cuda(ue::launch_gate_topk(ctx->z, ctx->gate, logits, idx, w, nullptr,
+                                          as_stream(stream)));
+}
+
+ue_status ue_gate_count(ue_ctx* ctx, const float* logits, int32_t* idx, float* w,
+                        int32_t* load_re, int32_t* load_e, void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(logits, 4) || !aligned(idx, 4) || !aligned(w, 4) ||
+        !aligned(load_re, 4) || !aligned(load_e, 4))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    const ue::GateCount cnt{load_re, load_e, ctx->d_gsync, ctx->d_err, ctx->cfg.T, ctx->cfg.R};
+    return from_cuda(ue::launch_gate_topk(ctx->z, ctx->gate, logits, idx, w, &cnt,
                                           as_stream(stream)));
 }
 

@@ -79,8 +79,29 @@ inline Sizes make_sizes(const ue_config& c)
 
 // Launch helpers, one per kernel family. Each returns the CUDA error of the
 // launch (cudaSuccess if nothing was launched because there was no work).
-cudaError_t launch_gate_topk(const Sizes& z, const float* logits, int32_t* idx,
-                             float* w, int grid, cudaStream_t st);
+// Gate launch shape, fixed once per context: `fast` (K = 8, E a multiple of
+// 32 from 64 to 256) uses contiguous blocks of rows_per_cta rows per CTA;
+// `fused` means the exact histogram can be taken inside that kernel.
+struct GateShape {
+    int grid;
+    int64_t rows_per_cta;
+    int fast, fused;
+};
+// The fused histogram's outputs and scratch: sync[0..3] = {ticket, finished
+// CTAs, launch epoch, zeroed-outputs flag}, zeroed once; each launch leaves
+// them ready for the next one.
+struct GateCount {
+    int32_t* load_re;
+    int32_t* load_e;
+    uint32_t* sync;
+    int* err;
+    int T, R;
+};
+GateShape plan_gate_shape(const Sizes& z, int num_sms);
+// cnt == nullptr: top-k and weights only; otherwise also the exact histogram
+// (inside the gate kernel when the shape allows, else by launch_count)
+cudaError_t launch_gate_topk(const Sizes& z, const GateShape& sh, const float* logits,
+                             int32_t* idx, float* w, const GateCount* cnt, cudaStream_t st);
 cudaError_t launch_count(const Sizes& z, const int32_t* idx, int32_t* load_re,
                          int32_t* load_e, int* err, cudaStream_t st);
 // greedy plan; min_tokens = 0: every expert may take a copy
@@ -137,7 +158,6 @@ cudaError_t launch_combine(const Sizes& z, const CombineShape& sh, const uint16_
                            const int32_t* dest_row, const float* w, float* out,
                            const uint16_t* zrow, int* err, cudaStream_t st);
 
-int gate_topk_grid(const Sizes& z, int num_sms);
 
 // Beside the forward path: backward of the combine (the permute's backward
 // is launch_combine with w == nullptr), weight sync and gradient reduction.

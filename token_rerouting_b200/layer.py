@@ -9,7 +9,8 @@ dispatch (permute) -> experts (outside; identity here unless ``y`` is given)
 """
 from __future__ import annotations
 
-from . import (make_config, placement, ue_combine, ue_count, ue_destroy, ue_gate_topk,
+from . import (make_config, placement, ue_combine, ue_count, ue_destroy, ue_gate_count,
+               ue_gate_topk,
                ue_get_error, ue_init, ue_locality_split, ue_permute, ue_plan, ue_plan_ex,
                ue_reroute, ue_reroute_ex, ue_reroute_local)
 
@@ -61,6 +62,10 @@ class Layer:
     def count(self, stream=None):
         ue_count(self.ctx, self.idx, self.load_re, self.load_e, stream)
 
+    def gate_count(self, stream=None):
+        """Top-k, weights and the exact histogram in one call."""
+        ue_gate_count(self.ctx, self.logits, self.idx, self.w, self.load_re, self.load_e, stream)
+
     def plan_step(self, stream=None):
         ue_plan(self.ctx, self.load_e, self.plan, stream)
 
@@ -90,9 +95,14 @@ class Layer:
         ue_combine(self.ctx, self.dispatch if y is None else y, self.dest_row, self.w,
                    self.out, stream)
 
-    def run_routing(self, stream=None):
-        self.gate(stream)
-        self.count(stream)
+    def run_routing(self, stream=None, fused=True):
+        """gate -> count -> plan -> reroute; with fused=True the gate and the
+        count are one call (ue_gate_count)."""
+        if fused:
+            self.gate_count(stream)
+        else:
+            self.gate(stream)
+            self.count(stream)
         self.plan_step(stream)
         self.reroute(stream)
 
