@@ -360,19 +360,20 @@ ue_status ue_grad_reduce(ue_ctx* ctx, const ue_placement* plan, const float* rep
  * pages have no counterpart to this call). For callers that cannot call
  * cudaMalloc: code running inside an allocator's hooks or under a memory
  * pool that forbids outside allocations, or code that keeps no context.
- * The look-back scratch is a fixed device array inside libue (2 MiB plus a
- * few words, held on every GPU that loads the library until the process
+ * The look-back scratch is a fixed device array inside libue (about
+ * 2.2 MiB, held on every GPU that loads the library until the process
  * exits): sizes with ceil(R*T*K / 8192) * E > 262144 are rejected with
  * UE_ERR_UNSUPPORTED before anything is launched. The first call made with
  * a given device current checks that the device is an sm_100 part
  * (UE_ERR_UNSUPPORTED otherwise), looks up that array's device address
- * (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture. cudaDeviceReset makes the cached address stale: do not
+ * (cudaGetSymbolAddress), caches it and sets the reroute kernel's shared
+ * memory limit; make that first call before any stream capture. cudaDeviceReset makes the cached address stale: do not
  * call this entry point again in a process that has reset the device.
  * Every call shares the array and it is never cleared: its status words
  * carry the call's epoch, so words left by an earlier call read as
- * unpublished, and each call's last CTA resets the tile ticket, also after
- * a call that ended in a device-side error. Calls that overlap on the GPU
+ * unpublished, each group of tiles' last arrival resets the group's
+ * counter, and each call's last CTA resets the tile ticket, also after a
+ * call that ended in a device-side error. Calls that overlap on the GPU
  * (other streams, other threads) race and give wrong results. Calls no
  * cudaMalloc or cudaFree.
  *   cfg, idx, plan, phys_slot, dest_row, stream: as for ue_init + ue_reroute

@@ -45,12 +45,9 @@
 namespace ue {
 namespace {
 
-constexpr int kTile = kRerouteTile;
 constexpr int kThreads = kRerouteThreads;
 constexpr int kWarps = kRerouteWarps;
-constexpr int kPerWarp = kTile / kWarps;
-constexpr int kRounds = kPerWarp / 32;
-constexpr int kWindow = 16;  // predecessors read per thread per look-back step
+constexpr int kWindow = 16;  // look-back items read per thread at a time
 constexpr int kMaxH = 4;     // threads per expert column in the look-back
 
 __device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p)
@@ -148,39 +145,55 @@ __device__ __forceinline__ int64_t pair_at(int64_t u, const OrderArgs& o)
     return ((int64_t)r * o.T + t) * o.K + k;
 }
 
-template <int kOrder>
-__global__ void __launch_bounds__(kThreads)
+// wait (bounded) until *p holds a word of this launch, then return it in w;
+// false when the wait ran out
+__device__ __forceinline__ bool wait_word(const unsigned long long* p, uint32_t tag,
+                                          unsigned long long& w, int64_t& polls,
+                                          int64_t spin_limit)
+{
+    while ((uint32_t)(w >> 32) != tag || ((uint32_t)w >> 30) == kFlagInvalid) {
+        if (++polls > spin_limit) return false;
+        __nanosleep(64);
+        w = ld_relaxed(p);
+    }
+    return true;
+}
+
+template <int kOrder, int kPer>
+__global__ void __launch_bounds__(kThreads, 2)
 reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
                ue_placement plan, OrderArgs ord, int32_t* __restrict__ phys_slot,
-               int32_t* __restrict__ dest_row, unsigned long long* status,
-               uint32_t* sync, int64_t spin_limit, int drop_first,
-               int* err)
+               int32_t* __restrict__ dest_row, RerouteScratch sc, int64_t spin_limit,
+               int drop_first, int* err)
 {
-    __shared__ short s_idx[kTile];        // expert ids of the tile (-1: none)
+    constexpr int kTileP = kThreads * kPer;    // pairs per tile
+    constexpr int kPerWarpP = kTileP / kWarps;  // pairs per warp sub-range
+    extern __shared__ __align__(16) short s_idx[];  // [kTileP] expert ids of the tile (-1: none)
     __shared__ short s_wh[kWarps][kMaxE]; // per-warp counts, then in-tile offsets
     __shared__ ExpA s_a[kMaxE];
     __shared__ ExpB s_bm[kMaxE];
     __shared__ ExpC s_c[kMaxE];
     __shared__ int s_cp[kMaxE + kMaxG];   // copy table: physical slot, copies of
     __shared__ int s_cr[kMaxE + kMaxG];   // each expert in order; first dispatch row;
-    __shared__ int s_cs[kMaxE + kMaxG];   // first pair index o of the copy
+    __shared__ int s_cs[kMaxE + kMaxG + 1];  // first pair index o of the copy
+    __shared__ short s_ce[kMaxE + kMaxG];    // expert of each copy-table entry
     __shared__ union {
         struct {  // building the copy table
-            int cnt[kMaxE], run[kMaxE];
+            int cnt[kMaxE], run[kMaxE], base[kMaxE], ff[kMaxE];
             int off[kMaxE + kMaxG + 1];   // plan: slot_offset
             int se[kMaxG];                // plan: slot_expert
             int sq[kMaxE + kMaxG];        // plan: slot_quota
         } pro;
-        struct {  // look-back: one window segment per (h, e)
+        struct {  // look-back: one partial sum per (h, e)
             uint32_t part[kMaxH][kMaxE];
             unsigned char state[kMaxH][kMaxE];
-            unsigned char cdone[kMaxE];  // column finished
         } lb;
     } u;
     __shared__ int s_wsum[kWarps];
     __shared__ int s_tile;
     __shared__ uint32_t s_tag;
     __shared__ int s_fail;
+    __shared__ int s_fin;
 
     const int M = E / R;
     const int G = R * S;
@@ -188,29 +201,35 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
+    const int ntiles = (int)gridDim.x;
 
     if (tid == 0) {
-        s_tile = (int)atomicAdd(&sync[0], 1u);
+        s_tile = (int)atomicAdd(&sc.sync[0], 1u);
         // this launch's tag; the epoch only moves after every CTA has read it
-        const uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(&sync[2]);
+        const uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(&sc.sync[2]);
         s_tag = epoch + 1u == 0u ? 1u : epoch + 1u;
         s_fail = 0;
     }
     for (int x = tid; x < kWarps * kMaxE; x += kThreads) (&s_wh[0][0])[x] = 0;
     for (int e = tid; e < E; e += kThreads) {
         u.pro.cnt[e] = 0;
-        u.pro.run[e] = 0;
+        u.pro.ff[e] = 1;
     }
+    // the plan, into registers now (its loads overlap the tile's)
+    int pl_off0 = 0, pl_off1 = 0, pl_sq = 0, pl_se = -1;
+    if (tid <= P) pl_off0 = __ldg(plan.slot_offset + tid);
+    if (tid + kThreads <= P) pl_off1 = __ldg(plan.slot_offset + tid + kThreads);
+    if (tid < P) pl_sq = __ldg(plan.slot_quota + tid);
+    if (tid < G) pl_se = __ldg(plan.slot_expert + tid);
     __syncthreads();
 
     // ---- stage the tile and count it per warp sub-range ----
     const int tile = s_tile;
     const uint32_t tag = s_tag;
-    const int64_t t0 = (int64_t)tile * kTile;
-    const int cnt_tile = (int)min((int64_t)kTile, Q - t0);
+    const int64_t t0 = (int64_t)tile * kTileP;
+    const int cnt_tile = (int)min((int64_t)kTileP, Q - t0);
     {
         // issue all of this thread's loads before using any of them
-        constexpr int kPer = kTile / kThreads;
         int v[kPer];
 #pragma unroll
         for (int q = 0; q < kPer; ++q) {
@@ -231,34 +250,69 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     }
     __syncthreads();
 #pragma unroll 4
-    for (int rd = 0; rd < kRounds; ++rd) {
-        const int e = s_idx[warp * kPerWarp + rd * 32 + lane];
+    for (int rd = 0; rd < kPer; ++rd) {
+        const int e = s_idx[warp * kPerWarpP + rd * 32 + lane];
         if (e >= 0) atomicAdd_block(reinterpret_cast<int*>(&s_wh[warp][0]) + (e >> 1),
                                     (e & 1) ? (1 << 16) : 1);
     }
     __syncthreads();
 
-    // ---- publish this tile's counts ----
+    // ---- publish this tile's counts and arrive at its group ----
     int acc = 0;
-    unsigned long long* mine = status + (size_t)tile * E + tid;
     if (tid < E) {
         for (int w = 0; w < kWarps; ++w) {
             const int t = s_wh[w][tid];
             s_wh[w][tid] = (short)acc;
             acc += t;
         }
-        if (tile == 0) {
-            if (!drop_first) st_relaxed(mine, status_word(tag, kFlagPrefix, (uint32_t)acc));
-        } else {
-            st_relaxed(mine, status_word(tag, kFlagAggregate, (uint32_t)acc));
+        if (!(drop_first && tile == 0))
+            st_relaxed(sc.status + (size_t)tile * E + tid,
+                       status_word(tag, kFlagAggregate, (uint32_t)acc));
+    }
+    const int grp = tile / kRerouteGroup;
+    const int gfirst = grp * kRerouteGroup;
+    const int members = min(kRerouteGroup, ntiles - gfirst);
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        s_fin = atomicAdd(&sc.gcount[grp], 1u) == (uint32_t)(members - 1) ? 1 : 0;
+        __threadfence();
+    }
+    // the plan into shared memory
+    if (tid <= P) u.pro.off[tid] = pl_off0;
+    if (tid + kThreads <= P) u.pro.off[tid + kThreads] = pl_off1;
+    if (tid < P) u.pro.sq[tid] = pl_sq;
+    if (tid < G) u.pro.se[tid] = pl_se;
+    __syncthreads();
+    if (s_fin) {
+        // the last tile of the group to arrive publishes the group's sum (its
+        // members published their counts before they arrived)
+        if (tid < E) {
+            unsigned long long v[kRerouteGroup];
+#pragma unroll
+            for (int i = 0; i < kRerouteGroup; ++i)
+                v[i] = i < members ? ld_relaxed(sc.status + (size_t)(gfirst + i) * E + tid) : 0ull;
+            uint32_t sum = 0, flag = kFlagAggregate;
+            int64_t polls = 0;
+#pragma unroll
+            for (int i = 0; i < kRerouteGroup; ++i) {
+                if (i < members && flag == kFlagAggregate) {
+                    if (wait_word(sc.status + (size_t)(gfirst + i) * E + tid, tag, v[i], polls,
+                                  spin_limit)) {
+                        sum += (uint32_t)v[i] & kValueMask;
+                    } else {
+                        raise_error(err, UE_ERR_TIMEOUT, gfirst + i);
+                        flag = kFlagError;
+                    }
+                }
+            }
+            st_relaxed(sc.gstatus + (size_t)grp * E + tid, status_word(tag, flag, sum));
         }
+        // every member has arrived: ready for the next launch
+        if (tid == 0) sc.gcount[grp] = 0u;
     }
 
-    // ---- copy table of every expert, from the plan (overlaps the wait) ----
-    for (int p = tid; p <= P; p += kThreads) u.pro.off[p] = __ldg(plan.slot_offset + p);
-    for (int p = tid; p < P; p += kThreads) u.pro.sq[p] = __ldg(plan.slot_quota + p);
-    for (int g = tid; g < G; g += kThreads) u.pro.se[g] = __ldg(plan.slot_expert + g);
-    __syncthreads();
+    // ---- copy table of every expert, from the plan ----
     for (int g = tid; g < G; g += kThreads) {
         const int e = u.pro.se[g];
         if (e >= 0 && e < E) {
@@ -268,6 +322,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         }
     }
     __syncthreads();
+    int nent;  // copy-table entries: every expert's master and replicas
     {
         // exclusive scan of copies per expert (1 + replicas) over experts
         const int c = tid < E ? 1 + u.pro.cnt[tid] : 0;
@@ -279,8 +334,12 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         }
         if (lane == 31) s_wsum[warp] = incl;
         __syncthreads();
-        int wofs = 0;
-        for (int w = 0; w < warp; ++w) wofs += s_wsum[w];
+        int wofs = 0, all = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            wofs += w < warp ? s_wsum[w] : 0;
+            all += s_wsum[w];
+        }
+        nent = all;
         if (tid < E) {
             const int e = tid;
             const int mp = (e / M) * (M + S) + (e % M);
@@ -288,6 +347,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
             s_c[e] = ExpC{c, cb};          // completed below
             s_cp[cb] = mp;                 // copy 0: the master
             s_cr[cb] = u.pro.off[mp];
+            s_ce[cb] = (short)e;
             u.pro.run[e] = cb + 1;         // next replica entry
         }
         __syncthreads();
@@ -307,6 +367,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
                 const int p = (g / S) * (M + S) + M + (g % S);
                 s_cp[ci] = p;
                 s_cr[ci] = u.pro.off[p];
+                s_ce[ci] = (short)e;
             }
             __syncwarp();
             if (e >= 0 && lane == __ffs(peers) - 1) u.pro.run[e] += __popc(peers);
@@ -314,110 +375,109 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         }
     }
     __syncthreads();
-    if (tid < E) {
-        // the expert's load, its copies' starts, and whether the quotas have
-        // the floor form b + [j < rem]
-        const int e = tid;
-        const ExpC c0 = s_c[e];
-        const int c = c0.b, cb = c0.cb;
-        int L = 0;
-        for (int j = 0; j < c; ++j) {
-            s_cs[cb + j] = L;
-            L += u.pro.sq[s_cp[cb + j]];
+    {
+        // every copy's start: an exclusive scan of the quotas over the
+        // entries (experts in order, each one's copies in copy order)
+        const int q = tid < nent ? u.pro.sq[s_cp[tid]] : 0;
+        int incl = q;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off) incl += o;
         }
-        const unsigned b = (unsigned)L / (unsigned)c;
-        const int rem = L - (int)b * c;
-        bool floor_form = kOrder != kOrderLocal;  // the local order needs the count
-        for (int j = 0; j < c; ++j)
-            floor_form &= u.pro.sq[s_cp[cb + j]] == (int)b + (j < rem ? 1 : 0);
-        s_a[e] = ExpA{0, L, rem * (int)(b + 1u), floor_form ? rem : -1};
-        s_bm[e] = ExpB{recip64(b + 1u), recip64(b)};
-        s_c[e] = ExpC{floor_form ? (int)b : c, cb};
+        if (lane == 31) s_wsum[warp] = incl;
+        __syncthreads();
+        int wofs = 0;
+        for (int w = 0; w < warp; ++w) wofs += s_wsum[w];
+        if (tid < nent) s_cs[tid] = wofs + incl - q;
+        if (tid == nent - 1) s_cs[nent] = wofs + incl;
+        __syncthreads();
+    }
+    if (tid < E) {
+        // the expert's load and its floor-form parameters b = floor(L/c), rem
+        const ExpC c0 = s_c[tid];
+        const int base = s_cs[c0.cb];
+        const int L = s_cs[c0.cb + c0.b] - base;
+        const unsigned b = (unsigned)L / (unsigned)c0.b;
+        u.pro.base[tid] = base;
+        s_a[tid] = ExpA{0, L, (L - (int)b * c0.b) * (int)(b + 1u), L - (int)b * c0.b};
+    }
+    __syncthreads();
+    if (tid < nent) {
+        // starts relative to the expert; quotas of the form b + [j < rem]?
+        const int e = s_ce[tid];
+        const ExpC c0 = s_c[e];
+        const int j = tid - c0.cb;
+        const int q = u.pro.sq[s_cp[tid]];
+        const unsigned b = (unsigned)s_a[e].L / (unsigned)c0.b;
+        if (kOrder == kOrderLocal || q != (int)b + (j < s_a[e].rem ? 1 : 0)) u.pro.ff[e] = 0;
+        s_cs[tid] -= u.pro.base[e];
+    }
+    __syncthreads();
+    if (tid < E) {
+        // the local order needs the number of copies, so it never takes the
+        // floor form
+        const ExpC c0 = s_c[tid];
+        const ExpA a = s_a[tid];
+        const bool floor_form = u.pro.ff[tid] != 0;
+        const unsigned b = (unsigned)a.L / (unsigned)c0.b;
+        s_a[tid] = ExpA{0, a.L, a.thr, floor_form ? a.rem : -1};
+        s_bm[tid] = ExpB{recip64(b + 1u), recip64(b)};
+        s_c[tid] = ExpC{floor_form ? (int)b : c0.b, c0.cb};
     }
     __syncthreads();  // the union switches from the copy table to look-back
 
-    // ---- look back over predecessor tiles, publish the inclusive prefix ----
-    // H threads per expert column; thread (h, e) reads predecessors
-    // base - h*W .. base - h*W - (W-1) of each step, so one step covers H*W
-    // tiles with independent loads.
+    // ---- look back: this tile's exclusive prefix per expert ----
+    // the group sums of the groups before this tile's group, plus the counts
+    // of the tiles before it in its group. H threads per expert column, each
+    // summing every H-th item, kWindow independent loads at a time.
     const int H = min(kMaxH, kThreads / E);
     const int h = tid / E;
     const int e = tid - h * E;
-    const bool lb = h < H;
-    uint32_t excl = 0;
-    if (lb && h == 0) u.lb.cdone[e] = (tile == 0) ? 1 : 0;
-    __syncthreads();
-    bool done = lb ? (u.lb.cdone[e] != 0) : true;
-    int base = tile - 1;  // nearest predecessor not yet added
-    int64_t polls = 0;
-    while (__syncthreads_or(!done)) {
-        if (!done) {
-            uint32_t sum = 0;
-            unsigned char st = 0;  // 0: no prefix in my segment, 1: prefix, 2: error
+    const int n_items = grp + (tile - gfirst);
+    if (h < H) {
+        uint32_t part = 0;
+        unsigned char st = 0;  // 0: fine, 2: error
+        int64_t polls = 0;
+        // item it: group sum `it` (it < grp), else the count of tile
+        // gfirst + it - grp
+        auto item = [&](int it) {
+            return it < grp ? sc.gstatus + (size_t)it * E + e
+                            : sc.status + (size_t)(gfirst + it - grp) * E + e;
+        };
+        for (int i0 = h; i0 < n_items && st == 0; i0 += H * kWindow) {
             unsigned long long v[kWindow];
 #pragma unroll
             for (int i = 0; i < kWindow; ++i) {
-                const int pred = base - h * kWindow - i;
-                v[i] = pred >= 0 ? ld_relaxed(status + (size_t)pred * E + e)
-                                 : status_word(tag, kFlagPrefix, 0u);
+                const int it = i0 + i * H;
+                v[i] = it < n_items ? ld_relaxed(item(it)) : 0ull;
             }
 #pragma unroll
             for (int i = 0; i < kWindow; ++i) {
-                if (st == 0) {
-                    const int pred = base - h * kWindow - i;
-                    unsigned long long sw = v[i];
-                    // not yet published in this launch (older tag or none)
-                    while (((uint32_t)(sw >> 32) != tag ||
-                            (((uint32_t)sw >> 30) == kFlagInvalid)) && st == 0) {
-                        if (++polls > spin_limit) {
-                            raise_error(err, UE_ERR_TIMEOUT, tile);
-                            st = 2;
-                        } else {
-                            __nanosleep(64);
-                            sw = ld_relaxed(status + (size_t)pred * E + e);
-                        }
-                    }
-                    if (st == 0) {
-                        const uint32_t flag = (uint32_t)sw >> 30;
-                        if (flag == kFlagError) {
-                            st = 2;
-                        } else {
-                            if (pred >= 0) sum += (uint32_t)sw & kValueMask;
-                            if (flag == kFlagPrefix) st = 1;
-                        }
+                if (i0 + i * H < n_items && st == 0) {
+                    if (!wait_word(item(i0 + i * H), tag, v[i], polls, spin_limit)) {
+                        raise_error(err, UE_ERR_TIMEOUT, tile);
+                        st = 2;
+                    } else if (((uint32_t)v[i] >> 30) == kFlagError) {
+                        st = 2;
+                    } else {
+                        part += (uint32_t)v[i] & kValueMask;
                     }
                 }
             }
-            u.lb.part[h][e] = sum;
-            u.lb.state[h][e] = st;
         }
-        __syncthreads();
-        if (!done && h == 0) {
-            // add the segments in order up to the first one holding a prefix
-            bool stop = false;
-            for (int hh = 0; hh < H && !stop; ++hh) {
-                const unsigned char st = u.lb.state[hh][e];
-                if (st == 2) {
-                    atomicOr(&s_fail, 1);
-                    stop = true;
-                } else {
-                    excl += u.lb.part[hh][e];
-                    if (st == 1) stop = true;
-                }
-            }
-            u.lb.cdone[e] = stop ? 1 : 0;
+        u.lb.part[h][e] = part;
+        u.lb.state[h][e] = st;
+    }
+    __syncthreads();
+    if (tid < E) {
+        uint32_t excl = 0;
+        for (int hh = 0; hh < H; ++hh) {
+            if (u.lb.state[hh][tid] != 0) s_fail = 1;
+            excl += u.lb.part[hh][tid];
         }
-        __syncthreads();
-        if (!done) done = u.lb.cdone[e] != 0;
-        base -= H * kWindow;
+        s_a[tid].pre = (int)excl;
     }
-    if (tid < E && tile > 0) {
-        if (s_fail)
-            st_relaxed(mine, status_word(tag, kFlagError, 0u));
-        else
-            st_relaxed(mine, status_word(tag, kFlagPrefix, excl + (uint32_t)acc));
-    }
-    if (tid < E) s_a[tid].pre = (int)excl;
     __syncthreads();
     const bool write_out = !s_fail;
 
@@ -426,8 +486,8 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     // while o < rem*(b+1), else rem + (o - rem*(b+1)) / b; otherwise the
     // last copy whose start is <= o. Row = first row of the copy + (o - start).
 #pragma unroll 2
-    for (int rd = 0; rd < (write_out ? kRounds : 0); ++rd) {
-        const int x = warp * kPerWarp + rd * 32 + lane;
+    for (int rd = 0; rd < (write_out ? kPer : 0); ++rd) {
+        const int x = warp * kPerWarpP + rd * 32 + lane;
         const int ex = s_idx[x];
         const unsigned peers = same_key_lanes(ex & 511);
         const int64_t i = pair_at<kOrder>(t0 + x, ord);
@@ -485,11 +545,11 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     __syncthreads();
     if (tid == 0) {
         __threadfence();
-        if (atomicAdd(&sync[1], 1u) == gridDim.x - 1) {
-            sync[0] = 0u;
-            sync[1] = 0u;
+        if (atomicAdd(&sc.sync[1], 1u) == gridDim.x - 1) {
+            sc.sync[0] = 0u;
+            sc.sync[1] = 0u;
             __threadfence();
-            atomicExch(&sync[2], tag);
+            atomicExch(&sc.sync[2], tag);
         }
     }
 }
@@ -564,50 +624,115 @@ OrderArgs make_order(const Sizes& z)
     return o;
 }
 
-template <int kOrder>
-cudaError_t launch_order(const Sizes& z, const int32_t* idx, const ue_placement& plan,
+template <int kOrder, int kPer>
+cudaError_t launch_tiles(const Sizes& z, const int32_t* idx, const ue_placement& plan,
                          const OrderArgs& ord, int32_t* phys_slot, int32_t* dest_row,
-                         unsigned long long* status, uint32_t* sync, int64_t spin_limit,
-                         int drop_first, int* err, cudaStream_t st)
+                         const RerouteScratch& sc, int64_t spin_limit, int drop_first, int* err,
+                         cudaStream_t st)
 {
-    const int64_t tiles = (z.Q + kTile - 1) / kTile;
-    reroute_kernel<kOrder><<<(unsigned)tiles, kThreads, 0, st>>>(
-        idx, z.Q, z.R, z.E, z.S, plan, ord, phys_slot, dest_row, status, sync, spin_limit,
-        drop_first, err);
+    const int64_t tiles = (z.Q + kThreads * kPer - 1) / (kThreads * kPer);
+    reroute_kernel<kOrder, kPer><<<(unsigned)tiles, kThreads, kThreads * kPer * sizeof(short), st>>>(
+        idx, z.Q, z.R, z.E, z.S, plan, ord, phys_slot, dest_row, sc, spin_limit, drop_first,
+        err);
     return cudaGetLastError();
+}
+
+template <int kOrder>
+cudaError_t launch_order(const Sizes& z, int tile, const int32_t* idx, const ue_placement& plan,
+                         const OrderArgs& ord, int32_t* phys_slot, int32_t* dest_row,
+                         const RerouteScratch& sc, int64_t spin_limit, int drop_first, int* err,
+                         cudaStream_t st)
+{
+    switch (tile) {
+    case kThreads * 16:
+        return launch_tiles<kOrder, 16>(z, idx, plan, ord, phys_slot, dest_row, sc, spin_limit,
+                                        drop_first, err, st);
+    case kThreads * 24:
+        return launch_tiles<kOrder, 24>(z, idx, plan, ord, phys_slot, dest_row, sc, spin_limit,
+                                        drop_first, err, st);
+    case kThreads * 32:
+        return launch_tiles<kOrder, 32>(z, idx, plan, ord, phys_slot, dest_row, sc, spin_limit,
+                                        drop_first, err, st);
+    default:
+        return cudaErrorInvalidValue;
+    }
+}
+
+template <int kPer>
+cudaError_t allow_smem()
+{
+    const int bytes = kThreads * kPer * (int)sizeof(short);
+    cudaError_t ce = cudaFuncSetAttribute(reroute_kernel<kOrderPrefix, kPer>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (ce == cudaSuccess)
+        ce = cudaFuncSetAttribute(reroute_kernel<kOrderInterleave, kPer>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (ce == cudaSuccess)
+        ce = cudaFuncSetAttribute(reroute_kernel<kOrderLocal, kPer>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    return ce;
+}
+
+template <int kPer>
+int64_t tile_slots(int num_sms)
+{
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reroute_kernel<kOrderPrefix, kPer>,
+                                                      kThreads, kThreads * kPer * sizeof(short)) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        per_sm = 1;
+    }
+    return (int64_t)std::max(per_sm, 1) * num_sms;
 }
 
 }  // namespace
 
-cudaError_t launch_reroute(const Sizes& z, const int32_t* idx,
-                           const ue_placement& plan, int32_t* phys_slot,
-                           int32_t* dest_row, unsigned long long* status,
-                           uint32_t* sync, int64_t spin_limit,
-                           int drop_first, int* err, cudaStream_t st)
+cudaError_t reroute_setup()
 {
-    return launch_reroute_order(z, idx, plan, kOrderPrefix, phys_slot, dest_row, status, sync,
+    cudaError_t ce = allow_smem<16>();
+    if (ce == cudaSuccess) ce = allow_smem<24>();
+    if (ce == cudaSuccess) ce = allow_smem<32>();
+    return ce;
+}
+
+int reroute_tile(const Sizes& z, int num_sms)
+{
+    // the smallest tile whose tiles are all resident at once (one wave), so
+    // that no tile waits for a CTA slot; 32 pairs per thread otherwise
+    if ((z.Q + kThreads * 16 - 1) / (kThreads * 16) <= tile_slots<16>(num_sms)) return kThreads * 16;
+    if ((z.Q + kThreads * 24 - 1) / (kThreads * 24) <= tile_slots<24>(num_sms)) return kThreads * 24;
+    return kThreads * 32;
+}
+
+cudaError_t launch_reroute(const Sizes& z, int tile, const int32_t* idx,
+                           const ue_placement& plan, int32_t* phys_slot, int32_t* dest_row,
+                           const RerouteScratch& sc, int64_t spin_limit, int drop_first, int* err,
+                           cudaStream_t st)
+{
+    return launch_reroute_order(z, tile, idx, plan, kOrderPrefix, phys_slot, dest_row, sc,
                                 spin_limit, drop_first, err, st);
 }
 
-cudaError_t launch_reroute_order(const Sizes& z, const int32_t* idx, const ue_placement& plan,
-                                 int order, int32_t* phys_slot, int32_t* dest_row,
-                                 unsigned long long* status, uint32_t* sync, int64_t spin_limit,
+cudaError_t launch_reroute_order(const Sizes& z, int tile, const int32_t* idx,
+                                 const ue_placement& plan, int order, int32_t* phys_slot,
+                                 int32_t* dest_row, const RerouteScratch& sc, int64_t spin_limit,
                                  int drop_first, int* err, cudaStream_t st)
 {
     if (z.Q == 0) return cudaSuccess;
     const OrderArgs ord = make_order(z);
     if (order == kOrderInterleave)
-        return launch_order<kOrderInterleave>(z, idx, plan, ord, phys_slot, dest_row, status,
-                                              sync, spin_limit, drop_first, err, st);
-    return launch_order<kOrderPrefix>(z, idx, plan, ord, phys_slot, dest_row, status, sync,
+        return launch_order<kOrderInterleave>(z, tile, idx, plan, ord, phys_slot, dest_row, sc,
+                                              spin_limit, drop_first, err, st);
+    return launch_order<kOrderPrefix>(z, tile, idx, plan, ord, phys_slot, dest_row, sc,
                                       spin_limit, drop_first, err, st);
 }
 
-cudaError_t launch_reroute_local(const Sizes& z, const int32_t* idx, const int32_t* load_re,
-                                 const ue_placement& plan, const int32_t* src_quota,
-                                 const int32_t* src_offset, int32_t* first, int32_t* rowb,
-                                 int32_t* phys_slot, int32_t* dest_row,
-                                 unsigned long long* status, uint32_t* sync, int64_t spin_limit,
+cudaError_t launch_reroute_local(const Sizes& z, int tile, const int32_t* idx,
+                                 const int32_t* load_re, const ue_placement& plan,
+                                 const int32_t* src_quota, const int32_t* src_offset,
+                                 int32_t* first, int32_t* rowb, int32_t* phys_slot,
+                                 int32_t* dest_row, const RerouteScratch& sc, int64_t spin_limit,
                                  int drop_first, int* err, cudaStream_t st)
 {
     if (z.Q == 0) return cudaSuccess;
@@ -619,7 +744,7 @@ cudaError_t launch_reroute_local(const Sizes& z, const int32_t* idx, const int32
     ord.first = first;
     ord.rowb = rowb;
     ord.quota = src_quota;
-    return launch_order<kOrderLocal>(z, idx, plan, ord, phys_slot, dest_row, status, sync,
+    return launch_order<kOrderLocal>(z, tile, idx, plan, ord, phys_slot, dest_row, sc,
                                      spin_limit, drop_first, err, st);
 }
 

@@ -17,14 +17,17 @@ struct ue_ctx {
     ue::CombineShape comb;
     ue::BwdShape bwd;       // combine backward launch shape
     int* d_err;             // [2] error code, detail
-    unsigned long long* d_status;  // [tiles][E] reroute look-back words
+    unsigned long long* d_status;  // [tiles][E] reroute tile counts
+    unsigned long long* d_gstatus; // [groups][E] reroute group sums
+    uint32_t* d_gcount;     // [groups] reroute group arrivals
     uint32_t* d_sync;       // [4] reroute ticket, finished CTAs, epoch
     uint32_t* d_gsync;      // [4] fused gate count: ticket, finished CTAs, epoch, flag
     int32_t* d_first;       // [R][P] locality order: first occurrence index
     int32_t* d_rowb;        // [R][P] locality order: row base
     uint16_t* d_zrow;       // [d] zeros: the combine reads it for a row out of range
     int32_t* d_grtab;       // [kGrTableWords] gradient reduction: replicated experts, their slots
-    int64_t tiles;
+    int rtile;              // reroute pairs per tile
+    int64_t tiles, groups;
     int64_t spin_limit;
     int drop_first;
     uint32_t magic;
@@ -51,12 +54,32 @@ ue_status use_device(const ue_ctx* ctx)
 
 ue_status from_cuda(cudaError_t e) { return e == cudaSuccess ? UE_OK : UE_ERR_CUDA; }
 
+ue::RerouteScratch rscratch(const ue_ctx* ctx)
+{
+    return ue::RerouteScratch{ctx->d_status, ctx->d_gstatus, ctx->d_gcount, ctx->d_sync};
+}
+
 bool placement_ok(const ue_ctx* ctx, const ue_placement* p)
 {
     if (p == nullptr) return false;
     if (ctx->z.G > 0 && !aligned(p->slot_expert, 4)) return false;
     return aligned(p->n_copies, 4) && aligned(p->slot_quota, 4) && aligned(p->slot_offset, 4) &&
            aligned(p->rank_load, 4) && aligned(p->stats, 4);
+}
+
+// free every device buffer of a context (null ones are skipped)
+void free_buffers(ue_ctx* ctx)
+{
+    cudaFree(ctx->d_err);
+    cudaFree(ctx->d_status);
+    cudaFree(ctx->d_gstatus);
+    cudaFree(ctx->d_gcount);
+    cudaFree(ctx->d_sync);
+    cudaFree(ctx->d_gsync);
+    cudaFree(ctx->d_first);
+    cudaFree(ctx->d_rowb);
+    cudaFree(ctx->d_zrow);
+    cudaFree(ctx->d_grtab);
 }
 
 }  // namespace
@@ -83,7 +106,14 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
     ctx->device = device;
     ctx->num_sms = prop.multiProcessorCount;
     ctx->gate = ue::plan_gate_shape(ctx->z, ctx->num_sms);
-    ctx->tiles = (ctx->z.Q + ue::kRerouteTile - 1) / ue::kRerouteTile;
+    if (ue::reroute_setup() != cudaSuccess) {
+        delete ctx;
+        cudaGetLastError();
+        return UE_ERR_CUDA;
+    }
+    ctx->rtile = ue::reroute_tile(ctx->z, ctx->num_sms);
+    ctx->tiles = ue::reroute_tiles(ctx->z, ctx->rtile);
+    ctx->groups = ue::reroute_groups(ctx->z, ctx->rtile);
     ctx->spin_limit = 1LL << 22;
     ctx->drop_first = 0;
 
@@ -97,41 +127,33 @@ ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out)
     }
 
     const size_t status_words = (size_t)std::max<int64_t>(ctx->tiles, 1) * ctx->z.E;
+    const size_t group_words = (size_t)std::max<int64_t>(ctx->groups, 1) * ctx->z.E;
+    const size_t groups = (size_t)std::max<int64_t>(ctx->groups, 1);
     const size_t table_words = (size_t)ctx->z.R * ctx->z.P;
     if (cudaMalloc(&ctx->d_err, 2 * sizeof(int)) != cudaSuccess ||
         cudaMalloc(&ctx->d_status, status_words * sizeof(unsigned long long)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_gstatus, group_words * sizeof(unsigned long long)) != cudaSuccess ||
+        cudaMalloc(&ctx->d_gcount, groups * sizeof(uint32_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_sync, 4 * sizeof(uint32_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_gsync, 4 * sizeof(uint32_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_first, table_words * sizeof(int32_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_rowb, table_words * sizeof(int32_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_zrow, (size_t)ctx->z.d * sizeof(uint16_t)) != cudaSuccess ||
         cudaMalloc(&ctx->d_grtab, ue::kGrTableWords * sizeof(int32_t)) != cudaSuccess) {
-        cudaFree(ctx->d_err);
-        cudaFree(ctx->d_status);
-        cudaFree(ctx->d_sync);
-        cudaFree(ctx->d_gsync);
-        cudaFree(ctx->d_first);
-        cudaFree(ctx->d_rowb);
-        cudaFree(ctx->d_zrow);
-        cudaFree(ctx->d_grtab);
+        free_buffers(ctx);
         delete ctx;
         cudaGetLastError();
         return UE_ERR_NOMEM;
     }
     if (cudaMemset(ctx->d_err, 0, 2 * sizeof(int)) != cudaSuccess ||
         cudaMemset(ctx->d_status, 0, status_words * sizeof(unsigned long long)) != cudaSuccess ||
+        cudaMemset(ctx->d_gstatus, 0, group_words * sizeof(unsigned long long)) != cudaSuccess ||
+        cudaMemset(ctx->d_gcount, 0, groups * sizeof(uint32_t)) != cudaSuccess ||
         cudaMemset(ctx->d_sync, 0, 4 * sizeof(uint32_t)) != cudaSuccess ||
         cudaMemset(ctx->d_gsync, 0, 4 * sizeof(uint32_t)) != cudaSuccess ||
         cudaMemset(ctx->d_zrow, 0, (size_t)ctx->z.d * sizeof(uint16_t)) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess) {
-        cudaFree(ctx->d_err);
-        cudaFree(ctx->d_status);
-        cudaFree(ctx->d_sync);
-        cudaFree(ctx->d_gsync);
-        cudaFree(ctx->d_first);
-        cudaFree(ctx->d_rowb);
-        cudaFree(ctx->d_zrow);
-        cudaFree(ctx->d_grtab);
+        free_buffers(ctx);
         delete ctx;
         return UE_ERR_CUDA;
     }
@@ -146,14 +168,7 @@ ue_status ue_destroy(ue_ctx* ctx)
     if (!ctx_ok(ctx)) return UE_ERR_INVALID_ARG;
     ue_status st = use_device(ctx);
     if (st == UE_OK && cudaDeviceSynchronize() != cudaSuccess) st = UE_ERR_CUDA;
-    cudaFree(ctx->d_err);
-    cudaFree(ctx->d_status);
-    cudaFree(ctx->d_sync);
-    cudaFree(ctx->d_gsync);
-    cudaFree(ctx->d_first);
-    cudaFree(ctx->d_rowb);
-    cudaFree(ctx->d_zrow);
-    cudaFree(ctx->d_grtab);
+    free_buffers(ctx);
     ctx->magic = 0;
     delete ctx;
     return st;
@@ -240,8 +255,8 @@ ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
         !aligned(phys_slot, 4) || !aligned(dest_row, 4))
         return UE_ERR_INVALID_ARG;
     if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
-    return from_cuda(ue::launch_reroute(ctx->z, idx, *plan, phys_slot, dest_row, ctx->d_status,
-                                        ctx->d_sync, ctx->spin_limit, ctx->drop_first,
+    return from_cuda(ue::launch_reroute(ctx->z, ctx->rtile, idx, *plan, phys_slot, dest_row,
+                                        rscratch(ctx), ctx->spin_limit, ctx->drop_first,
                                         ctx->d_err, as_stream(stream)));
 }
 
@@ -253,8 +268,8 @@ ue_status ue_reroute_ex(ue_ctx* ctx, const int32_t* idx, const ue_placement* pla
         (order != UE_ORDER_PREFIX && order != UE_ORDER_INTERLEAVE))
         return UE_ERR_INVALID_ARG;
     if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
-    return from_cuda(ue::launch_reroute_order(ctx->z, idx, *plan, order, phys_slot, dest_row,
-                                              ctx->d_status, ctx->d_sync, ctx->spin_limit,
+    return from_cuda(ue::launch_reroute_order(ctx->z, ctx->rtile, idx, *plan, order, phys_slot,
+                                              dest_row, rscratch(ctx), ctx->spin_limit,
                                               ctx->drop_first, ctx->d_err, as_stream(stream)));
 }
 
@@ -279,9 +294,9 @@ ue_status ue_reroute_local(ue_ctx* ctx, const int32_t* idx, const int32_t* load_
         !aligned(dest_row, 4))
         return UE_ERR_INVALID_ARG;
     if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
-    return from_cuda(ue::launch_reroute_local(ctx->z, idx, load_re, *plan, src_quota, src_offset,
-                                              ctx->d_first, ctx->d_rowb, phys_slot, dest_row,
-                                              ctx->d_status, ctx->d_sync, ctx->spin_limit,
+    return from_cuda(ue::launch_reroute_local(ctx->z, ctx->rtile, idx, load_re, *plan, src_quota,
+                                              src_offset, ctx->d_first, ctx->d_rowb, phys_slot,
+                                              dest_row, rscratch(ctx), ctx->spin_limit,
                                               ctx->drop_first, ctx->d_err, as_stream(stream)));
 }
 

@@ -23,10 +23,14 @@ __device__ __forceinline__ void raise_error(int* err, int code, int detail)
 constexpr int kWarp = 32;
 constexpr unsigned kFull = 0xffffffffu;
 
-// Reroute tiling: pairs per tile and threads per tile.
-constexpr int kRerouteTile = 8192;
+// Reroute tiling: threads per tile; a tile holds 16, 24 or 32 pairs per
+// thread (kRerouteTile: the 16-pair default), chosen per context so that
+// every tile is resident at once. The look-back adds the counts of groups of
+// kRerouteGroup tiles.
 constexpr int kRerouteThreads = 512;
 constexpr int kRerouteWarps = kRerouteThreads / kWarp;
+constexpr int kRerouteTile = kRerouteThreads * 16;
+constexpr int kRerouteGroup = 16;
 
 // Look-back status word (64-bit): [63:32] launch tag, [31:30] flag,
 // [29:0] count. A word whose tag is not the current launch's reads as
@@ -113,26 +117,41 @@ cudaError_t plan_bisect_setup(const Sizes& z);
 cudaError_t launch_plan_bisect(const Sizes& z, const int32_t* load_e, int eps_inv, int threshold,
                                int min_tokens, int allow_zero, const ue_placement& out, int* err,
                                cudaStream_t st);
-// Reroute scratch: tiles*E 64-bit status words and sync[0..2] = {tile
-// ticket, finished CTAs, launch epoch}, zeroed once; each launch leaves them
-// ready for the next one (the last CTA resets the ticket and the counter and
-// advances the epoch).
-cudaError_t launch_reroute(const Sizes& z, const int32_t* idx,
-                           const ue_placement& plan, int32_t* phys_slot,
-                           int32_t* dest_row, unsigned long long* status,
-                           uint32_t* sync, int64_t spin_limit,
-                           int drop_first, int* err, cudaStream_t st);
+// Reroute scratch, zeroed once; each launch leaves it ready for the next one
+// (the last CTA resets the ticket and the counter and advances the epoch;
+// each group's last arrival resets its counter).
+struct RerouteScratch {
+    unsigned long long* status;   // [tiles][E] tile counts, tagged with the launch epoch
+    unsigned long long* gstatus;  // [groups][E] group sums, tagged likewise
+    uint32_t* gcount;             // [groups] tiles of the group that have published
+    uint32_t* sync;               // [4] tile ticket, finished CTAs, launch epoch
+};
+inline int64_t reroute_tiles(const Sizes& z, int tile) { return (z.Q + tile - 1) / tile; }
+inline int64_t reroute_groups(const Sizes& z, int tile)
+{
+    return (reroute_tiles(z, tile) + kRerouteGroup - 1) / kRerouteGroup;
+}
+// the reroute kernels' dynamic shared memory limits, set once per device
+// (outside any stream capture) before the first launch
+cudaError_t reroute_setup();
+// pairs per tile for this GPU: the smallest of the three whose tiles fit at
+// once (call after reroute_setup)
+int reroute_tile(const Sizes& z, int num_sms);
+cudaError_t launch_reroute(const Sizes& z, int tile, const int32_t* idx,
+                           const ue_placement& plan, int32_t* phys_slot, int32_t* dest_row,
+                           const RerouteScratch& sc, int64_t spin_limit, int drop_first, int* err,
+                           cudaStream_t st);
 // order: 0 global (r, t, k), 1 interleaved (t, r, k)
-cudaError_t launch_reroute_order(const Sizes& z, const int32_t* idx, const ue_placement& plan,
-                                 int order, int32_t* phys_slot, int32_t* dest_row,
-                                 unsigned long long* status, uint32_t* sync, int64_t spin_limit,
+cudaError_t launch_reroute_order(const Sizes& z, int tile, const int32_t* idx,
+                                 const ue_placement& plan, int order, int32_t* phys_slot,
+                                 int32_t* dest_row, const RerouteScratch& sc, int64_t spin_limit,
                                  int drop_first, int* err, cudaStream_t st);
 // locality order: builds the [R][P] tables `first` and `rowb`, then reroutes
-cudaError_t launch_reroute_local(const Sizes& z, const int32_t* idx, const int32_t* load_re,
-                                 const ue_placement& plan, const int32_t* src_quota,
-                                 const int32_t* src_offset, int32_t* first, int32_t* rowb,
-                                 int32_t* phys_slot, int32_t* dest_row,
-                                 unsigned long long* status, uint32_t* sync, int64_t spin_limit,
+cudaError_t launch_reroute_local(const Sizes& z, int tile, const int32_t* idx,
+                                 const int32_t* load_re, const ue_placement& plan,
+                                 const int32_t* src_quota, const int32_t* src_offset,
+                                 int32_t* first, int32_t* rowb, int32_t* phys_slot,
+                                 int32_t* dest_row, const RerouteScratch& sc, int64_t spin_limit,
                                  int drop_first, int* err, cudaStream_t st);
 cudaError_t launch_locality_split(const Sizes& z, const int32_t* load_re,
                                   const ue_placement& plan, int32_t* src_quota,

@@ -7,12 +7,14 @@
 // outside allocations, in a process whose device memory is reserved up front
 // by another runtime) or code that has no place to keep a context. This entry
 // point needs no context and allocates nothing. Its scratch (the look-back
-// status words, the tile ticket, the finished-CTA counter and the launch
-// epoch) is a file-scope __device__ array of fixed size, which every GPU that
-// loads this library holds until the process exits. The array starts zeroed
-// and is never cleared: status words carry their launch's epoch, so words
-// left by an earlier call read as unpublished, and the last CTA of every
-// call resets the ticket and the counter.
+// status words of the tiles and of the groups of tiles, the groups' arrival
+// counters, the tile ticket, the finished-CTA counter and the launch epoch)
+// is a file-scope __device__ array of fixed size, which every GPU that loads
+// this library holds until the process exits. The array starts zeroed and
+// is never cleared: status words carry their launch's epoch, so words left
+// by an earlier call read as unpublished, each group's last arrival resets
+// its counter, and the last CTA of every call resets the ticket and the
+// counter.
 //
 // The array's name, used in host code, is only a host-side stand-in for the
 // symbol, not a device address. The device address is fetched once per
@@ -27,9 +29,16 @@
 
 namespace {
 
-constexpr size_t kStatusWords = size_t(1) << 18;  // 2 MiB of 64-bit look-back words
-constexpr size_t kSyncWord = kStatusWords;        // ticket, counter, epoch (as 32-bit)
-constexpr size_t kScratchWords = kStatusWords + 16;
+// Layout (64-bit words): tile counts [kStatusWords], group sums
+// [kGroupWords], group arrival counters [kGroupCounters as 32-bit], then the
+// ticket, counter and epoch (as 32-bit).
+constexpr size_t kStatusWords = size_t(1) << 18;  // 2 MiB: tiles * E <= 2^18
+constexpr size_t kGroupWords = (kStatusWords / ue::kRerouteGroup) + ue::kMaxE;  // groups * E
+constexpr size_t kGroupCounters = (kStatusWords / ue::kRerouteGroup) + 64;      // groups
+constexpr size_t kGroupWord = kStatusWords;
+constexpr size_t kCountWord = kGroupWord + kGroupWords;
+constexpr size_t kSyncWord = kCountWord + kGroupCounters / 2;
+constexpr size_t kScratchWords = kSyncWord + 16;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned long long g_reroute_scratch[kScratchWords];
@@ -56,7 +65,8 @@ ue_status scratch_address(int dev, unsigned long long** out)
             return UE_ERR_UNSUPPORTED;
         }
         void* p = nullptr;
-        const cudaError_t ce = cudaGetSymbolAddress(&p, g_reroute_scratch);
+        cudaError_t ce = ue::reroute_setup();
+        if (ce == cudaSuccess) ce = cudaGetSymbolAddress(&p, g_reroute_scratch);
         if (ce != cudaSuccess || p == nullptr) {
             cudaGetLastError();
             return UE_ERR_CUDA;
@@ -95,8 +105,11 @@ extern "C" ue_status ue_reroute_noalloc(const ue_config* cfg, const int32_t* idx
         !aligned4(plan->rank_load) || !aligned4(plan->stats) || !aligned4(idx) ||
         !aligned4(phys_slot) || !aligned4(dest_row) || !aligned4(error))
         return UE_ERR_INVALID_ARG;
-    const int64_t tiles = (z.Q + ue::kRerouteTile - 1) / ue::kRerouteTile;
-    if ((size_t)tiles * (size_t)z.E > kStatusWords) return UE_ERR_UNSUPPORTED;
+    const int64_t tiles = ue::reroute_tiles(z, ue::kRerouteTile);
+    const int64_t groups = ue::reroute_groups(z, ue::kRerouteTile);
+    if ((size_t)tiles * (size_t)z.E > kStatusWords ||
+        (size_t)groups * (size_t)z.E > kGroupWords || (size_t)groups > kGroupCounters)
+        return UE_ERR_UNSUPPORTED;
 
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return UE_ERR_CUDA;
@@ -108,9 +121,12 @@ extern "C" ue_status ue_reroute_noalloc(const ue_config* cfg, const int32_t* idx
         !on_device(error, dev) || !on_device(plan->slot_offset, dev) ||
         !on_device(plan->slot_quota, dev) || (z.G > 0 && !on_device(plan->slot_expert, dev)))
         return UE_ERR_INVALID_ARG;
-    uint32_t* sync = reinterpret_cast<uint32_t*>(base + kSyncWord);
-    const cudaError_t ce = ue::launch_reroute(z, idx, *plan, phys_slot, dest_row, base, sync,
-                                              int64_t(1) << 22, 0, reinterpret_cast<int*>(error),
+    const ue::RerouteScratch sc{base, base + kGroupWord,
+                                reinterpret_cast<uint32_t*>(base + kCountWord),
+                                reinterpret_cast<uint32_t*>(base + kSyncWord)};
+    const cudaError_t ce = ue::launch_reroute(z, ue::kRerouteTile, idx, *plan, phys_slot,
+                                              dest_row, sc, int64_t(1) << 22, 0,
+                                              reinterpret_cast<int*>(error),
                                               reinterpret_cast<cudaStream_t>(stream));
     return ce == cudaSuccess ? UE_OK : UE_ERR_CUDA;
 }
