@@ -204,7 +204,7 @@ __device__ __forceinline__ uint32_t packed_key(float v, uint32_t lo, uint32_t kh
     const uint32_t u = __float_as_uint(__fadd_rn(v, 0.0f));
     const uint32_t sgn = (uint32_t)((int32_t)u >> 31);
     uint32_t x, k;
-    asm("lop3.b32 %0, %1, %2, %3, 0x1e;" : "=r"(x) : "r"(u), "r"(sgn), "r"(0x80000000u));
+    asm("lop3.b32 %0, %1, %2, 0x80000000, 0x1e;" : "=r"(x) : "r"(u), "r"(sgn));
     asm("lop3.b32 %0, %1, %2, %3, 0xea;" : "=r"(k) : "r"(x), "r"(khi), "r"(lo));
     return k;
 }
@@ -295,13 +295,19 @@ __device__ __forceinline__ int fast_expert(int i, int lane)
     return i < 4 * NCH4 ? 128 * (i >> 2) + 4 * lane + (i & 3) : 128 * NCH4 + 32 * (i - 4 * NCH4) + lane;
 }
 
-// The K+1 packed picks of one row into win[0..K]; lane 0 writes them.
+// The K+1 packed picks of one row into win[0..K]; lane 0 writes them. The
+// rounds pop within the first D keys of each lane's sorted list only (three
+// shifts instead of VPL - 1); the keys below are a reserve. That is exact
+// unless a lane gives up all D listed keys and its next key lies above the
+// (K+1)-th pick, which the return value reports (the row is then selected
+// again with full keys).
 template <int NCH4, int NT>
-__device__ __forceinline__ void select_packed(const FastRow<NCH4, NT>& v,
+__device__ __forceinline__ bool select_packed(const FastRow<NCH4, NT>& v,
                                               const uint32_t (&lo)[4 * NCH4 + NT], uint32_t khi,
                                               uint32_t* win, bool writer)
 {
     constexpr int VPL = 4 * NCH4 + NT;
+    constexpr int D = VPL > 3 ? 3 : VPL;
     uint32_t key[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) key[i] = packed_key(v.at(i), lo[i], khi);
@@ -312,11 +318,17 @@ __device__ __forceinline__ void select_packed(const FastRow<NCH4, NT>& v,
         if (writer) win[k] = m;
         const bool pop = key[0] == m;
 #pragma unroll
-        for (int j = 0; j < VPL - 1; ++j) key[j] = pop ? key[j + 1] : key[j];
-        key[VPL - 1] = pop ? 0u : key[VPL - 1];
+        for (int j = 0; j < D - 1; ++j) key[j] = pop ? key[j + 1] : key[j];
+        key[D - 1] = pop ? 0u : key[D - 1];
     }
     const uint32_t m = __reduce_max_sync(kFull, key[0]);
     if (writer) win[kFastK] = m;
+    if constexpr (VPL > D) {
+        // packed keys are never 0, so key[0] == 0 means the list ran dry
+        return __any_sync(kFull, key[0] == 0u && key[D] > m);
+    } else {
+        return false;
+    }
 }
 
 // Exact selection of one row read again from global memory: full keys,
@@ -429,21 +441,24 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_
         FastRow<NCH4, NT> v[kFastRows];
 #pragma unroll
         for (int b = 0; b < kFastRows; ++b) v[b].load(logits + (row0 + b) * (int64_t)E, lane, b < rows);
+        unsigned dry = 0u;  // rows whose reserve keys may belong to the top K+1
         if (rows == kFastRows) {
 #pragma unroll
             for (int b = 0; b < kFastRows; ++b)
-                select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0);
+                if (select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0))
+                    dry |= 0xffu << (b * kFastK);
         } else {
 #pragma unroll
             for (int b = 0; b < kFastRows; ++b)
-                if (b < rows) select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0);
+                if (b < rows && select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0))
+                    dry |= 0xffu << (b * kFastK);
         }
         __syncwarp();
         // rows whose leading picks agree above the dropped bits: exact again
         const bool act = r < rows;
         const uint32_t a = s_win[warp][r][k];
         const uint32_t nx = s_win[warp][r][k + 1];
-        unsigned redo = __ballot_sync(kFull, act && (a >> LOB) == (nx >> LOB));
+        unsigned redo = __ballot_sync(kFull, act && (a >> LOB) == (nx >> LOB)) | dry;
         while (redo) {
             const int rr = (__ffs(redo) - 1) / kFastK;
             select_exact_row<NCH4, NT>(logits + (row0 + rr) * (int64_t)E, lane, s_win[warp][rr]);
@@ -459,13 +474,17 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_
         const double v_own = (double)vf;
         const double v0 = __shfl_sync(kFull, v_own, lead);
         const double x = act ? exp(v_own - v0) : 0.0;
-        double z = 0.0;
-#pragma unroll
-        for (int kk = 0; kk < kFastK; ++kk) z += __shfl_sync(kFull, x, act ? lead + kk : 0);
+        // the row's sum over its eight lanes (an aligned group): every lane
+        // of the group ends with the same value, the pairs being added in
+        // the same (commutative) pairs
+        double z = x;
+        z += __shfl_xor_sync(kFull, z, 1);
+        z += __shfl_xor_sync(kFull, z, 2);
+        z += __shfl_xor_sync(kFull, z, 4);
         if (act) {
             const int64_t pos = row * (int64_t)kFastK + k;
             idx[pos] = (int32_t)e;
-            w[pos] = (float)(x / z);
+            w[pos] = (float)(x * __drcp_rn(z));
             if constexpr (COUNT) {
                 // source rank of the row, relative to the CTA's first rank
                 const int64_t rel = row - rank0 * cnt.T;

@@ -35,21 +35,22 @@
 //    halved (at most 2G + E candidates);
 //  - each candidate is one 64-bit key: floor(L_e 2^17 / c) (exact and order
 //    preserving for c <= 257: two different ratios differ by more than
-//    2^-17), then 255 - e, then c - 1; a bitonic sort in shared memory puts
-//    them in pick order, and each pick's quota parameters follow in
-//    parallel (fewer than G picks end with an end marker).
+//    2^-17), then 255 - e, then c - 1; each key's place in pick order is the
+//    number of larger keys, counted by one thread per key against all the
+//    others, and each pick's quota parameters follow in parallel (fewer
+//    than G picks end with an end marker).
 // Then one warp runs the rank side alone, with the picks already in shared
 // memory: it keeps the rank loads and the redundant slots in registers (lane
 // l owns ranks l, l+32, ... and their slots, so every load change lands in
-// the lane that owns the rank). Per iteration: the stop test and the least
-// loaded rank with a free slot (two `redux` reductions, max load and min of
-// (load << 7 | r), when Q < 2^25; three otherwise), the placement in r*'s
-// lowest free slot, and the new quotas of e*'s copies: the master's goes
-// from ceil(L/(c-1)) to ceil(L/c); a first replica takes floor(L/2); later
-// replicas are found by ballots in ascending slot order. The count of
-// co-located copies does not depend on the order of placement and is taken
-// from the final slots. The rest of the CTA writes the outputs and scans the
-// slot offsets at the end.
+// the lane that owns the rank). Per iteration: the stop test as a vote (is
+// any load above floor(51 Q / (50 R))?) and the least loaded rank with a free
+// slot as one `redux` min of (load << 7 | r) when Q < 2^25 (three reductions
+// otherwise), the placement in r*'s lowest free slot, and the new quotas of
+// e*'s copies: the master's goes from ceil(L/(c-1)) to ceil(L/c); a first
+// replica takes floor(L/2); later replicas are found by ballots in ascending
+// slot order. The count of co-located copies does not depend on the order of
+// placement and is taken from the final slots. The rest of the CTA writes the
+// outputs and scans the slot offsets at the end.
 #include "ue_internal.cuh"
 
 namespace ue {
@@ -102,6 +103,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
     __shared__ int sSlotE[kMaxG];   // expert of redundant slot g, -1 empty (final)
     __shared__ int sSlotQ[kMaxG];   // quota of redundant slot g (final)
     __shared__ unsigned long long sKey[kCandMax];
+    __shared__ unsigned long long sOrd[kMaxG];  // the first G keys in pick order
     __shared__ Pick sPick[kMaxG + 1];  // the picks in order (then an end marker)
     __shared__ long long sRed[kPlanWarps];
     __shared__ int sUsedPicks;
@@ -137,9 +139,8 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
         atomicAdd(&sRank[e / M], L);
         part += (unsigned long long)L;
     }
-    if (part) atomicAdd(&sQ, part);
-    __syncthreads();
-    const unsigned long long Qall = sQ;
+    const unsigned long long Qall = (unsigned long long)block_sum((long long)part, sRed);
+    if (tid == 0) sQ = Qall;
 
     // ---- the pick sequence, in parallel ----
     // candidates per expert at threshold Q/(G+E)/2^lvl (one thread per expert)
@@ -189,48 +190,40 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
     }
     __syncthreads();
     // the keys: position p belongs to the expert whose range holds it
-    int n = 2;
-    while (n < total) n <<= 1;
-    for (int p = tid; p < n; p += blockDim.x) {
-        unsigned long long key = 0ull;
-        if (p < total) {
-            int lo = 0, hi = E - 1;  // last e with sCnt[e] <= p
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (sCnt[mid] <= p) lo = mid;
-                else hi = mid - 1;
-            }
-            const int e = lo;
-            const unsigned c = (unsigned)(p - sCnt[e] + 1);
-            const unsigned long long x = (unsigned long long)sL[e] << kRatioShift;
-            const unsigned long long ratio = c == 1u ? x : __umul64hi(x, sRecip[c]);
-            key = (ratio << 16) | ((unsigned long long)(255 - e) << 8) | (c - 1u);
+    for (int p = tid; p < total; p += blockDim.x) {
+        int lo = 0, hi = E - 1;  // last e with sCnt[e] <= p
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sCnt[mid] <= p) lo = mid;
+            else hi = mid - 1;
         }
-        sKey[p] = key;
+        const int e = lo;
+        const unsigned c = (unsigned)(p - sCnt[e] + 1);
+        const unsigned long long x = (unsigned long long)sL[e] << kRatioShift;
+        const unsigned long long ratio = c == 1u ? x : __umul64hi(x, sRecip[c]);
+        sKey[p] = (ratio << 16) | ((unsigned long long)(255 - e) << 8) | (c - 1u);
     }
     __syncthreads();
-    // bitonic sort, descending
-    for (int k = 2; k <= n; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int q = tid; q < (n >> 1); q += blockDim.x) {
-                const int i = (q / j) * 2 * j + (q % j);
-                const int ij = i + j;
-                const unsigned long long a = sKey[i], b = sKey[ij];
-                const bool desc = (i & k) == 0;
-                if (desc ? (a < b) : (a > b)) {
-                    sKey[i] = b;
-                    sKey[ij] = a;
-                }
-            }
-            __syncthreads();
-        }
+    // pick order: a key's place is the number of larger keys (keys are
+    // distinct), counted against every candidate (broadcast reads); the first
+    // G places are kept
+    for (int p = tid; p < total; p += blockDim.x) {
+        const unsigned long long key = sKey[p];
+        int place = 0;
+        int q = 0;
+        for (; q + 4 <= total; q += 4)
+            place += (sKey[q] > key) + (sKey[q + 1] > key) + (sKey[q + 2] > key) +
+                     (sKey[q + 3] > key);
+        for (; q < total; ++q) place += sKey[q] > key;
+        if (place < G) sOrd[place] = key;
     }
+    __syncthreads();
     const int npicks = min(G, total);
     for (int t = tid; t <= npicks && t < G + 1; t += blockDim.x) {
         if (t == npicks) {
             sPick[t] = Pick{-1, 0u, 0u, 0u, 0u, 0};
         } else {
-            const unsigned long long key = sKey[t];
+            const unsigned long long key = sOrd[t];
             const int e = 255 - (int)((key >> 8) & 255ull);
             const unsigned c = (unsigned)(key & 255ull) + 1u;  // copies before the pick
             const unsigned ce = c + 1u;
@@ -308,48 +301,31 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
 
             if (pk.e < 0) break;  // no expert may take another copy
             const int estar = pk.e;
-            const int rj = rstar >> 5;
+            const int rj = rstar >> 5;  // warp-uniform, as are rm and first
             const bool rown = lane == (rstar & 31);
-
-            // the new copy goes into r*'s lowest free slot (the slot index is
-            // made warp-uniform so that the slot arrays stay in registers)
-            int s_new = 0;
-#pragma unroll
-            for (int j = 0; j < NJR; ++j)
-                if (j == rj) s_new = used[j];
-            s_new = __shfl_sync(kFull, s_new, rstar & 31);
-            if (rown) {
-#pragma unroll
-                for (int j = 0; j < NJR; ++j)
-                    if (j == rj) {
-                        used[j] += 1;
-#pragma unroll
-                        for (int s = 0; s < SM; ++s)
-                            if (s == s_new) slotE[j][s] = estar;
-                    }
-            }
-            // master quota change, on the master rank's owner
             const int rm = pk.rm;
-            if (lane == (rm & 31)) {
+            const bool mown = lane == (rm & 31);
+            const bool first = pk.c == 2u;
+            // without branches on the lane: the new copy goes into r*'s lowest
+            // free slot; a first replica takes floor(L/2) (L mod 2 < 2 keeps
+            // the +1 on the master, the only other copy); the master's quota
+            // change lands on its rank's owner
 #pragma unroll
-                for (int j = 0; j < NJR; ++j)
-                    if (j == (rm >> 5)) load[j] += pk.dq0;
-            }
-            if (pk.c == 2u) {
-                // first replica: the only other copy is the master, and the
-                // replica's quota is floor(L/2) (L mod 2 < 2 keeps the +1 on
-                // the master)
-                if (rown) {
+            for (int j = 0; j < NJR; ++j) {
+                const bool own = rown && j == rj;
+                const int sn = used[j];
 #pragma unroll
-                    for (int j = 0; j < NJR; ++j)
-                        if (j == rj) {
-#pragma unroll
-                            for (int s = 0; s < SM; ++s)
-                                if (s < S && slotE[j][s] == estar) slotQ[j][s] = (int)pk.qb;
-                            load[j] += pk.qb;
-                        }
+                for (int s = 0; s < SM; ++s) {
+                    const bool here = own && s == sn;
+                    slotE[j][s] = here ? estar : slotE[j][s];
+                    slotQ[j][s] = (here && first) ? (int)pk.qb : slotQ[j][s];
                 }
-            } else {
+                used[j] += own ? 1 : 0;
+                unsigned add = (own && first) ? pk.qb : 0u;
+                add += (mown && j == (rm >> 5)) ? pk.dq0 : 0u;
+                load[j] += add;
+            }
+            if (!first) {
                 // replicas, ascending slot g = r*S + s (r = lane + 32 j)
                 unsigned before = 0u;
                 const unsigned lt = (1u << lane) - 1u;

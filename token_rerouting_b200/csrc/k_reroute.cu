@@ -637,6 +637,9 @@ cudaError_t launch_tiles(const Sizes& z, const int32_t* idx, const ue_placement&
     return cudaGetLastError();
 }
 
+// pairs per thread of the tile sizes on offer (tile = 512 * kPer)
+#define UE_REROUTE_PER(X) X(8) X(10) X(12) X(14) X(16) X(20) X(24) X(28) X(32)
+
 template <int kOrder>
 cudaError_t launch_order(const Sizes& z, int tile, const int32_t* idx, const ue_placement& plan,
                          const OrderArgs& ord, int32_t* phys_slot, int32_t* dest_row,
@@ -644,15 +647,12 @@ cudaError_t launch_order(const Sizes& z, int tile, const int32_t* idx, const ue_
                          cudaStream_t st)
 {
     switch (tile) {
-    case kThreads * 16:
-        return launch_tiles<kOrder, 16>(z, idx, plan, ord, phys_slot, dest_row, sc, spin_limit,
-                                        drop_first, err, st);
-    case kThreads * 24:
-        return launch_tiles<kOrder, 24>(z, idx, plan, ord, phys_slot, dest_row, sc, spin_limit,
-                                        drop_first, err, st);
-    case kThreads * 32:
-        return launch_tiles<kOrder, 32>(z, idx, plan, ord, phys_slot, dest_row, sc, spin_limit,
-                                        drop_first, err, st);
+#define UE_CASE(P)                                                                          \
+    case kThreads * P:                                                                      \
+        return launch_tiles<kOrder, P>(z, idx, plan, ord, phys_slot, dest_row, sc,          \
+                                       spin_limit, drop_first, err, st);
+        UE_REROUTE_PER(UE_CASE)
+#undef UE_CASE
     default:
         return cudaErrorInvalidValue;
     }
@@ -690,18 +690,22 @@ int64_t tile_slots(int num_sms)
 
 cudaError_t reroute_setup()
 {
-    cudaError_t ce = allow_smem<16>();
-    if (ce == cudaSuccess) ce = allow_smem<24>();
-    if (ce == cudaSuccess) ce = allow_smem<32>();
+    cudaError_t ce = cudaSuccess;
+#define UE_ALLOW(P) if (ce == cudaSuccess) ce = allow_smem<P>();
+    UE_REROUTE_PER(UE_ALLOW)
+#undef UE_ALLOW
     return ce;
 }
 
 int reroute_tile(const Sizes& z, int num_sms)
 {
-    // the smallest tile whose tiles are all resident at once (one wave), so
-    // that no tile waits for a CTA slot; 32 pairs per thread otherwise
-    if ((z.Q + kThreads * 16 - 1) / (kThreads * 16) <= tile_slots<16>(num_sms)) return kThreads * 16;
-    if ((z.Q + kThreads * 24 - 1) / (kThreads * 24) <= tile_slots<24>(num_sms)) return kThreads * 24;
+    // the most tiles that are all resident at once (one wave, about the same
+    // number of tiles on every SM), so that no tile waits for a CTA slot;
+    // 32 pairs per thread when even those are too many
+#define UE_FIT(P)                                                                        \
+    if ((z.Q + kThreads * P - 1) / (kThreads * P) <= tile_slots<P>(num_sms)) return kThreads * P;
+    UE_REROUTE_PER(UE_FIT)
+#undef UE_FIT
     return kThreads * 32;
 }
 

@@ -23,9 +23,9 @@ __device__ __forceinline__ void raise_error(int* err, int code, int detail)
 constexpr int kWarp = 32;
 constexpr unsigned kFull = 0xffffffffu;
 
-// Reroute tiling: threads per tile; a tile holds 16, 24 or 32 pairs per
-// thread (kRerouteTile: the 16-pair default), chosen per context so that
-// every tile is resident at once. The look-back adds the counts of groups of
+// Reroute tiling: threads per tile; a tile holds 8 to 32 pairs per thread
+// (kRerouteTile: the 16-pair default), chosen per context so that every tile
+// is resident at once. The look-back adds the counts of groups of
 // kRerouteGroup tiles.
 constexpr int kRerouteThreads = 512;
 constexpr int kRerouteWarps = kRerouteThreads / kWarp;
@@ -134,7 +134,7 @@ inline int64_t reroute_groups(const Sizes& z, int tile)
 // the reroute kernels' dynamic shared memory limits, set once per device
 // (outside any stream capture) before the first launch
 cudaError_t reroute_setup();
-// pairs per tile for this GPU: the smallest of the three whose tiles fit at
+// pairs per tile for this GPU: the smallest size on offer whose tiles fit at
 // once (call after reroute_setup)
 int reroute_tile(const Sizes& z, int num_sms);
 cudaError_t launch_reroute(const Sizes& z, int tile, const int32_t* idx,
