@@ -1181,7 +1181,7 @@ def main():
                     "combine); plan and reroute sequential",
             "sample": f"{tn} slice(s) of 512 tokens per rank x {w.R} ranks ({tp} pairs, "
                       f"{ts:.1f} s)",
-            "checked": "first slice's outputs equal to the single-threaded oracle's"}
+            "checked": "outputs on a 64-token-per-rank slice equal to the single-threaded oracle's"}
 
     if rank == 0:
         line = {
