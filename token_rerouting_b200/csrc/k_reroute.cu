@@ -19,27 +19,30 @@
 // the locality-aware split gave that rank (a per-(source rank, slot) table
 // of first occurrence and row base, built by local_tables_kernel).
 //
-// Design (B200): a single-pass stable counting sort with a decoupled
-// look-back. Each CTA takes a tile of 8192 pairs by an atomic ticket (so every
-// tile it waits on is already running), stages the ids in shared memory and
-// counts them per warp sub-range, then publishes its per-expert tile counts
-// at once so that successors never wait on its later work. While its
-// predecessors finish, it rebuilds the plan's copy lists (at most 512
-// entries). The look-back runs H = min(4, 512/E) threads per expert column;
-// each reads 16 predecessors per step with independent loads, so one step
-// covers 16*H tiles, and the column adds their counts up to the nearest
-// inclusive prefix. With every tile resident at once this cuts the serial
-// chain of L2 round trips by the window width.
-// Every wait is bounded: when it runs out the tile publishes an error flag,
-// records UE_ERR_TIMEOUT and writes nothing. Finally each warp re-walks its
-// 512 pairs in order, ranking equal ids within 32 lanes (the lanes holding
-// the same id come from nine ballots over the id's bits), and writes the
-// physical slot and dispatch row; for floor-form quotas the copy index comes
-// from one exact multiply-high by a per-expert reciprocal, otherwise from the
-// binary search.
+// Design (B200): a single-pass stable counting sort. Each CTA takes a tile
+// of 512 threads x 8 to 32 pairs by an atomic ticket (so every tile it waits
+// on is already running), stages the ids in shared memory, counts them per
+// warp sub-range and publishes its per-expert counts at once; then it
+// arrives at its group of 16 tiles. The group's last arrival, whose members
+// have all published, writes each member's exclusive prefix inside the group
+// into the member's word and the group's sum into the group's word, then
+// looks back over the groups before it (each group word is published by a
+// tile with a lower ticket) to the nearest inclusive prefix, and publishes
+// the group's inclusive prefix. A tile's exclusive prefix per expert is its
+// own word plus the previous group's inclusive prefix: two loads per expert
+// once they are out, so few tiles read the same words. Meanwhile each tile
+// rebuilds the plan's copy table (at most 512 entries).
+// Every wait is bounded: when it runs out the waiter records UE_ERR_TIMEOUT,
+// publishes an error flag where others wait on it, and its tile writes
+// nothing. Finally each warp re-walks its pairs in order, ranking equal ids
+// within 32 lanes (the lanes holding the same id come from eight or nine
+// ballots over the id's bits), and writes the physical slot and dispatch
+// row; for floor-form quotas the copy index comes from one exact
+// multiply-high by a per-expert reciprocal, otherwise from a binary search.
 // The status words carry the launch's tag, so nothing is cleared between
 // launches: words of earlier launches read as "not yet published". The last
-// CTA to finish resets the ticket and the counter and advances the epoch.
+// CTA to finish resets the ticket and the counter and advances the epoch;
+// each group's last arrival resets the group's counter.
 #include "ue_internal.cuh"
 
 namespace ue {
@@ -47,8 +50,6 @@ namespace {
 
 constexpr int kThreads = kRerouteThreads;
 constexpr int kWarps = kRerouteWarps;
-constexpr int kWindow = 16;  // look-back items read per thread at a time
-constexpr int kMaxH = 4;     // threads per expert column in the look-back
 
 __device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p)
 {
@@ -68,17 +69,33 @@ __device__ __forceinline__ unsigned long long status_word(uint32_t tag, uint32_t
     return ((unsigned long long)tag << 32) | (flag << 30) | (v & kValueMask);
 }
 
-// the lanes of the warp holding the same key (9-bit keys): one ballot per bit
-__device__ __forceinline__ unsigned same_key_lanes(int key)
+// the lanes of the warp holding the same expert id (-1 for none): one ballot
+// per bit of the id, 8 bits when E <= 255 (-1 reads as 255, which no expert
+// has), 9 otherwise
+__device__ __forceinline__ unsigned same_key_lanes(int ex, int E)
 {
     unsigned peers = kFull;
 #pragma unroll
-    for (int b = 0; b < 9; ++b) {
-        const bool bit = (key >> b) & 1;
+    for (int b = 0; b < 8; ++b) {
+        const bool bit = (ex >> b) & 1;
+        const unsigned m = __ballot_sync(kFull, bit);
+        peers &= bit ? m : ~m;
+    }
+    if (E > 255) {
+        const bool bit = (ex >> 8) & 1;
         const unsigned m = __ballot_sync(kFull, bit);
         peers &= bit ? m : ~m;
     }
     return peers;
+}
+
+// floor(x / d) for x < 2^32 and m = ceil(2^64 / d) (d >= 2), or x when d == 1:
+// the high 64 bits of x * m from two 32-bit products
+__device__ __forceinline__ unsigned div_m32(unsigned x, unsigned d, unsigned long long m)
+{
+    const unsigned long long t =
+        (unsigned long long)x * (unsigned)(m >> 32) + __umulhi(x, (unsigned)m);
+    return d == 1u ? x : (unsigned)(t >> 32);
 }
 
 // per-expert data used for every pair of the tile (16-byte aligned records)
@@ -173,8 +190,8 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     __shared__ ExpA s_a[kMaxE];
     __shared__ ExpB s_bm[kMaxE];
     __shared__ ExpC s_c[kMaxE];
-    __shared__ int s_cp[kMaxE + kMaxG];   // copy table: physical slot, copies of
-    __shared__ int s_cr[kMaxE + kMaxG];   // each expert in order; first dispatch row;
+    __shared__ int2 s_cpr[kMaxE + kMaxG]; // copy table, copies of each expert in
+                                          // order: (physical slot, first dispatch row);
     __shared__ int s_cs[kMaxE + kMaxG + 1];  // first pair index o of the copy
     __shared__ short s_ce[kMaxE + kMaxG];    // expert of each copy-table entry
     __shared__ union {
@@ -184,10 +201,6 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
             int se[kMaxG];                // plan: slot_expert
             int sq[kMaxE + kMaxG];        // plan: slot_quota
         } pro;
-        struct {  // look-back: one partial sum per (h, e)
-            uint32_t part[kMaxH][kMaxE];
-            unsigned char state[kMaxH][kMaxE];
-        } lb;
     } u;
     __shared__ int s_wsum[kWarps];
     __shared__ int s_tile;
@@ -285,28 +298,64 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     if (tid < G) u.pro.se[tid] = pl_se;
     __syncthreads();
     if (s_fin) {
-        // the last tile of the group to arrive publishes the group's sum (its
-        // members published their counts before they arrived)
+        // the last tile of the group to arrive (its members published their
+        // counts before they arrived): each member's exclusive prefix inside
+        // the group goes into the member's own word (flag: prefix), and the
+        // group's sum into the group's word (flag: aggregate)
         if (tid < E) {
             unsigned long long v[kRerouteGroup];
 #pragma unroll
             for (int i = 0; i < kRerouteGroup; ++i)
                 v[i] = i < members ? ld_relaxed(sc.status + (size_t)(gfirst + i) * E + tid) : 0ull;
-            uint32_t sum = 0, flag = kFlagAggregate;
+            uint32_t run = 0, flag = kFlagAggregate;
             int64_t polls = 0;
 #pragma unroll
             for (int i = 0; i < kRerouteGroup; ++i) {
                 if (i < members && flag == kFlagAggregate) {
                     if (wait_word(sc.status + (size_t)(gfirst + i) * E + tid, tag, v[i], polls,
                                   spin_limit)) {
-                        sum += (uint32_t)v[i] & kValueMask;
+                        st_relaxed(sc.status + (size_t)(gfirst + i) * E + tid,
+                                   status_word(tag, kFlagPrefix, run));
+                        run += (uint32_t)v[i] & kValueMask;
                     } else {
                         raise_error(err, UE_ERR_TIMEOUT, gfirst + i);
                         flag = kFlagError;
                     }
                 }
             }
-            st_relaxed(sc.gstatus + (size_t)grp * E + tid, status_word(tag, flag, sum));
+            if (flag == kFlagError) {
+                for (int i = 0; i < members; ++i)
+                    st_relaxed(sc.status + (size_t)(gfirst + i) * E + tid,
+                               status_word(tag, kFlagError, 0u));
+            }
+            st_relaxed(sc.gstatus + (size_t)grp * E + tid, status_word(tag, flag, run));
+            // then the group's inclusive prefix: its sum plus the sums of the
+            // groups before it, back to the nearest group whose inclusive
+            // prefix is out (decoupled look-back over groups, each of whose
+            // words is published by a tile with a lower ticket)
+            if (flag == kFlagAggregate) {
+                uint32_t pre = 0;
+                int gb = grp - 1;
+                bool done = gb < 0;
+                while (!done) {
+                    unsigned long long w = ld_relaxed(sc.gstatus + (size_t)gb * E + tid);
+                    if (!wait_word(sc.gstatus + (size_t)gb * E + tid, tag, w, polls, spin_limit)) {
+                        raise_error(err, UE_ERR_TIMEOUT, gb);
+                        flag = kFlagError;
+                        break;
+                    }
+                    const uint32_t f = (uint32_t)w >> 30;
+                    if (f == kFlagError) {
+                        flag = kFlagError;
+                        break;
+                    }
+                    pre += (uint32_t)w & kValueMask;
+                    done = f == kFlagPrefix || --gb < 0;
+                }
+                st_relaxed(sc.gstatus + (size_t)grp * E + tid,
+                           status_word(tag, flag == kFlagError ? kFlagError : kFlagPrefix,
+                                       pre + run));
+            }
         }
         // every member has arrived: ready for the next launch
         if (tid == 0) sc.gcount[grp] = 0u;
@@ -345,8 +394,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
             const int mp = (e / M) * (M + S) + (e % M);
             const int cb = wofs + incl - c;
             s_c[e] = ExpC{c, cb};          // completed below
-            s_cp[cb] = mp;                 // copy 0: the master
-            s_cr[cb] = u.pro.off[mp];
+            s_cpr[cb] = make_int2(mp, u.pro.off[mp]);  // copy 0: the master
             s_ce[cb] = (short)e;
             u.pro.run[e] = cb + 1;         // next replica entry
         }
@@ -365,8 +413,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
             if (e >= 0) {
                 const int ci = u.pro.run[e] + __popc(peers & ((1u << lane) - 1u));
                 const int p = (g / S) * (M + S) + M + (g % S);
-                s_cp[ci] = p;
-                s_cr[ci] = u.pro.off[p];
+                s_cpr[ci] = make_int2(p, u.pro.off[p]);
                 s_ce[ci] = (short)e;
             }
             __syncwarp();
@@ -378,7 +425,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     {
         // every copy's start: an exclusive scan of the quotas over the
         // entries (experts in order, each one's copies in copy order)
-        const int q = tid < nent ? u.pro.sq[s_cp[tid]] : 0;
+        const int q = tid < nent ? u.pro.sq[s_cpr[tid].x] : 0;
         int incl = q;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -408,7 +455,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         const int e = s_ce[tid];
         const ExpC c0 = s_c[e];
         const int j = tid - c0.cb;
-        const int q = u.pro.sq[s_cp[tid]];
+        const int q = u.pro.sq[s_cpr[tid].x];
         const unsigned b = (unsigned)s_a[e].L / (unsigned)c0.b;
         if (kOrder == kOrderLocal || q != (int)b + (j < s_a[e].rem ? 1 : 0)) u.pro.ff[e] = 0;
         s_cs[tid] -= u.pro.base[e];
@@ -425,57 +472,49 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         s_bm[tid] = ExpB{recip64(b + 1u), recip64(b)};
         s_c[tid] = ExpC{floor_form ? (int)b : c0.b, c0.cb};
     }
-    __syncthreads();  // the union switches from the copy table to look-back
+    __syncthreads();
 
     // ---- look back: this tile's exclusive prefix per expert ----
-    // the group sums of the groups before this tile's group, plus the counts
-    // of the tiles before it in its group. H threads per expert column, each
-    // summing every H-th item, kWindow independent loads at a time.
-    const int H = min(kMaxH, kThreads / E);
-    const int h = tid / E;
-    const int e = tid - h * E;
-    const int n_items = grp + (tile - gfirst);
-    if (h < H) {
-        uint32_t part = 0;
-        unsigned char st = 0;  // 0: fine, 2: error
-        int64_t polls = 0;
-        // item it: group sum `it` (it < grp), else the count of tile
-        // gfirst + it - grp
-        auto item = [&](int it) {
-            return it < grp ? sc.gstatus + (size_t)it * E + e
-                            : sc.status + (size_t)(gfirst + it - grp) * E + e;
-        };
-        for (int i0 = h; i0 < n_items && st == 0; i0 += H * kWindow) {
-            unsigned long long v[kWindow];
-#pragma unroll
-            for (int i = 0; i < kWindow; ++i) {
-                const int it = i0 + i * H;
-                v[i] = it < n_items ? ld_relaxed(item(it)) : 0ull;
-            }
-#pragma unroll
-            for (int i = 0; i < kWindow; ++i) {
-                if (i0 + i * H < n_items && st == 0) {
-                    if (!wait_word(item(i0 + i * H), tag, v[i], polls, spin_limit)) {
-                        raise_error(err, UE_ERR_TIMEOUT, tile);
-                        st = 2;
-                    } else if (((uint32_t)v[i] >> 30) == kFlagError) {
-                        st = 2;
-                    } else {
-                        part += (uint32_t)v[i] & kValueMask;
-                    }
-                }
-            }
-        }
-        u.lb.part[h][e] = part;
-        u.lb.state[h][e] = st;
-    }
-    __syncthreads();
+    // the tile's own word (its exclusive prefix inside its group, put there
+    // by the group's last arrival) plus the inclusive prefix of the group
+    // before (or, while that is not out yet, the sums of the groups before,
+    // back to the nearest inclusive prefix)
     if (tid < E) {
         uint32_t excl = 0;
-        for (int hh = 0; hh < H; ++hh) {
-            if (u.lb.state[hh][tid] != 0) s_fail = 1;
-            excl += u.lb.part[hh][tid];
+        bool fail = false;
+        int64_t polls = 0;
+        const unsigned long long* own = sc.status + (size_t)tile * E + tid;
+        unsigned long long w = ld_relaxed(own);
+        // wait for the prefix flag (the tile's own count is there first)
+        while (!fail && ((uint32_t)(w >> 32) != tag || ((uint32_t)w >> 30) == kFlagInvalid ||
+                         ((uint32_t)w >> 30) == kFlagAggregate)) {
+            if (++polls > spin_limit) {
+                raise_error(err, UE_ERR_TIMEOUT, tile);
+                fail = true;
+            } else {
+                __nanosleep(64);
+                w = ld_relaxed(own);
+            }
         }
+        if (!fail && ((uint32_t)w >> 30) == kFlagError) fail = true;
+        excl = (uint32_t)w & kValueMask;
+        int gb = grp - 1;
+        while (!fail && gb >= 0) {
+            unsigned long long gw = ld_relaxed(sc.gstatus + (size_t)gb * E + tid);
+            if (!wait_word(sc.gstatus + (size_t)gb * E + tid, tag, gw, polls, spin_limit)) {
+                raise_error(err, UE_ERR_TIMEOUT, tile);
+                fail = true;
+                break;
+            }
+            const uint32_t f = (uint32_t)gw >> 30;
+            if (f == kFlagError) {
+                fail = true;
+                break;
+            }
+            excl += (uint32_t)gw & kValueMask;
+            gb = f == kFlagPrefix ? -1 : gb - 1;
+        }
+        if (fail) s_fail = 1;
         s_a[tid].pre = (int)excl;
     }
     __syncthreads();
@@ -485,17 +524,35 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     // the o-th pair of expert e: with floor-form quotas, copy j = o / (b+1)
     // while o < rem*(b+1), else rem + (o - rem*(b+1)) / b; otherwise the
     // last copy whose start is <= o. Row = first row of the copy + (o - start).
+    const unsigned lt = (1u << lane) - 1u;
 #pragma unroll 2
     for (int rd = 0; rd < (write_out ? kPer : 0); ++rd) {
         const int x = warp * kPerWarpP + rd * 32 + lane;
         const int ex = s_idx[x];
-        const unsigned peers = same_key_lanes(ex & 511);
+        const unsigned peers = same_key_lanes(ex, E);
+        const unsigned below = __popc(peers & lt);  // same expert, lower lanes
+        const int ev = ex < 0 ? 0 : ex;             // a safe index for the loads
         const int64_t i = pair_at<kOrder>(t0 + x, ord);
+        const int base = s_wh[warp][ev];
+        const ExpA a = s_a[ev];
+        const ExpC c = s_c[ev];
+        const int o = a.pre + base + (int)below;
         int p = -1, row = -1;
-        if (ex >= 0) {
-            const ExpA a = s_a[ex];
-            const int o = a.pre + s_wh[warp][ex] + __popc(peers & ((1u << lane) - 1u));
-            const ExpC c = s_c[ex];
+        if (kOrder != kOrderLocal && __all_sync(kFull, ex < 0 || (a.rem >= 0 && o < a.L))) {
+            // every lane of the round has floor-form quotas: no branches
+            const ExpB bm = s_bm[ev];
+            const bool big = o < a.thr;
+            const unsigned d = big ? (unsigned)c.b + 1u : (unsigned)c.b;
+            const unsigned x0 = big ? (unsigned)o : (unsigned)(o - a.thr);
+            const unsigned q = div_m32(x0, d, big ? bm.m1 : bm.m0);
+            const int j = big ? (int)q : a.rem + (int)q;
+            const int start = j * c.b + min(j, a.rem);
+            const int2 cr = s_cpr[c.cb + j];
+            if (ex >= 0) {
+                p = cr.x;
+                row = cr.y + (o - start);
+            }
+        } else if (ex >= 0) {
             if (o >= a.L) {
                 // the plan does not cover this pair (plan from other ids)
                 raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(i, (int64_t)INT_MAX));
@@ -504,8 +561,8 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
                 // splits them (c.b is the number of copies here)
                 const unsigned r = div_m((unsigned)i, ord.TK, ord.mTK);
                 const int32_t* fr = ord.first + (size_t)r * ord.P;
-                const int j = last_at_most(c.b, o, [&](int jj) { return __ldg(fr + s_cp[c.cb + jj]); });
-                const int pj = s_cp[c.cb + j];
+                const int j = last_at_most(c.b, o, [&](int jj) { return __ldg(fr + s_cpr[c.cb + jj].x); });
+                const int pj = s_cpr[c.cb + j].x;
                 const size_t rp = (size_t)r * ord.P + pj;
                 if (o - __ldg(fr + pj) < __ldg(ord.quota + rp)) {
                     p = pj;
@@ -515,24 +572,25 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
                     raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(i, (int64_t)INT_MAX));
                 }
             } else if (a.rem >= 0) {
-                const ExpB bm = s_bm[ex];
+                const ExpB bm = s_bm[ev];
                 const bool big = o < a.thr;
                 const unsigned d = big ? (unsigned)c.b + 1u : (unsigned)c.b;
                 const unsigned x0 = big ? (unsigned)o : (unsigned)(o - a.thr);
-                const unsigned q = div_m(x0, d, big ? bm.m1 : bm.m0);
+                const unsigned q = div_m32(x0, d, big ? bm.m1 : bm.m0);
                 const int j = big ? (int)q : a.rem + (int)q;
                 const int start = j * c.b + min(j, a.rem);
-                const int ci = c.cb + j;
-                p = s_cp[ci];
-                row = s_cr[ci] + (o - start);
+                const int2 cr = s_cpr[c.cb + j];
+                p = cr.x;
+                row = cr.y + (o - start);
             } else {
                 const int ci = c.cb + last_at_most(c.b, o, [&](int jj) { return s_cs[c.cb + jj]; });
-                p = s_cp[ci];
-                row = s_cr[ci] + (o - s_cs[ci]);
+                p = s_cpr[ci].x;
+                row = s_cpr[ci].y + (o - s_cs[ci]);
             }
         }
         __syncwarp();
-        if (ex >= 0 && lane == __ffs(peers) - 1) s_wh[warp][ex] += (short)__popc(peers);
+        // the lowest lane of each expert's group moves the warp's count on
+        if (ex >= 0 && below == 0u) s_wh[warp][ev] = (short)(base + (int)__popc(peers));
         __syncwarp();
         if (x < cnt_tile) {
             phys_slot[i] = p;
