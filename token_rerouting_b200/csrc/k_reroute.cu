@@ -139,9 +139,30 @@ __device__ __forceinline__ int last_at_most(int n, int o, Key key)
 }
 
 // ceil(2^64 / d) for d >= 2; floor(x / d) = umul64hi(x, m) exactly when x*d < 2^64
+// (computed as floor((2^64 - 1) / d) + 1: the high half by a 32-bit division,
+// the low half, a quotient below 2^32, by an fp64 estimate within one unit
+// corrected with the exact remainder)
 __device__ __forceinline__ unsigned long long recip64(unsigned d)
 {
-    return d <= 1u ? 0ull : (0xffffffffffffffffull / d) + 1ull;
+    if (d <= 1u) return 0ull;
+    const unsigned hi = 0xffffffffu / d;
+    const unsigned r1 = 0xffffffffu - hi * d;  // < d
+    const unsigned long long x = ((unsigned long long)r1 << 32) | 0xffffffffull;  // < d 2^32
+    unsigned long long lo = (unsigned long long)((double)x / (double)d);
+    long long rem = (long long)(x - lo * d);   // small: the estimate is within one unit
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+        if (rem < 0) {
+            --lo;
+            rem += d;
+        }
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+        if (rem >= (long long)d) {
+            ++lo;
+            rem -= d;
+        }
+    return ((unsigned long long)hi << 32) + lo + 1ull;
 }
 
 __device__ __forceinline__ unsigned div_m(unsigned x, unsigned d, unsigned long long m)
@@ -696,7 +717,7 @@ cudaError_t launch_tiles(const Sizes& z, const int32_t* idx, const ue_placement&
 }
 
 // pairs per thread of the tile sizes on offer (tile = 512 * kPer)
-#define UE_REROUTE_PER(X) X(8) X(10) X(12) X(14) X(16) X(20) X(24) X(28) X(32)
+#define UE_REROUTE_PER(X) X(7) X(8) X(10) X(12) X(14) X(16) X(18) X(20) X(24) X(28) X(32)
 
 template <int kOrder>
 cudaError_t launch_order(const Sizes& z, int tile, const int32_t* idx, const ue_placement& plan,
