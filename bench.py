@@ -840,6 +840,63 @@ def planner_oracle_baseline(w, logits):
                       "plan feeds the reroutes)"}
 
 
+def run_routing_row(args, w):
+    """The routing half alone (gate with the count fused in, plan, reroute) on
+    one layer instance without row buffers (logits and routing arrays only:
+    a small device footprint, for kernel captures). Each call timed alone as
+    replays of a CUDA graph of back-to-back launches, CUDA events on the
+    replay stream."""
+    import torch
+
+    import token_rerouting_b200 as ue
+    from token_rerouting_b200 import build as ue_build
+
+    ue_build.build()
+    dev = torch.device("cuda", 0)
+    L = ue.Layer(w.R, w.T, w.E, w.K, w.S, w.d, device=0, with_rows=False)
+    L.logits.copy_(torch.from_numpy(synth_logits(w)))
+    for _ in range(max(3, args.warmup)):
+        L.run_routing()
+    torch.cuda.synchronize(dev)
+    s = torch.cuda.Stream(dev)
+    us = {}
+    for name, f in (("gate_count", L.gate_count), ("plan", L.plan_step), ("reroute", L.reroute)):
+        with torch.cuda.stream(s):
+            f(stream=s)
+            torch.cuda.synchronize(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(args.steps):
+                    f(stream=s)
+            g.replay()
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            g.replay()
+            b.record(s)
+        torch.cuda.synchronize(dev)
+        us[name] = a.elapsed_time(b) * 1e3 / args.steps
+        del g
+    rc = L.error()
+    plan = L.plan_arrays()
+    L.close()
+    if rc != 0:
+        raise SystemExit(f"device error: {ue.STATUS.get(rc, rc)}")
+    ab = algorithmic_bytes(w)
+    peak, peak_kind = load_peaks()
+    line = {"row": "routing", "config": dict(workload=w.name, R=w.R, T=w.T, E=w.E, K=w.K, S=w.S,
+                                              pairs=w.Q),
+            "steps": args.steps, "us": us,
+            "frac_of_peak": {k: ab[k] / (us[k] / 1e6) / 1e9 / peak for k in ("gate_count",
+                                                                              "reroute")},
+            "peak_kind": f"of {peak_kind}",
+            "us_routing_total": sum(us.values()),
+            "plan": {"iterations": int(plan["stats"][0]),
+                     "max_over_mean_before": float(plan["stats"][1]) / (w.Q / w.R),
+                     "max_over_mean_after": float(plan["stats"][2]) / (w.Q / w.R)}}
+    print(json.dumps(line), flush=True)
+
+
 def synth_logits(w):
     import synth
     return synth.logits(w)
@@ -866,9 +923,10 @@ def main():
     ap.add_argument("--planner", choices=("greedy", "bisect"), default="greedy",
                     help="planner of the sweep (greedy: the path's rule)")
     ap.add_argument("--row", choices=("backward", "weight_sync", "grad_reduce", "planner",
-                                      "layouts"),
+                                      "layouts", "routing"),
                     default=None, help="measure one of the rows beside the forward path "
-                    "(planner: the planner variants, on pages_ep64_e256_t8k by default)")
+                    "(planner: the planner variants, on pages_ep64_e256_t8k by default; "
+                    "routing: the routing half alone, without row buffers)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -888,6 +946,9 @@ def main():
         return
     if args.row == "planner":
         run_planner(args, w)
+        return
+    if args.row == "routing":
+        run_routing_row(args, w)
         return
     if args.row:
         run_row(args, w)
