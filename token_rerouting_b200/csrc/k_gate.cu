@@ -405,11 +405,13 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_
     __shared__ int s_hist[COUNT ? kGateHist : 1][HE];
     __shared__ uint32_t s_epoch, s_ticket, s_ok;
 
+    // row indices fit 32 bits here: K = 8 and Q < 2^30 give N < 2^27
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int64_t row_beg = (int64_t)blockIdx.x * rows_per_cta;
-    const int64_t row_end = min(N, row_beg + rows_per_cta);
-    int64_t rank0 = 0;
+    const int row_beg = (int)blockIdx.x * (int)rows_per_cta;
+    const int row_end = (int)min(N, (int64_t)row_beg + rows_per_cta);
+    int rank0 = 0;
+    int bnd[kGateHist - 1] = {};  // first rows of the source ranks after rank0
     if constexpr (COUNT) {
         for (int x = threadIdx.x; x < kGateHist * E; x += blockDim.x) (&s_hist[0][0])[x] = 0;
         if (threadIdx.x == 0) {
@@ -427,6 +429,8 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_
             if (threadIdx.x == 0) st_release_gpu(cnt.sync + 3, s_epoch + 1u);
         }
         rank0 = row_beg / cnt.T;
+#pragma unroll
+        for (int q = 1; q < kGateHist; ++q) bnd[q - 1] = (rank0 + q) * cnt.T;
     }
 
     uint32_t lo[VPL];
@@ -435,12 +439,12 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_
     const int r = lane / kFastK;   // this lane's row of the group in the epilogue
     const int k = lane % kFastK;   // and its rank among the row's picks
 
-    for (int64_t row0 = row_beg + (int64_t)warp * kFastRows; row0 < row_end;
-         row0 += (int64_t)kGateWarps * kFastRows) {
-        const int rows = (int)min((int64_t)kFastRows, row_end - row0);
+    for (int row0 = row_beg + warp * kFastRows; row0 < row_end; row0 += kGateWarps * kFastRows) {
+        const int rows = min(kFastRows, row_end - row0);
+        const float* grp_rows = logits + (size_t)row0 * E;
         FastRow<NCH4, NT> v[kFastRows];
 #pragma unroll
-        for (int b = 0; b < kFastRows; ++b) v[b].load(logits + (row0 + b) * (int64_t)E, lane, b < rows);
+        for (int b = 0; b < kFastRows; ++b) v[b].load(grp_rows + b * E, lane, b < rows);
         unsigned dry = 0u;  // rows whose reserve keys may belong to the top K+1
         if (rows == kFastRows) {
 #pragma unroll
@@ -461,15 +465,15 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_
         unsigned redo = __ballot_sync(kFull, act && (a >> LOB) == (nx >> LOB)) | dry;
         while (redo) {
             const int rr = (__ffs(redo) - 1) / kFastK;
-            select_exact_row<NCH4, NT>(logits + (row0 + rr) * (int64_t)E, lane, s_win[warp][rr]);
+            select_exact_row<NCH4, NT>(grp_rows + rr * E, lane, s_win[warp][rr]);
             redo &= ~(0xffu << (rr * kFastK));
         }
         __syncwarp();
         // gate weights of the whole group at once, fp64
         // (lanes of rows past the end hold stale picks: they read nothing)
         const int e = act ? (E - 1) - (int)(s_win[warp][r][k] & kLo) : 0;
-        const int64_t row = row0 + (act ? r : 0);
-        const float vf = act ? __ldg(logits + row * (int64_t)E + e) : 0.0f;
+        const int row = row0 + (act ? r : 0);
+        const float vf = act ? __ldg(grp_rows + r * E + e) : 0.0f;
         const int lead = act ? r * kFastK : 0;
         const double v_own = (double)vf;
         const double v0 = __shfl_sync(kFull, v_own, lead);
@@ -482,15 +486,14 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_
         z += __shfl_xor_sync(kFull, z, 2);
         z += __shfl_xor_sync(kFull, z, 4);
         if (act) {
-            const int64_t pos = row * (int64_t)kFastK + k;
+            const int pos = row * kFastK + k;
             idx[pos] = (int32_t)e;
             w[pos] = (float)(x * __drcp_rn(z));
             if constexpr (COUNT) {
                 // source rank of the row, relative to the CTA's first rank
-                const int64_t rel = row - rank0 * cnt.T;
                 int hs = 0;
 #pragma unroll
-                for (int q = 1; q < kGateHist; ++q) hs += rel >= (int64_t)q * cnt.T ? 1 : 0;
+                for (int q = 0; q < kGateHist - 1; ++q) hs += row >= bnd[q] ? 1 : 0;
                 atomicAdd(&s_hist[hs][e], 1);
             }
         }
@@ -517,7 +520,7 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_
                 const int h = (&s_hist[0][0])[x];
                 if (h) {
                     const int hs = x / E, ex = x - hs * E;
-                    atomicAdd(&cnt.load_re[(rank0 + hs) * E + ex], h);
+                    atomicAdd(&cnt.load_re[(size_t)(rank0 + hs) * E + ex], h);
                     atomicAdd(&cnt.load_e[ex], h);
                 }
             }
