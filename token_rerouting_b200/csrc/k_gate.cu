@@ -172,10 +172,13 @@ gate_topk_kernel(const float* __restrict__ logits, int64_t N, int E, int Krt,
 // exactly that: if the first K+1 packed picks of a row differ pairwise in
 // their high parts (adjacent ones suffice: they are sorted), every unpicked
 // key lies strictly below the K-th pick, and the picks are in exact order.
+// Each lane pops from a list of its three largest keys only (select_packed);
+// a lane that gives up its whole list shows up as two equal adjacent picks.
 // Rows that fail the check (two of the leading values within 2^-16 relative
-// of each other, or exact ties) are selected again with full keys and the
-// id tie rule, from the row read again (an L1 hit: the loads allocate in
-// L1). The results are identical to the generic kernel's in every case.
+// of each other, exact ties, or a lane holding three or more of the first K
+// picks) are selected again with full keys and the id tie rule, from the row
+// read again (an L1 hit: the loads allocate in L1). The results are
+// identical to the generic kernel's in every case.
 //
 // Lane l holds experts e = 128 c + 4 l + j (chunk c < NCH4, j < 4: one
 // 16-byte load per chunk) and then 128 NCH4 + 32 t + l (t < NT: one 4-byte
@@ -262,6 +265,49 @@ __device__ __forceinline__ void sort_desc(uint32_t (&k)[VPL])
     }
 }
 
+// descending sort of four distinct keys held anywhere
+__device__ __forceinline__ void sort4_desc(uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d)
+{
+    cas_desc(a, b); cas_desc(c, d);
+    cas_desc(a, c); cas_desc(b, d);
+    cas_desc(b, c);
+}
+
+// The D largest of VPL distinct keys into k[0..D-1], descending (the rest of
+// k is left unspecified). D >= VPL sorts the whole list; otherwise the first
+// four are sorted and the others merged in: two sorted quadruples through
+// the max of opposite ends (the top D of both, a bitonic sequence, then
+// sorted), single keys by insertion at the bottom of the top D.
+template <int VPL, int D>
+__device__ __forceinline__ void top_desc(uint32_t (&k)[VPL])
+{
+    if constexpr (D >= VPL || VPL == 4) {
+        sort_desc<VPL>(k);
+    } else if constexpr (VPL == 8) {
+        static_assert(D == 3 || D == 4, "fast gate path: list depth 3 or 4");
+        sort4_desc(k[0], k[1], k[2], k[3]);
+        sort4_desc(k[4], k[5], k[6], k[7]);
+#pragma unroll
+        for (int i = 0; i < D; ++i) k[i] = max(k[i], k[4 + D - 1 - i]);
+        if constexpr (D == 4) {
+            cas_desc(k[0], k[2]); cas_desc(k[1], k[3]);
+            cas_desc(k[0], k[1]); cas_desc(k[2], k[3]);
+        } else {
+            cas_desc(k[0], k[1]); cas_desc(k[1], k[2]); cas_desc(k[0], k[1]);
+        }
+    } else {
+        static_assert(VPL > 4 && VPL < 8 && (D == 3 || D == 4),
+                      "fast gate path: list depth 3 or 4");
+        sort4_desc(k[0], k[1], k[2], k[3]);
+#pragma unroll
+        for (int i = 4; i < VPL; ++i) {
+            k[D - 1] = max(k[D - 1], k[i]);
+#pragma unroll
+            for (int j = D - 1; j > 0; --j) cas_desc(k[j - 1], k[j]);
+        }
+    }
+}
+
 template <int NCH4, int NT>
 struct FastRow {
     static constexpr int VPL = 4 * NCH4 + NT;
@@ -295,23 +341,31 @@ __device__ __forceinline__ int fast_expert(int i, int lane)
     return i < 4 * NCH4 ? 128 * (i >> 2) + 4 * lane + (i & 3) : 128 * NCH4 + 32 * (i - 4 * NCH4) + lane;
 }
 
-// The K+1 packed picks of one row into win[0..K]; lane 0 writes them. The
-// rounds pop within the first D keys of each lane's sorted list only (three
-// shifts instead of VPL - 1); the keys below are a reserve. That is exact
-// unless a lane gives up all D listed keys and its next key lies above the
-// (K+1)-th pick, which the return value reports (the row is then selected
-// again with full keys).
+// Depth of the per-lane lists of the packed selection: every key when a
+// lane holds at most three, else the three largest.
+__host__ __device__ constexpr int fast_depth(int vpl) { return vpl < 3 ? vpl : 3; }
+
+// The K+1 packed picks of one row into win[0..K]; lane 0 writes them. Each
+// lane keeps its D largest keys, sorted, and a pop shifts the list up.
+// With at most three keys a lane (D = VPL) the pop fills the bottom with 0,
+// which never wins, and every pick is exact. Otherwise the pop leaves the
+// last entry in place: a lane that gives up all D keys before the last round
+// then offers its last key again, which is the largest key left in the row
+// and is picked again at once. Those two equal adjacent picks send the row to
+// the exact selection (the caller checks adjacent picks); without them every
+// pick is exact, since a lane's keys below its list lie below its last entry.
 template <int NCH4, int NT>
-__device__ __forceinline__ bool select_packed(const FastRow<NCH4, NT>& v,
+__device__ __forceinline__ void select_packed(const FastRow<NCH4, NT>& v,
                                               const uint32_t (&lo)[4 * NCH4 + NT], uint32_t khi,
                                               uint32_t* win, bool writer)
 {
     constexpr int VPL = 4 * NCH4 + NT;
-    constexpr int D = VPL > 3 ? 3 : VPL;
+    constexpr int D = fast_depth(VPL);
+    constexpr bool kFill = VPL < 4;
     uint32_t key[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) key[i] = packed_key(v.at(i), lo[i], khi);
-    sort_desc<VPL>(key);
+    top_desc<VPL, D>(key);
 #pragma unroll
     for (int k = 0; k < kFastK; ++k) {
         const uint32_t m = __reduce_max_sync(kFull, key[0]);
@@ -319,16 +373,10 @@ __device__ __forceinline__ bool select_packed(const FastRow<NCH4, NT>& v,
         const bool pop = key[0] == m;
 #pragma unroll
         for (int j = 0; j < D - 1; ++j) key[j] = pop ? key[j + 1] : key[j];
-        key[D - 1] = pop ? 0u : key[D - 1];
+        if constexpr (kFill) key[D - 1] = pop ? 0u : key[D - 1];
     }
     const uint32_t m = __reduce_max_sync(kFull, key[0]);
     if (writer) win[kFastK] = m;
-    if constexpr (VPL > D) {
-        // packed keys are never 0, so key[0] == 0 means the list ran dry
-        return __any_sync(kFull, key[0] == 0u && key[D] > m);
-    } else {
-        return false;
-    }
 }
 
 // Exact selection of one row read again from global memory: full keys,
@@ -443,26 +491,27 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_
         const int rows = min(kFastRows, row_end - row0);
         const float* grp_rows = logits + (size_t)row0 * E;
         FastRow<NCH4, NT> v[kFastRows];
-#pragma unroll
-        for (int b = 0; b < kFastRows; ++b) v[b].load(grp_rows + b * E, lane, b < rows);
-        unsigned dry = 0u;  // rows whose reserve keys may belong to the top K+1
         if (rows == kFastRows) {
 #pragma unroll
-            for (int b = 0; b < kFastRows; ++b)
-                if (select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0))
-                    dry |= 0xffu << (b * kFastK);
-        } else {
+            for (int b = 0; b < kFastRows; ++b) v[b].load(grp_rows + b * E, lane, true);
 #pragma unroll
             for (int b = 0; b < kFastRows; ++b)
-                if (b < rows && select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0))
-                    dry |= 0xffu << (b * kFastK);
+                select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0);
+        } else {
+            // the last group of the CTA: rows past its end read the last row
+#pragma unroll
+            for (int b = 0; b < kFastRows; ++b)
+                v[b].load(grp_rows + min(b, rows - 1) * E, lane, true);
+#pragma unroll
+            for (int b = 0; b < kFastRows; ++b)
+                if (b < rows) select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0);
         }
         __syncwarp();
         // rows whose leading picks agree above the dropped bits: exact again
         const bool act = r < rows;
         const uint32_t a = s_win[warp][r][k];
         const uint32_t nx = s_win[warp][r][k + 1];
-        unsigned redo = __ballot_sync(kFull, act && (a >> LOB) == (nx >> LOB)) | dry;
+        unsigned redo = __ballot_sync(kFull, act && (a >> LOB) == (nx >> LOB));
         while (redo) {
             const int rr = (__ffs(redo) - 1) / kFastK;
             select_exact_row<NCH4, NT>(grp_rows + rr * E, lane, s_win[warp][rr]);
