@@ -7,6 +7,9 @@ row whose first K+1 picks are not separated above the dropped bits. These
 tests mix, inside the same warp groups of four rows, rows of distinct normal
 logits (packed picks kept), rows of exact ties and signed zeros, and rows of
 values a few fp32 ulps apart (both re-selected), with a ragged last group.
+Each lane pops from a short list of its largest keys; rows whose leading
+values sit in one lane (three or more of them, before or at the last round)
+test the hand-over from a lane that ran out of its list.
 Both paths must give the oracle's ids bit for bit and its weights within one
 fp32 ulp; a logits buffer that is not 16-byte aligned takes the generic
 kernel, which must agree as well.
@@ -95,6 +98,59 @@ def test_unaligned_logits_take_the_generic_kernel(E):
     gh.assert_weights_close(w_a, w_or)
     gh.assert_weights_close(w_u, w_or)
     np.testing.assert_array_equal(w_a, w_u)
+
+
+def lane_experts(E, lane):
+    """Experts one lane of the fast kernel holds: 128 c + 4 lane + j for each
+    16-byte chunk c, then 128 C + 32 t + lane for each 4-byte tail load t."""
+    nch, nt = E // 128, (E % 128) // 32
+    ids = [128 * c + 4 * lane + j for c in range(nch) for j in range(4)]
+    return ids + [128 * nch + 32 * t + lane for t in range(nt)]
+
+
+# positions among the leading K+1 values that one lane's experts take
+CLUSTERS = [(0, 1, 2), (0, 1, 8), (0, 4, 7), (5, 6, 7, 8), (1, 2, 3, 4), (0, 1, 2, 3, 4, 5),
+            (2, 7), (7, 8)]
+
+
+def clustered_logits(N, E, seed):
+    """Rows whose leading values sit in one lane of the fast kernel, at the
+    positions CLUSTERS lists (a lane that gives up its whole list before the
+    last round, or exactly at it), between rows of distinct normal logits."""
+    rng = np.random.default_rng(seed)
+    out = rng.standard_normal((N, E)).astype(np.float32)
+    for n in range(0, N, 2):
+        pos = CLUSTERS[(n // 2) % len(CLUSTERS)]
+        mine = lane_experts(E, int(rng.integers(32)))
+        pos = pos[:len(mine)]
+        out[n] -= 10.0
+        others = rng.permutation(np.setdiff1d(np.arange(E), mine))
+        chosen = rng.permutation(mine)[:len(pos)]
+        o = 0
+        for p in range(9):
+            if p in pos:
+                e = chosen[pos.index(p)]
+            else:
+                e = others[o]
+                o += 1
+            out[n, e] = np.float32(10.0 - p)
+    return out
+
+
+@pytest.mark.parametrize("E", [64, 96, 128, 160, 192, 224, 256])
+def test_one_lane_holding_many_leading_picks(E):
+    gh.ensure_built()
+    N = 2002
+    logits = clustered_logits(N, E, seed=7 * E)
+    idx_or, w_or = oracle.gate_topk(logits, 8)
+    idx, w = run_gate(E, N, logits)
+    np.testing.assert_array_equal(idx, idx_or)
+    gh.assert_weights_close(w, w_or)
+    (res,) = run_gate_count(2, N // 2, E, [logits])
+    np.testing.assert_array_equal(res[0], idx_or)
+    lre_or, le_or = oracle.count(idx_or, 2, N // 2, E)
+    np.testing.assert_array_equal(res[2], lre_or)
+    np.testing.assert_array_equal(res[3], le_or)
 
 
 def test_all_rows_equal_pick_the_lowest_ids():

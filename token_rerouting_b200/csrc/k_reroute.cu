@@ -58,6 +58,17 @@ __device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long lon
     return v;
 }
 
+// atomic add with release and acquire semantics at GPU scope: the arrival
+// publishes what the CTA wrote before it (ordered by the barrier before) and
+// sees what earlier arrivals published
+__device__ __forceinline__ uint32_t add_acq_rel(uint32_t* p, uint32_t v)
+{
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;"
+                 : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 __device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long long v)
 {
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
@@ -183,6 +194,18 @@ __device__ __forceinline__ int64_t pair_at(int64_t u, const OrderArgs& o)
     return ((int64_t)r * o.T + t) * o.K + k;
 }
 
+// the same for Q < 2^30, in 32 bits
+template <int kOrder>
+__device__ __forceinline__ unsigned pair_at32(unsigned u, const OrderArgs& o)
+{
+    if (kOrder != kOrderInterleave) return u;
+    const unsigned t = div_m(u, o.RK, o.mRK);
+    const unsigned w = u - t * o.RK;
+    const unsigned r = div_m(w, o.K, o.mK);
+    const unsigned k = w - r * o.K;
+    return (r * o.T + t) * o.K + k;
+}
+
 // wait (bounded) until *p holds a word of this launch, then return it in w;
 // false when the wait ran out
 __device__ __forceinline__ bool wait_word(const unsigned long long* p, uint32_t tag,
@@ -216,10 +239,11 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     __shared__ int s_cs[kMaxE + kMaxG + 1];  // first pair index o of the copy
     __shared__ short s_ce[kMaxE + kMaxG];    // expert of each copy-table entry
     __shared__ union {
+        int4 align16;
         struct {  // building the copy table
-            int cnt[kMaxE], run[kMaxE], base[kMaxE], ff[kMaxE];
+            int se[kMaxG];                // plan: slot_expert (16-byte aligned)
+            int cnt[kMaxE], base[kMaxE], ff[kMaxE];
             int off[kMaxE + kMaxG + 1];   // plan: slot_offset
-            int se[kMaxG];                // plan: slot_expert
             int sq[kMaxE + kMaxG];        // plan: slot_quota
         } pro;
     } u;
@@ -228,6 +252,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     __shared__ uint32_t s_tag;
     __shared__ int s_fail;
     __shared__ int s_fin;
+    __shared__ int s_allff;  // every expert's quotas of the floor form
 
     const int M = E / R;
     const int G = R * S;
@@ -243,6 +268,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         const uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(&sc.sync[2]);
         s_tag = epoch + 1u == 0u ? 1u : epoch + 1u;
         s_fail = 0;
+        s_allff = kOrder == kOrderLocal ? 0 : 1;
     }
     for (int x = tid; x < kWarps * kMaxE; x += kThreads) (&s_wh[0][0])[x] = 0;
     for (int e = tid; e < E; e += kThreads) {
@@ -307,11 +333,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     const int gfirst = grp * kRerouteGroup;
     const int members = min(kRerouteGroup, ntiles - gfirst);
     __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        s_fin = atomicAdd(&sc.gcount[grp], 1u) == (uint32_t)(members - 1) ? 1 : 0;
-        __threadfence();
-    }
+    if (tid == 0) s_fin = add_acq_rel(&sc.gcount[grp], 1u) == (uint32_t)(members - 1) ? 1 : 0;
     // the plan into shared memory
     if (tid <= P) u.pro.off[tid] = pl_off0;
     if (tid + kThreads <= P) u.pro.off[tid + kThreads] = pl_off1;
@@ -383,12 +405,25 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     }
 
     // ---- copy table of every expert, from the plan ----
-    for (int g = tid; g < G; g += kThreads) {
-        const int e = u.pro.se[g];
-        if (e >= 0 && e < E) {
-            atomicAdd(&u.pro.cnt[e], 1);
-        } else if (e >= E) {
-            raise_error(err, UE_ERR_DEVICE_BOUNDS, g);
+    // slot g (one per thread: G <= kMaxG <= kThreads) counts the slots of
+    // its expert below it, which places it among the expert's replicas
+    // (ascending g), and adds itself to the expert's copies
+    int slot_e = -1, slot_rank = 0;
+    if (tid < G) {
+        slot_e = u.pro.se[tid];
+        if (slot_e >= E) {
+            raise_error(err, UE_ERR_DEVICE_BOUNDS, tid);
+            slot_e = -1;
+        }
+        if (slot_e >= 0) {
+            const int4* se4 = reinterpret_cast<const int4*>(u.pro.se);
+            int g = 0;
+            for (; g + 4 <= tid; g += 4) {
+                const int4 q = se4[g >> 2];
+                slot_rank += (q.x == slot_e) + (q.y == slot_e) + (q.z == slot_e) + (q.w == slot_e);
+            }
+            for (; g < tid; ++g) slot_rank += u.pro.se[g] == slot_e;
+            atomicAdd(&u.pro.cnt[slot_e], 1);
         }
     }
     __syncthreads();
@@ -417,30 +452,15 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
             s_c[e] = ExpC{c, cb};          // completed below
             s_cpr[cb] = make_int2(mp, u.pro.off[mp]);  // copy 0: the master
             s_ce[cb] = (short)e;
-            u.pro.run[e] = cb + 1;         // next replica entry
         }
         __syncthreads();
     }
-    if (warp == 0) {
-        // replicas in ascending g after each expert's master
-        for (int g0 = 0; g0 < G; g0 += 32) {
-            const int g = g0 + lane;
-            int e = -1;
-            if (g < G) {
-                e = u.pro.se[g];
-                if (e >= E) e = -1;
-            }
-            const unsigned peers = __match_any_sync(kFull, e);
-            if (e >= 0) {
-                const int ci = u.pro.run[e] + __popc(peers & ((1u << lane) - 1u));
-                const int p = (g / S) * (M + S) + M + (g % S);
-                s_cpr[ci] = make_int2(p, u.pro.off[p]);
-                s_ce[ci] = (short)e;
-            }
-            __syncwarp();
-            if (e >= 0 && lane == __ffs(peers) - 1) u.pro.run[e] += __popc(peers);
-            __syncwarp();
-        }
+    if (slot_e >= 0) {
+        // the replicas after their expert's master, in ascending g
+        const int ci = s_c[slot_e].cb + 1 + slot_rank;
+        const int p = (tid / S) * (M + S) + M + (tid % S);
+        s_cpr[ci] = make_int2(p, u.pro.off[p]);
+        s_ce[ci] = (short)slot_e;
     }
     __syncthreads();
     {
@@ -488,6 +508,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         const ExpC c0 = s_c[tid];
         const ExpA a = s_a[tid];
         const bool floor_form = u.pro.ff[tid] != 0;
+        if (!floor_form) s_allff = 0;
         const unsigned b = (unsigned)a.L / (unsigned)c0.b;
         s_a[tid] = ExpA{0, a.L, a.thr, floor_form ? a.rem : -1};
         s_bm[tid] = ExpB{recip64(b + 1u), recip64(b)};
@@ -546,53 +567,63 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     // while o < rem*(b+1), else rem + (o - rem*(b+1)) / b; otherwise the
     // last copy whose start is <= o. Row = first row of the copy + (o - start).
     const unsigned lt = (1u << lane) - 1u;
+    if (kOrder != kOrderLocal && s_allff) {
+        // every expert has floor-form quotas: no per-round vote. A pair
+        // beyond its expert's load (ids that do not match the plan) is
+        // reported, and its rank is clamped so that the table reads stay
+        // inside the expert's copies.
+        const unsigned t0u = (unsigned)t0;
 #pragma unroll 2
-    for (int rd = 0; rd < (write_out ? kPer : 0); ++rd) {
-        const int x = warp * kPerWarpP + rd * 32 + lane;
-        const int ex = s_idx[x];
-        const unsigned peers = same_key_lanes(ex, E);
-        const unsigned below = __popc(peers & lt);  // same expert, lower lanes
-        const int ev = ex < 0 ? 0 : ex;             // a safe index for the loads
-        const int64_t i = pair_at<kOrder>(t0 + x, ord);
-        const int base = s_wh[warp][ev];
-        const ExpA a = s_a[ev];
-        const ExpC c = s_c[ev];
-        const int o = a.pre + base + (int)below;
-        int p = -1, row = -1;
-        if (kOrder != kOrderLocal && __all_sync(kFull, ex < 0 || (a.rem >= 0 && o < a.L))) {
-            // every lane of the round has floor-form quotas: no branches
+        for (int rd = 0; rd < (write_out ? kPer : 0); ++rd) {
+            const int x = warp * kPerWarpP + rd * 32 + lane;
+            const int ex = s_idx[x];
+            const unsigned peers = same_key_lanes(ex, E);
+            const unsigned below = __popc(peers & lt);
+            const int ev = ex < 0 ? 0 : ex;
+            const unsigned i = pair_at32<kOrder>(t0u + (unsigned)x, ord);
+            const int base = s_wh[warp][ev];
+            const ExpA a = s_a[ev];
+            const ExpC c = s_c[ev];
             const ExpB bm = s_bm[ev];
-            const bool big = o < a.thr;
+            const int o = a.pre + base + (int)below;
+            const int oc = min(o, max(a.L - 1, 0));
+            const bool big = oc < a.thr;
             const unsigned d = big ? (unsigned)c.b + 1u : (unsigned)c.b;
-            const unsigned x0 = big ? (unsigned)o : (unsigned)(o - a.thr);
+            const unsigned x0 = big ? (unsigned)oc : (unsigned)(oc - a.thr);
             const unsigned q = div_m32(x0, d, big ? bm.m1 : bm.m0);
             const int j = big ? (int)q : a.rem + (int)q;
             const int start = j * c.b + min(j, a.rem);
             const int2 cr = s_cpr[c.cb + j];
-            if (ex >= 0) {
-                p = cr.x;
-                row = cr.y + (o - start);
+            int p = cr.x, row = cr.y + (oc - start);
+            if (ex < 0 || o >= a.L) {
+                if (ex >= 0) raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(i, (unsigned)INT_MAX));
+                p = -1;
+                row = -1;
             }
-        } else if (ex >= 0) {
-            if (o >= a.L) {
-                // the plan does not cover this pair (plan from other ids)
-                raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(i, (int64_t)INT_MAX));
-            } else if (kOrder == kOrderLocal) {
-                // copies of e in copy order, as this pair's source rank
-                // splits them (c.b is the number of copies here)
-                const unsigned r = div_m((unsigned)i, ord.TK, ord.mTK);
-                const int32_t* fr = ord.first + (size_t)r * ord.P;
-                const int j = last_at_most(c.b, o, [&](int jj) { return __ldg(fr + s_cpr[c.cb + jj].x); });
-                const int pj = s_cpr[c.cb + j].x;
-                const size_t rp = (size_t)r * ord.P + pj;
-                if (o - __ldg(fr + pj) < __ldg(ord.quota + rp)) {
-                    p = pj;
-                    row = __ldg(ord.rowb + rp) + o;
-                } else {
-                    // the split does not cover this pair (split from other ids)
-                    raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(i, (int64_t)INT_MAX));
-                }
-            } else if (a.rem >= 0) {
+            __syncwarp();
+            if (ex >= 0 && below == 0u) s_wh[warp][ev] = (short)(base + (int)__popc(peers));
+            __syncwarp();
+            if (x < cnt_tile) {
+                phys_slot[i] = p;
+                dest_row[i] = row;
+            }
+        }
+    } else {
+#pragma unroll 2
+        for (int rd = 0; rd < (write_out ? kPer : 0); ++rd) {
+            const int x = warp * kPerWarpP + rd * 32 + lane;
+            const int ex = s_idx[x];
+            const unsigned peers = same_key_lanes(ex, E);
+            const unsigned below = __popc(peers & lt);  // same expert, lower lanes
+            const int ev = ex < 0 ? 0 : ex;             // a safe index for the loads
+            const int64_t i = pair_at<kOrder>(t0 + x, ord);
+            const int base = s_wh[warp][ev];
+            const ExpA a = s_a[ev];
+            const ExpC c = s_c[ev];
+            const int o = a.pre + base + (int)below;
+            int p = -1, row = -1;
+            if (kOrder != kOrderLocal && __all_sync(kFull, ex < 0 || (a.rem >= 0 && o < a.L))) {
+                // every lane of the round has floor-form quotas: no branches
                 const ExpB bm = s_bm[ev];
                 const bool big = o < a.thr;
                 const unsigned d = big ? (unsigned)c.b + 1u : (unsigned)c.b;
@@ -601,21 +632,54 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
                 const int j = big ? (int)q : a.rem + (int)q;
                 const int start = j * c.b + min(j, a.rem);
                 const int2 cr = s_cpr[c.cb + j];
-                p = cr.x;
-                row = cr.y + (o - start);
-            } else {
-                const int ci = c.cb + last_at_most(c.b, o, [&](int jj) { return s_cs[c.cb + jj]; });
-                p = s_cpr[ci].x;
-                row = s_cpr[ci].y + (o - s_cs[ci]);
+                if (ex >= 0) {
+                    p = cr.x;
+                    row = cr.y + (o - start);
+                }
+            } else if (ex >= 0) {
+                if (o >= a.L) {
+                    // the plan does not cover this pair (plan from other ids)
+                    raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(i, (int64_t)INT_MAX));
+                } else if (kOrder == kOrderLocal) {
+                    // copies of e in copy order, as this pair's source rank
+                    // splits them (c.b is the number of copies here)
+                    const unsigned r = div_m((unsigned)i, ord.TK, ord.mTK);
+                    const int32_t* fr = ord.first + (size_t)r * ord.P;
+                    const int j = last_at_most(c.b, o, [&](int jj) { return __ldg(fr + s_cpr[c.cb + jj].x); });
+                    const int pj = s_cpr[c.cb + j].x;
+                    const size_t rp = (size_t)r * ord.P + pj;
+                    if (o - __ldg(fr + pj) < __ldg(ord.quota + rp)) {
+                        p = pj;
+                        row = __ldg(ord.rowb + rp) + o;
+                    } else {
+                        // the split does not cover this pair (split from other ids)
+                        raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(i, (int64_t)INT_MAX));
+                    }
+                } else if (a.rem >= 0) {
+                    const ExpB bm = s_bm[ev];
+                    const bool big = o < a.thr;
+                    const unsigned d = big ? (unsigned)c.b + 1u : (unsigned)c.b;
+                    const unsigned x0 = big ? (unsigned)o : (unsigned)(o - a.thr);
+                    const unsigned q = div_m32(x0, d, big ? bm.m1 : bm.m0);
+                    const int j = big ? (int)q : a.rem + (int)q;
+                    const int start = j * c.b + min(j, a.rem);
+                    const int2 cr = s_cpr[c.cb + j];
+                    p = cr.x;
+                    row = cr.y + (o - start);
+                } else {
+                    const int ci = c.cb + last_at_most(c.b, o, [&](int jj) { return s_cs[c.cb + jj]; });
+                    p = s_cpr[ci].x;
+                    row = s_cpr[ci].y + (o - s_cs[ci]);
+                }
             }
-        }
-        __syncwarp();
-        // the lowest lane of each expert's group moves the warp's count on
-        if (ex >= 0 && below == 0u) s_wh[warp][ev] = (short)(base + (int)__popc(peers));
-        __syncwarp();
-        if (x < cnt_tile) {
-            phys_slot[i] = p;
-            dest_row[i] = row;
+            __syncwarp();
+            // the lowest lane of each expert's group moves the warp's count on
+            if (ex >= 0 && below == 0u) s_wh[warp][ev] = (short)(base + (int)__popc(peers));
+            __syncwarp();
+            if (x < cnt_tile) {
+                phys_slot[i] = p;
+                dest_row[i] = row;
+            }
         }
     }
 
@@ -623,8 +687,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     // ready for the next launch
     __syncthreads();
     if (tid == 0) {
-        __threadfence();
-        if (atomicAdd(&sc.sync[1], 1u) == gridDim.x - 1) {
+        if (add_acq_rel(&sc.sync[1], 1u) == gridDim.x - 1) {
             sc.sync[0] = 0u;
             sc.sync[1] = 0u;
             __threadfence();
