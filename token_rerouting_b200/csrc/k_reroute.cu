@@ -239,10 +239,10 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     __shared__ int s_cs[kMaxE + kMaxG + 1];  // first pair index o of the copy
     __shared__ short s_ce[kMaxE + kMaxG];    // expert of each copy-table entry
     __shared__ union {
-        int4 align16;
         struct {  // building the copy table
-            int se[kMaxG];                // plan: slot_expert (16-byte aligned)
-            int cnt[kMaxE], base[kMaxE], ff[kMaxE];
+            int se[kMaxG];                // plan: slot_expert
+            unsigned char cntc[kMaxG / 32][kMaxE];  // slots of each expert per chunk of 32
+            int base[kMaxE], ff[kMaxE];
             int off[kMaxE + kMaxG + 1];   // plan: slot_offset
             int sq[kMaxE + kMaxG];        // plan: slot_quota
         } pro;
@@ -271,10 +271,9 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         s_allff = kOrder == kOrderLocal ? 0 : 1;
     }
     for (int x = tid; x < kWarps * kMaxE; x += kThreads) (&s_wh[0][0])[x] = 0;
-    for (int e = tid; e < E; e += kThreads) {
-        u.pro.cnt[e] = 0;
-        u.pro.ff[e] = 1;
-    }
+    for (int x = tid; x < kMaxG / 32 * kMaxE / 4; x += kThreads)
+        reinterpret_cast<int*>(&u.pro.cntc[0][0])[x] = 0;
+    for (int e = tid; e < E; e += kThreads) u.pro.ff[e] = 1;
     // the plan, into registers now (its loads overlap the tile's)
     int pl_off0 = 0, pl_off1 = 0, pl_sq = 0, pl_se = -1;
     if (tid <= P) pl_off0 = __ldg(plan.slot_offset + tid);
@@ -405,9 +404,10 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     }
 
     // ---- copy table of every expert, from the plan ----
-    // slot g (one per thread: G <= kMaxG <= kThreads) counts the slots of
-    // its expert below it, which places it among the expert's replicas
-    // (ascending g), and adds itself to the expert's copies
+    // slot g (one per thread: G <= kMaxG <= kThreads) takes its place among
+    // its expert's replicas (ascending g): its rank inside its chunk of 32
+    // slots (lanes holding the same expert) plus the expert's slots in the
+    // chunks below, from a per-chunk count
     int slot_e = -1, slot_rank = 0;
     if (tid < G) {
         slot_e = u.pro.se[tid];
@@ -415,22 +415,25 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
             raise_error(err, UE_ERR_DEVICE_BOUNDS, tid);
             slot_e = -1;
         }
+    }
+    if (warp * 32 < G) {  // warp-uniform
+        const unsigned peers = same_key_lanes(slot_e, E);
         if (slot_e >= 0) {
-            const int4* se4 = reinterpret_cast<const int4*>(u.pro.se);
-            int g = 0;
-            for (; g + 4 <= tid; g += 4) {
-                const int4 q = se4[g >> 2];
-                slot_rank += (q.x == slot_e) + (q.y == slot_e) + (q.z == slot_e) + (q.w == slot_e);
-            }
-            for (; g < tid; ++g) slot_rank += u.pro.se[g] == slot_e;
-            atomicAdd(&u.pro.cnt[slot_e], 1);
+            slot_rank = __popc(peers & ((1u << lane) - 1u));
+            if (slot_rank == 0) u.pro.cntc[warp][slot_e] = (unsigned char)__popc(peers);
         }
     }
     __syncthreads();
+    const int nchunks = (G + 31) / 32;
+    if (slot_e >= 0)
+        for (int ch = 0; ch < warp; ++ch) slot_rank += u.pro.cntc[ch][slot_e];
+    int ncopies = 1;  // of expert tid: the master and its replicas
+    if (tid < E)
+        for (int ch = 0; ch < nchunks; ++ch) ncopies += u.pro.cntc[ch][tid];
     int nent;  // copy-table entries: every expert's master and replicas
     {
         // exclusive scan of copies per expert (1 + replicas) over experts
-        const int c = tid < E ? 1 + u.pro.cnt[tid] : 0;
+        const int c = tid < E ? ncopies : 0;
         int incl = c;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
