@@ -57,9 +57,6 @@ TRAFFIC = {
     },
     # ncu --set full at 512 tokens per rank, times 8
     "qwen3_layer_r64_e128": {
-        "gate_count": {"bytes_per_launch": 134520000, "source_sha": "f9c2f7be091df85a"},
-        "plan": {"bytes_per_launch": 29000, "source_sha": "2edfc203d9880067"},
-        "reroute": {"bytes_per_launch": 8968000, "source_sha": "237f5cbb848c661f"},
         "permute": {"bytes_per_launch": 18890168000, "source_sha": "07222823ab0e9db7"},
         "combine": {"bytes_per_launch": 21242032000, "source_sha": "c0631738399ffc37"},
     },
