@@ -76,6 +76,18 @@ struct Pick {
     int rm;        // the master's rank, e / M
 };
 
+// floor(x / d) for 0 < d < 2^31 and a quotient below 2^51 (here x < 2^50, or
+// x < 2^63 with x / d < 2^33): the fp64 estimate x * (1/d) is within one unit
+// of it, and the exact remainder moves the estimate to the right side
+__device__ __forceinline__ unsigned long long floor_div_exact(unsigned long long x,
+                                                              unsigned long long d, double inv)
+{
+    unsigned long long q = (unsigned long long)((double)x * inv);
+    if (q * d > x) --q;
+    else if ((q + 1ull) * d <= x) ++q;
+    return q;
+}
+
 // block-wide sum of v over all threads (every thread gets the total)
 __device__ __forceinline__ long long block_sum(long long v, long long* scratch)
 {
@@ -102,7 +114,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
     __shared__ int sRank[kMaxR];    // rank loads (initial, then final)
     __shared__ int sSlotE[kMaxG];   // expert of redundant slot g, -1 empty (final)
     __shared__ int sSlotQ[kMaxG];   // quota of redundant slot g (final)
-    __shared__ unsigned long long sKey[kCandMax];
+    __shared__ __align__(16) unsigned long long sKey[kCandMax];
     __shared__ unsigned long long sOrd[kMaxG];  // the first G keys in pick order
     __shared__ Pick sPick[kMaxG + 1];  // the picks in order (then an end marker)
     __shared__ long long sRed[kPlanWarps];
@@ -141,6 +153,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
     }
     const unsigned long long Qall = (unsigned long long)block_sum((long long)part, sRed);
     if (tid == 0) sQ = Qall;
+    const double invQ = Qall > 0ull ? 1.0 / (double)Qall : 0.0;
 
     // ---- the pick sequence, in parallel ----
     // candidates per expert at threshold Q/(G+E)/2^lvl (one thread per expert)
@@ -154,10 +167,9 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
                 if (min_tokens > 0u) cap = min(cap, L / (long long)min_tokens - 1);
                 if (L > 0 && cap > 0) {
                     const unsigned long long num = (unsigned long long)L * (unsigned)(G + E);
-                    const unsigned long long q = num / Qall, r = num - q * Qall;
                     long long th;
-                    if (lvl >= 10 && q > 0ull) th = cap;  // q * 2^lvl >= 1024 > cap
-                    else th = (long long)((q << lvl) + ((r << lvl) / Qall));
+                    if (lvl >= 10 && num >= Qall) th = cap;  // num 2^lvl / Q >= 1024 > cap
+                    else th = (long long)floor_div_exact(num << lvl, Qall, invQ);
                     cnt = (int)min(cap, th);
                     cut = th < cap;
                 }
@@ -211,9 +223,11 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
         const unsigned long long key = sKey[p];
         int place = 0;
         int q = 0;
-        for (; q + 4 <= total; q += 4)
-            place += (sKey[q] > key) + (sKey[q + 1] > key) + (sKey[q + 2] > key) +
-                     (sKey[q + 3] > key);
+        const ulonglong2* key2 = reinterpret_cast<const ulonglong2*>(sKey);
+        for (; q + 4 <= total; q += 4) {
+            const ulonglong2 a = key2[q >> 1], b = key2[(q >> 1) + 1];
+            place += (a.x > key) + (a.y > key) + (b.x > key) + (b.y > key);
+        }
         for (; q < total; ++q) place += sKey[q] > key;
         if (place < G) sOrd[place] = key;
     }
@@ -240,7 +254,8 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
     if (warp == 0) {
         // ---- rank side: stop test, least loaded free rank, bookkeeping ----
         const long long Q = (long long)sQ;
-        const long long stop_rhs = 51LL * Q;
+        // the stop test 50 R max_r load_r <= 51 Q, as max_r load_r <= floor(51 Q / (50 R))
+        const unsigned stop_max = (unsigned)((51LL * Q) / (50LL * R));
         unsigned load[NJR];
         int used[NJR];
         int slotE[NJR][SM], slotQ[NJR][SM];
@@ -257,6 +272,9 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
         }
         int iters = 0;
         unsigned max_before = 0u;
+#pragma unroll
+        for (int j = 0; j < NJR; ++j) max_before = max(max_before, load[j]);
+        max_before = __reduce_max_sync(kFull, max_before);
         // with every rank load below 2^25 (Q < 2^25), a rank's load and its
         // index (< 128) pack into one 32-bit key, and the least loaded rank
         // with a free slot (ties to the lowest r) is one reduction
@@ -278,8 +296,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
                 }
                 maxl = __reduce_max_sync(kFull, maxl);
                 key = __reduce_min_sync(kFull, key);
-                if (iters == 0) max_before = maxl;
-                if (50LL * R * (long long)maxl <= stop_rhs) break;
+                if (maxl <= stop_max) break;
                 if (key == 0xffffffffu) break;  // no free slot anywhere
                 rstar = (int)(key & 127u);
             } else {
@@ -293,8 +310,7 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
                 }
                 maxl = __reduce_max_sync(kFull, maxl);
                 const unsigned ml = __reduce_min_sync(kFull, bestl);
-                if (iters == 0) max_before = maxl;
-                if (50LL * R * (long long)maxl <= stop_rhs) break;
+                if (maxl <= stop_max) break;
                 if (ml == 0xffffffffu) break;  // no free slot anywhere
                 rstar = (int)__reduce_min_sync(kFull, bestl == ml ? bestr : 0xffffffffu);
             }
