@@ -842,7 +842,8 @@ def run_routing_row(args, w):
     one layer instance without row buffers (logits and routing arrays only:
     a small device footprint, for kernel captures). Each call timed alone as
     replays of a CUDA graph of back-to-back launches, CUDA events on the
-    replay stream."""
+    replay stream. The separate count call (ue_count, the same counts from
+    idx) is timed beside them but not part of the routing total."""
     import torch
 
     import token_rerouting_b200 as ue
@@ -857,7 +858,8 @@ def run_routing_row(args, w):
     torch.cuda.synchronize(dev)
     s = torch.cuda.Stream(dev)
     us = {}
-    for name, f in (("gate_count", L.gate_count), ("plan", L.plan_step), ("reroute", L.reroute)):
+    for name, f in (("gate_count", L.gate_count), ("plan", L.plan_step), ("reroute", L.reroute),
+                    ("count", L.count)):
         with torch.cuda.stream(s):
             f(stream=s)
             torch.cuda.synchronize(dev)
@@ -887,7 +889,7 @@ def run_routing_row(args, w):
             "frac_of_peak": {k: ab[k] / (us[k] / 1e6) / 1e9 / peak for k in ("gate_count",
                                                                               "reroute")},
             "peak_kind": f"of {peak_kind}",
-            "us_routing_total": sum(us.values()),
+            "us_routing_total": us["gate_count"] + us["plan"] + us["reroute"],
             "plan": {"iterations": int(plan["stats"][0]),
                      "max_over_mean_before": float(plan["stats"][1]) / (w.Q / w.R),
                      "max_over_mean_after": float(plan["stats"][2]) / (w.Q / w.R)}}

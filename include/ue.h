@@ -137,8 +137,11 @@ ue_status ue_gate_topk(ue_ctx* ctx, const float* logits, int32_t* idx,
  *   idx     int32 [N][K] expert ids (from ue_gate_topk).
  *   load_re int32 [R][E]: pairs of source rank r routed to expert e.
  *   load_e  int32 [E]: sum over r of load_re.
- * Both outputs are overwritten (zeroed on the stream first). An id outside
- * [0, E) is skipped and sets UE_ERR_DEVICE_BOUNDS. */
+ * Both outputs are overwritten: the kernel's first CTA zeroes them, and the
+ * others add their counts after it (a bounded wait; UE_ERR_TIMEOUT if it
+ * runs out). Uses the same context scratch as ue_gate_count (a ticket, a
+ * counter, an epoch and a flag), so calls on one context must not overlap on
+ * the GPU. An id outside [0, E) is skipped and sets UE_ERR_DEVICE_BOUNDS. */
 ue_status ue_count(ue_ctx* ctx, const int32_t* idx, int32_t* load_re,
                    int32_t* load_e, void* stream);
 

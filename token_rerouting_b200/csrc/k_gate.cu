@@ -426,18 +426,6 @@ __device__ __forceinline__ void select_exact_row(const float* row, int lane, uin
     }
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v)
-{
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 template <int NCH4, int NT, bool COUNT>
 __global__ void __launch_bounds__(kGateThreads, 4)
 gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_per_cta,
@@ -652,7 +640,7 @@ cudaError_t launch_gate_topk(const Sizes& z, const GateShape& sh, const float* l
 {
     if (z.N == 0) {
         if (cnt == nullptr) return cudaSuccess;
-        return launch_count(z, idx, cnt->load_re, cnt->load_e, cnt->err, st);
+        return launch_count(z, idx, cnt->load_re, cnt->load_e, cnt->sync, cnt->err, st);
     }
     if (sh.fast && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0) {
         const GateCount* fc = (cnt != nullptr && sh.fused) ? cnt : nullptr;
@@ -667,7 +655,7 @@ cudaError_t launch_gate_topk(const Sizes& z, const GateShape& sh, const float* l
         default: ce = launch_fast<2, 0>(z, sh, logits, idx, w, fc, st); break;
         }
         if (ce != cudaSuccess || cnt == nullptr || fc != nullptr) return ce;
-        return launch_count(z, idx, cnt->load_re, cnt->load_e, cnt->err, st);
+        return launch_count(z, idx, cnt->load_re, cnt->load_e, cnt->sync, cnt->err, st);
     }
     cudaError_t ce;
     switch ((z.E + 31) / 32) {
@@ -682,7 +670,7 @@ cudaError_t launch_gate_topk(const Sizes& z, const GateShape& sh, const float* l
     default: return cudaErrorInvalidValue;
     }
     if (ce != cudaSuccess || cnt == nullptr) return ce;
-    return launch_count(z, idx, cnt->load_re, cnt->load_e, cnt->err, st);
+    return launch_count(z, idx, cnt->load_re, cnt->load_e, cnt->sync, cnt->err, st);
 }
 
 }  // namespace ue

@@ -215,7 +215,7 @@ ue_status ue_count(ue_ctx* ctx, const int32_t* idx, int32_t* load_re, int32_t* l
     if (!ctx_ok(ctx) || !aligned(idx, 4) || !aligned(load_re, 4) || !aligned(load_e, 4))
         return UE_ERR_INVALID_ARG;
     if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
-    return from_cuda(ue::launch_count(ctx->z, idx, load_re, load_e, ctx->d_err,
+    return from_cuda(ue::launch_count(ctx->z, idx, load_re, load_e, ctx->d_gsync, ctx->d_err,
                                       as_stream(stream)));
 }
 

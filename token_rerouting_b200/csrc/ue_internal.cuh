@@ -20,6 +20,19 @@ __device__ __forceinline__ void raise_error(int* err, int code, int detail)
     }
 }
 
+// acquire load and release store of a 32-bit flag at GPU scope
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 constexpr int kWarp = 32;
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -106,8 +119,10 @@ GateShape plan_gate_shape(const Sizes& z, int num_sms);
 // (inside the gate kernel when the shape allows, else by launch_count)
 cudaError_t launch_gate_topk(const Sizes& z, const GateShape& sh, const float* logits,
                              int32_t* idx, float* w, const GateCount* cnt, cudaStream_t st);
+// sync: the same four words as GateCount's (ticket, finished CTAs, epoch,
+// flag), left ready for the next launch of either kernel
 cudaError_t launch_count(const Sizes& z, const int32_t* idx, int32_t* load_re,
-                         int32_t* load_e, int* err, cudaStream_t st);
+                         int32_t* load_e, uint32_t* sync, int* err, cudaStream_t st);
 // greedy plan; min_tokens = 0: every expert may take a copy
 cudaError_t launch_plan(const Sizes& z, const int32_t* load_e, int min_tokens,
                         const ue_placement& out, int* err, cudaStream_t st);
