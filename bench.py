@@ -40,6 +40,7 @@ UNIT = "pairs/s"
 DEFAULT_WORKLOAD = "prefill_ep40_e160"
 KERNELS = ("gate_count", "plan", "reroute", "permute", "combine")
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal: the roofline is also reported against it
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
 # each workload's kernels, from one ncu capture of the same workload at a
@@ -655,7 +656,8 @@ def run_row(args, w):
     line = {"row": args.row, "config": workload, "steps": args.steps, "kernels": out,
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": out[dom]["gbs"], "peak": peak,
                          "unit": "GB/s", "frac": out[dom]["frac_of_peak"],
-                         "peak_kind": f"of {peak_kind}"}}
+                         "peak_kind": f"of {peak_kind}", "nominal_peak": NOMINAL_HBM_GBS,
+                         "frac_of_nominal": out[dom]["gbs"] / NOMINAL_HBM_GBS}}
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = row_oracle_baseline(args, w, se_host)
     print(json.dumps(line), flush=True)
@@ -1134,7 +1136,8 @@ def main():
     traffic = (tr["bytes_per_launch"] if tr and tr.get("source_sha") == sha_of(src) else None)
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "peak_kind": f"of {peak_kind}",
-                "traffic": traffic, "algorithmic_bytes": abytes[dom]}
+                "traffic": traffic, "algorithmic_bytes": abytes[dom],
+                "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS}
     kernels = {}
     for k in KERNELS:
         ms = per_kernel_ms[k]
