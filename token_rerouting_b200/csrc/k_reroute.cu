@@ -50,6 +50,13 @@ namespace {
 
 constexpr int kThreads = kRerouteThreads;
 constexpr int kWarps = kRerouteWarps;
+constexpr int kHalf = kThreads / 2;  // threads of each half of a tile's CTA
+
+// barrier of one half of the CTA (named barriers 1 and 2; 0 is __syncthreads)
+__device__ __forceinline__ void half_sync(int id)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kHalf) : "memory");
+}
 
 __device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p)
 {
@@ -270,252 +277,272 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         s_fail = 0;
         s_allff = kOrder == kOrderLocal ? 0 : 1;
     }
-    for (int x = tid; x < kWarps * kMaxE; x += kThreads) (&s_wh[0][0])[x] = 0;
-    for (int x = tid; x < kMaxG / 32 * kMaxE / 4; x += kThreads)
-        reinterpret_cast<int*>(&u.pro.cntc[0][0])[x] = 0;
-    for (int e = tid; e < E; e += kThreads) u.pro.ff[e] = 1;
-    // the plan, into registers now (its loads overlap the tile's)
-    int pl_off0 = 0, pl_off1 = 0, pl_sq = 0, pl_se = -1;
-    if (tid <= P) pl_off0 = __ldg(plan.slot_offset + tid);
-    if (tid + kThreads <= P) pl_off1 = __ldg(plan.slot_offset + tid + kThreads);
-    if (tid < P) pl_sq = __ldg(plan.slot_quota + tid);
-    if (tid < G) pl_se = __ldg(plan.slot_expert + tid);
     __syncthreads();
-
-    // ---- stage the tile and count it per warp sub-range ----
     const int tile = s_tile;
     const uint32_t tag = s_tag;
     const int64_t t0 = (int64_t)tile * kTileP;
     const int cnt_tile = (int)min((int64_t)kTileP, Q - t0);
-    {
-        // issue all of this thread's loads before using any of them
-        int v[kPer];
-#pragma unroll
-        for (int q = 0; q < kPer; ++q) {
-            const int x = tid + q * kThreads;
-            v[q] = x < cnt_tile ? __ldg(idx + pair_at<kOrder>(t0 + x, ord)) : -1;
-        }
-#pragma unroll
-        for (int q = 0; q < kPer; ++q) {
-            const int x = tid + q * kThreads;
-            int e = v[q];
-            if (x < cnt_tile && (unsigned)e >= (unsigned)E) {
-                raise_error(err, UE_ERR_DEVICE_BOUNDS,
-                            (int)min(pair_at<kOrder>(t0 + x, ord), (int64_t)INT_MAX));
-                e = -1;
-            }
-            s_idx[x] = (short)e;
-        }
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int rd = 0; rd < kPer; ++rd) {
-        const int e = s_idx[warp * kPerWarpP + rd * 32 + lane];
-        if (e >= 0) atomicAdd_block(reinterpret_cast<int*>(&s_wh[warp][0]) + (e >> 1),
-                                    (e & 1) ? (1 << 16) : 1);
-    }
-    __syncthreads();
-
-    // ---- publish this tile's counts and arrive at its group ----
-    int acc = 0;
-    if (tid < E) {
-        for (int w = 0; w < kWarps; ++w) {
-            const int t = s_wh[w][tid];
-            s_wh[w][tid] = (short)acc;
-            acc += t;
-        }
-        if (!(drop_first && tile == 0))
-            st_relaxed(sc.status + (size_t)tile * E + tid,
-                       status_word(tag, kFlagAggregate, (uint32_t)acc));
-    }
     const int grp = tile / kRerouteGroup;
     const int gfirst = grp * kRerouteGroup;
     const int members = min(kRerouteGroup, ntiles - gfirst);
-    __syncthreads();
-    if (tid == 0) s_fin = add_acq_rel(&sc.gcount[grp], 1u) == (uint32_t)(members - 1) ? 1 : 0;
-    // the plan into shared memory
-    if (tid <= P) u.pro.off[tid] = pl_off0;
-    if (tid + kThreads <= P) u.pro.off[tid + kThreads] = pl_off1;
-    if (tid < P) u.pro.sq[tid] = pl_sq;
-    if (tid < G) u.pro.se[tid] = pl_se;
-    __syncthreads();
-    if (s_fin) {
-        // the last tile of the group to arrive (its members published their
-        // counts before they arrived): each member's exclusive prefix inside
-        // the group goes into the member's own word (flag: prefix), and the
-        // group's sum into the group's word (flag: aggregate)
-        if (tid < E) {
-            unsigned long long v[kRerouteGroup];
-#pragma unroll
-            for (int i = 0; i < kRerouteGroup; ++i)
-                v[i] = i < members ? ld_relaxed(sc.status + (size_t)(gfirst + i) * E + tid) : 0ull;
-            uint32_t run = 0, flag = kFlagAggregate;
-            int64_t polls = 0;
-#pragma unroll
-            for (int i = 0; i < kRerouteGroup; ++i) {
-                if (i < members && flag == kFlagAggregate) {
-                    if (wait_word(sc.status + (size_t)(gfirst + i) * E + tid, tag, v[i], polls,
-                                  spin_limit)) {
-                        st_relaxed(sc.status + (size_t)(gfirst + i) * E + tid,
-                                   status_word(tag, kFlagPrefix, run));
-                        run += (uint32_t)v[i] & kValueMask;
-                    } else {
-                        raise_error(err, UE_ERR_TIMEOUT, gfirst + i);
-                        flag = kFlagError;
-                    }
-                }
-            }
-            if (flag == kFlagError) {
-                for (int i = 0; i < members; ++i)
-                    st_relaxed(sc.status + (size_t)(gfirst + i) * E + tid,
-                               status_word(tag, kFlagError, 0u));
-            }
-            st_relaxed(sc.gstatus + (size_t)grp * E + tid, status_word(tag, flag, run));
-            // then the group's inclusive prefix: its sum plus the sums of the
-            // groups before it, back to the nearest group whose inclusive
-            // prefix is out (decoupled look-back over groups, each of whose
-            // words is published by a tile with a lower ticket)
-            if (flag == kFlagAggregate) {
-                uint32_t pre = 0;
-                int gb = grp - 1;
-                bool done = gb < 0;
-                while (!done) {
-                    unsigned long long w = ld_relaxed(sc.gstatus + (size_t)gb * E + tid);
-                    if (!wait_word(sc.gstatus + (size_t)gb * E + tid, tag, w, polls, spin_limit)) {
-                        raise_error(err, UE_ERR_TIMEOUT, gb);
-                        flag = kFlagError;
-                        break;
-                    }
-                    const uint32_t f = (uint32_t)w >> 30;
-                    if (f == kFlagError) {
-                        flag = kFlagError;
-                        break;
-                    }
-                    pre += (uint32_t)w & kValueMask;
-                    done = f == kFlagPrefix || --gb < 0;
-                }
-                st_relaxed(sc.gstatus + (size_t)grp * E + tid,
-                           status_word(tag, flag == kFlagError ? kFlagError : kFlagPrefix,
-                                       pre + run));
-            }
-        }
-        // every member has arrived: ready for the next launch
-        if (tid == 0) sc.gcount[grp] = 0u;
-    }
 
-    // ---- copy table of every expert, from the plan ----
-    // slot g (one per thread: G <= kMaxG <= kThreads) takes its place among
-    // its expert's replicas (ascending g): its rank inside its chunk of 32
-    // slots (lanes holding the same expert) plus the expert's slots in the
-    // chunks below, from a per-chunk count
-    int slot_e = -1, slot_rank = 0;
-    if (tid < G) {
-        slot_e = u.pro.se[tid];
-        if (slot_e >= E) {
-            raise_error(err, UE_ERR_DEVICE_BOUNDS, tid);
-            slot_e = -1;
-        }
-    }
-    if (warp * 32 < G) {  // warp-uniform
-        const unsigned peers = same_key_lanes(slot_e, E);
-        if (slot_e >= 0) {
-            slot_rank = __popc(peers & ((1u << lane) - 1u));
-            if (slot_rank == 0) u.pro.cntc[warp][slot_e] = (unsigned char)__popc(peers);
-        }
-    }
-    __syncthreads();
-    const int nchunks = (G + 31) / 32;
-    if (slot_e >= 0)
-        for (int ch = 0; ch < warp; ++ch) slot_rank += u.pro.cntc[ch][slot_e];
-    int ncopies = 1;  // of expert tid: the master and its replicas
-    if (tid < E)
-        for (int ch = 0; ch < nchunks; ++ch) ncopies += u.pro.cntc[ch][tid];
-    int nent;  // copy-table entries: every expert's master and replicas
-    {
-        // exclusive scan of copies per expert (1 + replicas) over experts
-        const int c = tid < E ? ncopies : 0;
-        int incl = c;
+    // Two halves of the CTA work side by side, each with its own barrier:
+    // warps 0-7 stage, count and publish the tile and arrive at its group;
+    // warps 8-15 rebuild the copy table from the plan, which does not depend
+    // on the tile.
+    if (tid < kHalf) {
+        // ---- stage the tile and count it per warp sub-range ----
+        for (int x = tid; x < kWarps * kMaxE; x += kHalf) (&s_wh[0][0])[x] = 0;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(kFull, incl, off);
-            if (lane >= off) incl += o;
+        for (int hb = 0; hb < 2; ++hb) {
+            // issue all of this batch's loads before using any of them
+            int v[kPer];
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                const int x = tid + (hb * kPer + q) * kHalf;
+                v[q] = x < cnt_tile ? __ldg(idx + pair_at<kOrder>(t0 + x, ord)) : -1;
+            }
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                const int x = tid + (hb * kPer + q) * kHalf;
+                int e = v[q];
+                if (x < cnt_tile && (unsigned)e >= (unsigned)E) {
+                    raise_error(err, UE_ERR_DEVICE_BOUNDS,
+                                (int)min(pair_at<kOrder>(t0 + x, ord), (int64_t)INT_MAX));
+                    e = -1;
+                }
+                s_idx[x] = (short)e;
+            }
         }
-        if (lane == 31) s_wsum[warp] = incl;
-        __syncthreads();
-        int wofs = 0, all = 0;
-        for (int w = 0; w < kWarps; ++w) {
-            wofs += w < warp ? s_wsum[w] : 0;
-            all += s_wsum[w];
+        half_sync(1);
+        // warp w counts the sub-ranges of output warps 2w and 2w + 1
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+            const int ow = 2 * warp + sub;
+#pragma unroll 4
+            for (int rd = 0; rd < kPer; ++rd) {
+                const int e = s_idx[ow * kPerWarpP + rd * 32 + lane];
+                if (e >= 0) atomicAdd_block(reinterpret_cast<int*>(&s_wh[ow][0]) + (e >> 1),
+                                            (e & 1) ? (1 << 16) : 1);
+            }
         }
-        nent = all;
+        half_sync(1);
+
+        // ---- publish this tile's counts and arrive at its group ----
         if (tid < E) {
-            const int e = tid;
-            const int mp = (e / M) * (M + S) + (e % M);
-            const int cb = wofs + incl - c;
-            s_c[e] = ExpC{c, cb};          // completed below
-            s_cpr[cb] = make_int2(mp, u.pro.off[mp]);  // copy 0: the master
-            s_ce[cb] = (short)e;
+            int acc = 0;
+            for (int w = 0; w < kWarps; ++w) {
+                const int t = s_wh[w][tid];
+                s_wh[w][tid] = (short)acc;
+                acc += t;
+            }
+            if (!(drop_first && tile == 0))
+                st_relaxed(sc.status + (size_t)tile * E + tid,
+                           status_word(tag, kFlagAggregate, (uint32_t)acc));
         }
-        __syncthreads();
-    }
-    if (slot_e >= 0) {
-        // the replicas after their expert's master, in ascending g
-        const int ci = s_c[slot_e].cb + 1 + slot_rank;
-        const int p = (tid / S) * (M + S) + M + (tid % S);
-        s_cpr[ci] = make_int2(p, u.pro.off[p]);
-        s_ce[ci] = (short)slot_e;
-    }
-    __syncthreads();
-    {
-        // every copy's start: an exclusive scan of the quotas over the
-        // entries (experts in order, each one's copies in copy order)
-        const int q = tid < nent ? u.pro.sq[s_cpr[tid].x] : 0;
-        int incl = q;
+        half_sync(1);
+        if (tid == 0)
+            s_fin = add_acq_rel(&sc.gcount[grp], 1u) == (uint32_t)(members - 1) ? 1 : 0;
+        half_sync(1);
+        if (s_fin) {
+            // the last tile of the group to arrive (its members published their
+            // counts before they arrived): each member's exclusive prefix inside
+            // the group goes into the member's own word (flag: prefix), and the
+            // group's sum into the group's word (flag: aggregate)
+            if (tid < E) {
+                unsigned long long v[kRerouteGroup];
+    #pragma unroll
+                for (int i = 0; i < kRerouteGroup; ++i)
+                    v[i] = i < members ? ld_relaxed(sc.status + (size_t)(gfirst + i) * E + tid) : 0ull;
+                uint32_t run = 0, flag = kFlagAggregate;
+                int64_t polls = 0;
+    #pragma unroll
+                for (int i = 0; i < kRerouteGroup; ++i) {
+                    if (i < members && flag == kFlagAggregate) {
+                        if (wait_word(sc.status + (size_t)(gfirst + i) * E + tid, tag, v[i], polls,
+                                      spin_limit)) {
+                            st_relaxed(sc.status + (size_t)(gfirst + i) * E + tid,
+                                       status_word(tag, kFlagPrefix, run));
+                            run += (uint32_t)v[i] & kValueMask;
+                        } else {
+                            raise_error(err, UE_ERR_TIMEOUT, gfirst + i);
+                            flag = kFlagError;
+                        }
+                    }
+                }
+                if (flag == kFlagError) {
+                    for (int i = 0; i < members; ++i)
+                        st_relaxed(sc.status + (size_t)(gfirst + i) * E + tid,
+                                   status_word(tag, kFlagError, 0u));
+                }
+                st_relaxed(sc.gstatus + (size_t)grp * E + tid, status_word(tag, flag, run));
+                // then the group's inclusive prefix: its sum plus the sums of the
+                // groups before it, back to the nearest group whose inclusive
+                // prefix is out (decoupled look-back over groups, each of whose
+                // words is published by a tile with a lower ticket)
+                if (flag == kFlagAggregate) {
+                    uint32_t pre = 0;
+                    int gb = grp - 1;
+                    bool done = gb < 0;
+                    while (!done) {
+                        unsigned long long w = ld_relaxed(sc.gstatus + (size_t)gb * E + tid);
+                        if (!wait_word(sc.gstatus + (size_t)gb * E + tid, tag, w, polls, spin_limit)) {
+                            raise_error(err, UE_ERR_TIMEOUT, gb);
+                            flag = kFlagError;
+                            break;
+                        }
+                        const uint32_t f = (uint32_t)w >> 30;
+                        if (f == kFlagError) {
+                            flag = kFlagError;
+                            break;
+                        }
+                        pre += (uint32_t)w & kValueMask;
+                        done = f == kFlagPrefix || --gb < 0;
+                    }
+                    st_relaxed(sc.gstatus + (size_t)grp * E + tid,
+                               status_word(tag, flag == kFlagError ? kFlagError : kFlagPrefix,
+                                           pre + run));
+                }
+            }
+            // every member has arrived: ready for the next launch
+            if (tid == 0) sc.gcount[grp] = 0u;
+        }
+    } else {
+        // ---- copy table of every expert, from the plan ----
+        const int bt = tid - kHalf;  // 0 .. kHalf - 1
+        const int bw = bt >> 5;
+        for (int x = bt; x < kMaxG / 32 * kMaxE / 4; x += kHalf)
+            reinterpret_cast<int*>(&u.pro.cntc[0][0])[x] = 0;
+        for (int e = bt; e < E; e += kHalf) u.pro.ff[e] = 1;
+        for (int x = bt; x <= P; x += kHalf) u.pro.off[x] = __ldg(plan.slot_offset + x);
+        for (int x = bt; x < P; x += kHalf) u.pro.sq[x] = __ldg(plan.slot_quota + x);
+        if (bt < G) u.pro.se[bt] = __ldg(plan.slot_expert + bt);
+        half_sync(2);
+        // slot g (one per thread: G <= kMaxG <= kHalf) takes its place among
+        // its expert's replicas (ascending g): its rank inside its chunk of 32
+        // slots (lanes holding the same expert) plus the expert's slots in
+        // the chunks below, from a per-chunk count
+        int slot_e = -1, slot_rank = 0;
+        if (bt < G) {
+            slot_e = u.pro.se[bt];
+            if (slot_e >= E) {
+                raise_error(err, UE_ERR_DEVICE_BOUNDS, bt);
+                slot_e = -1;
+            }
+        }
+        if (bw * 32 < G) {  // warp-uniform
+            const unsigned peers = same_key_lanes(slot_e, E);
+            if (slot_e >= 0) {
+                slot_rank = __popc(peers & ((1u << lane) - 1u));
+                if (slot_rank == 0) u.pro.cntc[bw][slot_e] = (unsigned char)__popc(peers);
+            }
+        }
+        half_sync(2);
+        const int nchunks = (G + 31) / 32;
+        if (slot_e >= 0)
+            for (int ch = 0; ch < bw; ++ch) slot_rank += u.pro.cntc[ch][slot_e];
+        int ncopies = 1;  // of expert bt: the master and its replicas
+        if (bt < E)
+            for (int ch = 0; ch < nchunks; ++ch) ncopies += u.pro.cntc[ch][bt];
+        int nent;  // copy-table entries: every expert's master and replicas
+        {
+            // exclusive scan of copies per expert (1 + replicas) over experts
+            const int c = bt < E ? ncopies : 0;
+            int incl = c;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(kFull, incl, off);
-            if (lane >= off) incl += o;
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(kFull, incl, off);
+                if (lane >= off) incl += o;
+            }
+            if (lane == 31) s_wsum[bw] = incl;
+            half_sync(2);
+            int wofs = 0, all = 0;
+            for (int w = 0; w < kWarps / 2; ++w) {
+                wofs += w < bw ? s_wsum[w] : 0;
+                all += s_wsum[w];
+            }
+            nent = all;
+            if (bt < E) {
+                const int e = bt;
+                const int mp = (e / M) * (M + S) + (e % M);
+                const int cb = wofs + incl - c;
+                s_c[e] = ExpC{c, cb};          // completed below
+                s_cpr[cb] = make_int2(mp, u.pro.off[mp]);  // copy 0: the master
+                s_ce[cb] = (short)e;
+            }
+            half_sync(2);
         }
-        if (lane == 31) s_wsum[warp] = incl;
-        __syncthreads();
-        int wofs = 0;
-        for (int w = 0; w < warp; ++w) wofs += s_wsum[w];
-        if (tid < nent) s_cs[tid] = wofs + incl - q;
-        if (tid == nent - 1) s_cs[nent] = wofs + incl;
-        __syncthreads();
-    }
-    if (tid < E) {
-        // the expert's load and its floor-form parameters b = floor(L/c), rem
-        const ExpC c0 = s_c[tid];
-        const int base = s_cs[c0.cb];
-        const int L = s_cs[c0.cb + c0.b] - base;
-        const unsigned b = (unsigned)L / (unsigned)c0.b;
-        u.pro.base[tid] = base;
-        s_a[tid] = ExpA{0, L, (L - (int)b * c0.b) * (int)(b + 1u), L - (int)b * c0.b};
-    }
-    __syncthreads();
-    if (tid < nent) {
-        // starts relative to the expert; quotas of the form b + [j < rem]?
-        const int e = s_ce[tid];
-        const ExpC c0 = s_c[e];
-        const int j = tid - c0.cb;
-        const int q = u.pro.sq[s_cpr[tid].x];
-        const unsigned b = (unsigned)s_a[e].L / (unsigned)c0.b;
-        if (kOrder == kOrderLocal || q != (int)b + (j < s_a[e].rem ? 1 : 0)) u.pro.ff[e] = 0;
-        s_cs[tid] -= u.pro.base[e];
-    }
-    __syncthreads();
-    if (tid < E) {
-        // the local order needs the number of copies, so it never takes the
-        // floor form
-        const ExpC c0 = s_c[tid];
-        const ExpA a = s_a[tid];
-        const bool floor_form = u.pro.ff[tid] != 0;
-        if (!floor_form) s_allff = 0;
-        const unsigned b = (unsigned)a.L / (unsigned)c0.b;
-        s_a[tid] = ExpA{0, a.L, a.thr, floor_form ? a.rem : -1};
-        s_bm[tid] = ExpB{recip64(b + 1u), recip64(b)};
-        s_c[tid] = ExpC{floor_form ? (int)b : c0.b, c0.cb};
+        if (slot_e >= 0) {
+            // the replicas after their expert's master, in ascending g
+            const int ci = s_c[slot_e].cb + 1 + slot_rank;
+            const int pp = (bt / S) * (M + S) + M + (bt % S);
+            s_cpr[ci] = make_int2(pp, u.pro.off[pp]);
+            s_ce[ci] = (short)slot_e;
+        }
+        half_sync(2);
+        {
+            // every copy's start: an exclusive scan of the quotas over the
+            // entries (experts in order, each one's copies in copy order);
+            // thread bt owns entries 2 bt and 2 bt + 1 (nent <= E + G <= 512)
+            const int e0 = 2 * bt, e1 = 2 * bt + 1;
+            const int q0 = e0 < nent ? u.pro.sq[s_cpr[e0].x] : 0;
+            const int q1 = e1 < nent ? u.pro.sq[s_cpr[e1].x] : 0;
+            const int mine = q0 + q1;
+            int incl = mine;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int o = __shfl_up_sync(kFull, incl, off);
+                if (lane >= off) incl += o;
+            }
+            if (lane == 31) s_wsum[bw] = incl;
+            half_sync(2);
+            int wofs = 0;
+            for (int w = 0; w < bw; ++w) wofs += s_wsum[w];
+            const int excl = wofs + incl - mine;
+            if (e0 < nent) s_cs[e0] = excl;
+            if (e1 < nent) s_cs[e1] = excl + q0;
+            if (e0 == nent - 1) s_cs[nent] = excl + q0;
+            if (e1 == nent - 1) s_cs[nent] = excl + mine;
+            half_sync(2);
+        }
+        if (bt < E) {
+            // the expert's load and its floor-form parameters b = floor(L/c), rem
+            const ExpC c0 = s_c[bt];
+            const int base = s_cs[c0.cb];
+            const int L = s_cs[c0.cb + c0.b] - base;
+            const unsigned b = (unsigned)L / (unsigned)c0.b;
+            u.pro.base[bt] = base;
+            s_a[bt] = ExpA{0, L, (L - (int)b * c0.b) * (int)(b + 1u), L - (int)b * c0.b};
+        }
+        half_sync(2);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int ei = 2 * bt + h;
+            if (ei < nent) {
+                // starts relative to the expert; quotas of the form b + [j < rem]?
+                const int e = s_ce[ei];
+                const ExpC c0 = s_c[e];
+                const int j = ei - c0.cb;
+                const int q = u.pro.sq[s_cpr[ei].x];
+                const unsigned b = (unsigned)s_a[e].L / (unsigned)c0.b;
+                if (kOrder == kOrderLocal || q != (int)b + (j < s_a[e].rem ? 1 : 0))
+                    u.pro.ff[e] = 0;
+                s_cs[ei] -= u.pro.base[e];
+            }
+        }
+        half_sync(2);
+        if (bt < E) {
+            // the local order needs the number of copies, so it never takes
+            // the floor form
+            const ExpC c0 = s_c[bt];
+            const ExpA a = s_a[bt];
+            const bool floor_form = u.pro.ff[bt] != 0;
+            if (!floor_form) s_allff = 0;
+            const unsigned b = (unsigned)a.L / (unsigned)c0.b;
+            s_a[bt] = ExpA{0, a.L, a.thr, floor_form ? a.rem : -1};
+            s_bm[bt] = ExpB{recip64(b + 1u), recip64(b)};
+            s_c[bt] = ExpC{floor_form ? (int)b : c0.b, c0.cb};
+        }
     }
     __syncthreads();
 
