@@ -52,6 +52,23 @@ constexpr int kThreads = kRerouteThreads;
 constexpr int kWarps = kRerouteWarps;
 constexpr int kHalf = kThreads / 2;  // threads of each half of a tile's CTA
 
+// asynchronous global -> shared copies (cp.async, no registers held) and the
+// wait for all of this thread's copies
+__device__ __forceinline__ void copy_async16(int* dst, const int32_t* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 ::"r"((unsigned)__cvta_generic_to_shared(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void copy_async4(int* dst, const int32_t* src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
+                 ::"r"((unsigned)__cvta_generic_to_shared(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void copy_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // barrier of one half of the CTA (named barriers 1 and 2; 0 is __syncthreads)
 __device__ __forceinline__ void half_sync(int id)
 {
@@ -236,7 +253,7 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
 {
     constexpr int kTileP = kThreads * kPer;    // pairs per tile
     constexpr int kPerWarpP = kTileP / kWarps;  // pairs per warp sub-range
-    extern __shared__ __align__(16) short s_idx[];  // [kTileP] expert ids of the tile (-1: none)
+    extern __shared__ __align__(16) int s_idx[];  // [kTileP] expert ids of the tile (-1: none)
     __shared__ short s_wh[kWarps][kMaxE]; // per-warp counts, then in-tile offsets
     __shared__ ExpA s_a[kMaxE];
     __shared__ ExpB s_bm[kMaxE];
@@ -293,27 +310,26 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     if (tid < kHalf) {
         // ---- stage the tile and count it per warp sub-range ----
         for (int x = tid; x < kWarps * kMaxE; x += kHalf) (&s_wh[0][0])[x] = 0;
+        // the ids go straight to shared memory (cp.async, all copies in
+        // flight at once); the count below checks them
+        if (kOrder != kOrderInterleave && (reinterpret_cast<uintptr_t>(idx) & 15u) == 0) {
+            for (int c4 = tid; c4 < kTileP / 4; c4 += kHalf) {
+                const int x = 4 * c4;
+                if (x + 4 <= cnt_tile) {
+                    copy_async16(&s_idx[x], idx + t0 + x);
+                } else {
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-            // issue all of this batch's loads before using any of them
-            int v[kPer];
-#pragma unroll
-            for (int q = 0; q < kPer; ++q) {
-                const int x = tid + (hb * kPer + q) * kHalf;
-                v[q] = x < cnt_tile ? __ldg(idx + pair_at<kOrder>(t0 + x, ord)) : -1;
-            }
-#pragma unroll
-            for (int q = 0; q < kPer; ++q) {
-                const int x = tid + (hb * kPer + q) * kHalf;
-                int e = v[q];
-                if (x < cnt_tile && (unsigned)e >= (unsigned)E) {
-                    raise_error(err, UE_ERR_DEVICE_BOUNDS,
-                                (int)min(pair_at<kOrder>(t0 + x, ord), (int64_t)INT_MAX));
-                    e = -1;
+                    for (int k = 0; k < 4; ++k)
+                        s_idx[x + k] = x + k < cnt_tile ? __ldg(idx + t0 + x + k) : -1;
                 }
-                s_idx[x] = (short)e;
+            }
+        } else {
+            for (int x = tid; x < kTileP; x += kHalf) {
+                if (x < cnt_tile) copy_async4(&s_idx[x], idx + pair_at<kOrder>(t0 + x, ord));
+                else s_idx[x] = -1;
             }
         }
+        copy_async_wait_all();
         half_sync(1);
         // warp w counts the sub-ranges of output warps 2w and 2w + 1
 #pragma unroll
@@ -321,7 +337,15 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
             const int ow = 2 * warp + sub;
 #pragma unroll 4
             for (int rd = 0; rd < kPer; ++rd) {
-                const int e = s_idx[ow * kPerWarpP + rd * 32 + lane];
+                const int x = ow * kPerWarpP + rd * 32 + lane;
+                int e = s_idx[x];
+                if (x < cnt_tile && (unsigned)e >= (unsigned)E) {
+                    // an id out of range: reported and skipped from here on
+                    raise_error(err, UE_ERR_DEVICE_BOUNDS,
+                                (int)min(pair_at<kOrder>(t0 + x, ord), (int64_t)INT_MAX));
+                    e = -1;
+                    s_idx[x] = -1;
+                }
                 if (e >= 0) atomicAdd_block(reinterpret_cast<int*>(&s_wh[ow][0]) + (e >> 1),
                                             (e & 1) ? (1 << 16) : 1);
             }
@@ -803,7 +827,7 @@ cudaError_t launch_tiles(const Sizes& z, const int32_t* idx, const ue_placement&
                          cudaStream_t st)
 {
     const int64_t tiles = (z.Q + kThreads * kPer - 1) / (kThreads * kPer);
-    reroute_kernel<kOrder, kPer><<<(unsigned)tiles, kThreads, kThreads * kPer * sizeof(short), st>>>(
+    reroute_kernel<kOrder, kPer><<<(unsigned)tiles, kThreads, kThreads * kPer * sizeof(int), st>>>(
         idx, z.Q, z.R, z.E, z.S, plan, ord, phys_slot, dest_row, sc, spin_limit, drop_first,
         err);
     return cudaGetLastError();
@@ -833,7 +857,7 @@ cudaError_t launch_order(const Sizes& z, int tile, const int32_t* idx, const ue_
 template <int kPer>
 cudaError_t allow_smem()
 {
-    const int bytes = kThreads * kPer * (int)sizeof(short);
+    const int bytes = kThreads * kPer * (int)sizeof(int);
     cudaError_t ce = cudaFuncSetAttribute(reroute_kernel<kOrderPrefix, kPer>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (ce == cudaSuccess)
@@ -850,7 +874,7 @@ int64_t tile_slots(int num_sms)
 {
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reroute_kernel<kOrderPrefix, kPer>,
-                                                      kThreads, kThreads * kPer * sizeof(short)) !=
+                                                      kThreads, kThreads * kPer * sizeof(int)) !=
         cudaSuccess) {
         cudaGetLastError();
         per_sm = 1;
