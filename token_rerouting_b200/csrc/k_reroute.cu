@@ -20,18 +20,19 @@
 // of first occurrence and row base, built by local_tables_kernel).
 //
 // Design (B200): a single-pass stable counting sort. Each CTA takes a tile
-// of 512 threads x 8 to 32 pairs by an atomic ticket (so every tile it waits
-// on is already running), stages the ids in shared memory, counts them per
-// warp sub-range and publishes its per-expert counts at once; then it
-// arrives at its group of 16 tiles. The group's last arrival, whose members
-// have all published, writes each member's exclusive prefix inside the group
-// into the member's word and the group's sum into the group's word, then
-// looks back over the groups before it (each group word is published by a
-// tile with a lower ticket) to the nearest inclusive prefix, and publishes
-// the group's inclusive prefix. A tile's exclusive prefix per expert is its
+// of 512 threads x 7 to 32 pairs by an atomic ticket (so every tile it waits
+// on is already running) and works in two halves on named barriers: warps
+// 0-7 copy the tile's ids into shared memory (cp.async), count them per warp
+// sub-range of the output phase and publish its per-expert counts at once,
+// then arrive at its group of 16 tiles; warps 8-15 meanwhile rebuild the
+// plan's copy table (at most 512 entries). The group's last arrival, whose
+// members have all published, writes each member's exclusive prefix inside
+// the group into the member's word and the group's sum into the group's
+// word, then looks back over the groups before it (each group word is
+// published by a tile with a lower ticket) to the nearest inclusive prefix,
+// and publishes the group's inclusive prefix. A tile's exclusive prefix per expert is its
 // own word plus the previous group's inclusive prefix: two loads per expert
-// once they are out, so few tiles read the same words. Meanwhile each tile
-// rebuilds the plan's copy table (at most 512 entries).
+// once they are out, so few tiles read the same words.
 // Every wait is bounded: when it runs out the waiter records UE_ERR_TIMEOUT,
 // publishes an error flag where others wait on it, and its tile writes
 // nothing. Finally each warp re-walks its pairs in order, ranking equal ids
