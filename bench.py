@@ -56,6 +56,12 @@ TRAFFIC = {
         "permute": {"bytes_per_launch": 29715613013, "source_sha": "07222823ab0e9db7"},
         "combine": {"bytes_per_launch": 33329068032, "source_sha": "c0631738399ffc37"},
     },
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum at 512 tokens
+    # per rank (8 launches each), times 4
+    "dsv3_layer_r64_e256": {
+        "permute": {"bytes_per_launch": 16669049472, "source_sha": "07222823ab0e9db7"},
+        "combine": {"bytes_per_launch": 18684903552, "source_sha": "c0631738399ffc37"},
+    },
     # ncu --set full at 512 tokens per rank, times 8
     "qwen3_layer_r64_e128": {
         "permute": {"bytes_per_launch": 18890168000, "source_sha": "07222823ab0e9db7"},
