@@ -345,8 +345,10 @@ __device__ __forceinline__ int fast_expert(int i, int lane)
 // lane holds at most three, else the three largest.
 __host__ __device__ constexpr int fast_depth(int vpl) { return vpl < 3 ? vpl : 3; }
 
-// The K+1 packed picks of one row into win[0..K]; lane 0 writes them. Each
-// lane keeps its D largest keys, sorted, and a pop shifts the list up.
+// The K+1 packed picks of one row into win[0..K]; the lane holding a pick
+// writes it (keys are distinct within a row, so exactly one lane does, and
+// the pick stays in a vector register). Each lane keeps its D largest keys,
+// sorted, and a pop shifts the list up.
 // With at most three keys a lane (D = VPL) the pop fills the bottom with 0,
 // which never wins, and every pick is exact. Otherwise the pop leaves the
 // last entry in place: a lane that gives up all D keys before the last round
@@ -357,7 +359,7 @@ __host__ __device__ constexpr int fast_depth(int vpl) { return vpl < 3 ? vpl : 3
 template <int NCH4, int NT>
 __device__ __forceinline__ void select_packed(const FastRow<NCH4, NT>& v,
                                               const uint32_t (&lo)[4 * NCH4 + NT], uint32_t khi,
-                                              uint32_t* win, bool writer)
+                                              uint32_t* win)
 {
     constexpr int VPL = 4 * NCH4 + NT;
     constexpr int D = fast_depth(VPL);
@@ -369,14 +371,14 @@ __device__ __forceinline__ void select_packed(const FastRow<NCH4, NT>& v,
 #pragma unroll
     for (int k = 0; k < kFastK; ++k) {
         const uint32_t m = __reduce_max_sync(kFull, key[0]);
-        if (writer) win[k] = m;
         const bool pop = key[0] == m;
+        if (pop) win[k] = key[0];
 #pragma unroll
         for (int j = 0; j < D - 1; ++j) key[j] = pop ? key[j + 1] : key[j];
         if constexpr (kFill) key[D - 1] = pop ? 0u : key[D - 1];
     }
     const uint32_t m = __reduce_max_sync(kFull, key[0]);
-    if (writer) win[kFastK] = m;
+    if (key[0] == m) win[kFastK] = key[0];
 }
 
 // Exact selection of one row read again from global memory: full keys,
@@ -484,7 +486,7 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_
             for (int b = 0; b < kFastRows; ++b) v[b].load(grp_rows + b * E, lane, true);
 #pragma unroll
             for (int b = 0; b < kFastRows; ++b)
-                select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0);
+                select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b]);
         } else {
             // the last group of the CTA: rows past its end read the last row
 #pragma unroll
@@ -492,7 +494,7 @@ gate_topk_fast_kernel(const float* __restrict__ logits, int64_t N, int64_t rows_
                 v[b].load(grp_rows + min(b, rows - 1) * E, lane, true);
 #pragma unroll
             for (int b = 0; b < kFastRows; ++b)
-                if (b < rows) select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b], lane == 0);
+                if (b < rows) select_packed<NCH4, NT>(v[b], lo, kHi, s_win[warp][b]);
         }
         __syncwarp();
         // rows whose leading picks agree above the dropped bits: exact again
