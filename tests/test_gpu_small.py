@@ -13,6 +13,7 @@ import torch
 
 import oracle
 import synth
+import token_rerouting_b200 as ue
 from tests import gpu_helpers as gh
 
 pytestmark = pytest.mark.gpu
@@ -129,5 +130,35 @@ def test_reroute_is_deterministic_across_launches():
             torch.cuda.synchronize()
             assert torch.equal(L.dest_row, first)
         assert L.error() == 0
+    finally:
+        L.close()
+
+
+@pytest.mark.parametrize("R,T,E,K,S", [(8, 512, 64, 4, 2), (5, 411, 40, 5, 1), (64, 37, 128, 8, 2)])
+def test_reroute_from_ids_not_16_byte_aligned(R, T, E, K, S):
+    """The reroute copies a tile's ids into shared memory with 16-byte
+    asynchronous copies when the id buffer is 16-byte aligned, and with 4-byte
+    copies otherwise. Ids at offsets of one to three int32 take the second
+    path and must give the oracle's slots and rows, as the aligned call does."""
+    wl = synth.custom(R, T, E, K, S, 8, cid=2000 + E + K, zipf_s=1.3)
+    logits = synth.logits(wl)
+    o = oracle.run_path(logits, R, T, S, K)
+    N, Q = R * T, R * T * K
+    L = gh.make_layer(R, T, E, K, S, 8, with_rows=False)
+    try:
+        gh.load_inputs(L, logits)
+        L.run_routing()
+        assert L.error() == 0
+        np.testing.assert_array_equal(L.dest_row.cpu().numpy(), o["dest_row"])
+        buf = torch.empty(Q + 3, dtype=torch.int32, device=L.device)
+        for off in (1, 2, 3):
+            ids = buf[off:off + Q].view(N, K)
+            ids.copy_(L.idx)
+            phys = torch.full_like(L.phys_slot, -7)
+            dest = torch.full_like(L.dest_row, -7)
+            ue.ue_reroute(L.ctx, ids, L.plan, phys, dest)
+            assert L.error() == 0
+            np.testing.assert_array_equal(phys.cpu().numpy(), o["phys_slot"])
+            np.testing.assert_array_equal(dest.cpu().numpy(), o["dest_row"])
     finally:
         L.close()
