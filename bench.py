@@ -463,10 +463,10 @@ def run_sweep(args):
     def run_once(st):
         L.gate_count(st)
         if opts is None:
-            L.plan_step(st)
+            L.plan_reroute(st)
         else:
             L.plan_ex(opts, st)
-        L.reroute(st)
+            L.reroute(st)
         L.permute(st)
         L.combine(stream=st)
 
@@ -866,8 +866,18 @@ def run_routing_row(args, w):
     torch.cuda.synchronize(dev)
     s = torch.cuda.Stream(dev)
     us = {}
+    def chain(stream):
+        L.gate_count(stream)
+        L.plan_step(stream)
+        L.reroute(stream)
+
+    def chain_overlap(stream):
+        L.gate_count(stream)
+        L.plan_reroute(stream)
+
     for name, f in (("gate_count", L.gate_count), ("plan", L.plan_step), ("reroute", L.reroute),
-                    ("count", L.count)):
+                    ("count", L.count), ("plan_reroute", L.plan_reroute), ("chain", chain),
+                    ("chain_overlap", chain_overlap)):
         with torch.cuda.stream(s):
             f(stream=s)
             torch.cuda.synchronize(dev)
@@ -898,6 +908,10 @@ def run_routing_row(args, w):
                                                                               "reroute")},
             "peak_kind": f"of {peak_kind}",
             "us_routing_total": us["gate_count"] + us["plan"] + us["reroute"],
+            # one routing pass as launched: gate, plan and reroute back to back
+            # (separate calls), and with plan and reroute overlapped
+            "us_routing_chain": us["chain"],
+            "us_routing_chain_overlap": us["chain_overlap"],
             "plan": {"iterations": int(plan["stats"][0]),
                      "max_over_mean_before": float(plan["stats"][1]) / (w.Q / w.R),
                      "max_over_mean_after": float(plan["stats"][2]) / (w.Q / w.R)}}
@@ -995,7 +1009,9 @@ def main():
     LB.hidden.copy_(L.hidden)
     stream = torch.cuda.current_stream(dev)
 
-    steps_fn = [L.gate_count, L.plan_step, L.reroute, L.permute, L.combine]
+    # plan and reroute in one call: the reroute kernel starts while the plan
+    # runs (programmatic dependent launch) and reads the plan once it is done
+    steps_fn = [L.gate_count, L.plan_reroute, L.permute, L.combine]
 
     def step():
         for f in steps_fn:
@@ -1023,7 +1039,7 @@ def main():
             x = i % 2
             I = insts[x]
             side.wait_event(ev_done[x])
-            for f in (I.gate_count, I.plan_step, I.reroute):
+            for f in (I.gate_count, I.plan_reroute):
                 f(stream=side)
             ev_routed[x].record(side)
             stream.wait_event(ev_routed[x])
@@ -1097,8 +1113,14 @@ def main():
     # replays of a CUDA graph of back-to-back launches on gstream (every
     # kernel is idempotent on the instance's current buffers), timed with
     # CUDA events on gstream; per launch = elapsed / launches
+    kernel_fns = dict(zip(KERNELS, (L.gate_count, L.plan_step, L.reroute, L.permute, L.combine)))
+
+    def routing_chain(stream):
+        L.gate_count(stream=stream)
+        L.plan_reroute(stream=stream)
+
     per_kernel_ms = {}
-    for name, f in zip(KERNELS, steps_fn):
+    for name, f in list(kernel_fns.items()) + [("routing_chain", routing_chain)]:
         reps = 4 if name in ("permute", "combine") else 20
         gstream.wait_stream(stream)
         with torch.cuda.stream(gstream):
@@ -1123,6 +1145,7 @@ def main():
         per_kernel_ms[name] = ka.elapsed_time(kb) / (nrep * reps)
         del kg
     clk = clocks.stop()
+    chain_ms = per_kernel_ms.pop("routing_chain")
     rc = L.error(stream)
     if rc != 0:
         raise SystemExit(f"device error in the breakdown steps: {ue.STATUS.get(rc, rc)}")
@@ -1156,8 +1179,10 @@ def main():
     gate_to_permute = sum(per_kernel_ms[k] for k in KERNELS[:4])
     cfg.update(us_per_layer_gate_to_permute=1e3 * gate_to_permute,
                us_per_layer_incl_combine=1e3 * sum(per_kernel_ms.values()),
-               timing="exactly `steps` steps, each the path's five calls (gate with the count "
-                      "fused, plan, reroute, permute, combine) over one batch; two layer "
+               us_routing_chain=1e3 * chain_ms,
+               timing="exactly `steps` steps, each the path's five kernels in four calls (gate "
+                      "with the count fused; plan and reroute, the reroute launched as the "
+                      "plan's programmatic dependent; permute; combine) over one batch; two layer "
                       "instances alternate, and step i+1's routing (gate and count, plan, reroute) "
                       "runs on a second stream during step i's permute and combine (events "
                       "order each instance's uses); per-kernel times: each kernel alone as CUDA "
@@ -1201,7 +1226,7 @@ def main():
             ev_in[b].record(s_in)
             s_run.wait_event(ev_in[b])
             s_run.wait_event(ev_out[b])          # its previous result has been read out
-            for f in [Lb.gate_count, Lb.plan_step, Lb.reroute, Lb.permute, Lb.combine]:
+            for f in [Lb.gate_count, Lb.plan_reroute, Lb.permute, Lb.combine]:
                 f(stream=s_run)
             ev_run[b].record(s_run)
             s_out.wait_event(ev_run[b])

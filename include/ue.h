@@ -237,6 +237,22 @@ ue_status ue_plan_ex(ue_ctx* ctx, const int32_t* load_e, const ue_plan_opts* opt
 ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
                      int32_t* phys_slot, int32_t* dest_row, void* stream);
 
+/* ue_plan then ue_reroute on one stream, overlapped: the reroute kernel is
+ * launched as a programmatic dependent of the plan kernel, so its tiles copy,
+ * count and look back over idx on the other SMs while the plan's single CTA
+ * runs, and read the plan only after the plan kernel has completed. The
+ * results are exactly those of ue_plan followed by ue_reroute.
+ *   load_e int32 [E] the histogram of idx (as for ue_plan).
+ *   idx, phys_slot, dest_row as for ue_reroute; plan as for both (written,
+ *   then read).
+ * idx is read while the plan kernel runs. Whatever writes it must come
+ * before this call in stream order (as ue_gate_count does); it has then
+ * completed before the plan kernel starts. Errors as for ue_plan and
+ * ue_reroute. */
+ue_status ue_plan_reroute(ue_ctx* ctx, const int32_t* load_e, const int32_t* idx,
+                          const ue_placement* plan, int32_t* phys_slot, int32_t* dest_row,
+                          void* stream);
+
 enum { UE_ORDER_PREFIX = 0, UE_ORDER_INTERLEAVE = 1 };
 
 /* ue_reroute with a choice of pair order ("UltraEP" README, "Performance

@@ -78,6 +78,7 @@ def test_calls_reject_null_context(lib):
     assert lib.ue_count(None, 16, 16, 16, None) == ue.UE_ERR_INVALID_ARG
     assert lib.ue_plan(None, 16, None, None) == ue.UE_ERR_INVALID_ARG
     assert lib.ue_reroute(None, 16, None, 16, 16, None) == ue.UE_ERR_INVALID_ARG
+    assert lib.ue_plan_reroute(None, 16, 16, None, 16, 16, None) == ue.UE_ERR_INVALID_ARG
     opts = ue.plan_opts(ue.UE_SOLVER_BISECT)
     assert lib.ue_plan_ex(None, 16, ctypes.byref(opts), None, None) == ue.UE_ERR_INVALID_ARG
     assert lib.ue_reroute_ex(None, 16, None, 1, 16, 16, None) == ue.UE_ERR_INVALID_ARG

@@ -21,8 +21,8 @@ pytestmark = pytest.mark.gpu
 
 def run_case(R, T, E, K, S, d, logits, seed=0):
     """Run the whole path on the GPU and on the oracle; compare everything
-    (the routing both through ue_gate_count and through ue_gate_topk then
-    ue_count)."""
+    (the routing both through ue_gate_count and ue_plan_reroute, and through
+    ue_gate_topk, ue_count, ue_plan and ue_reroute)."""
     N, Q = R * T, R * T * K
     hidden = synth.bf16_normal(N, d, seed, 7, R, T, E)
     y = synth.bf16_normal(Q, d, seed, 8, R, T, E)
@@ -44,8 +44,9 @@ def run_case(R, T, E, K, S, d, logits, seed=0):
                                       err_msg="dispatch rows")
         rows = y[o["dest_row"].ravel()].reshape(N, K, d)
         gh.assert_combine_close(L.out.cpu().numpy(), out_or, gh.combine_scale(rows, o["w"]))
-        # the separate gate and count calls give the same routing as the fused one
-        L.run_routing(fused=False)
+        # the separate gate, count, plan and reroute calls give the same
+        # routing as the fused and overlapped ones
+        L.run_routing(fused=False, overlap=False)
         assert L.error() == 0
         gh.assert_routing_equal(gh.routing_results(L), o)
         return g, o

@@ -67,10 +67,10 @@ def test_sweep_graph_captured(planner):
     def run_once(st):
         L.gate_count(st)
         if opts is None:
-            L.plan_step(st)
+            L.plan_reroute(st)
         else:
             L.plan_ex(opts, st)
-        L.reroute(st)
+            L.reroute(st)
         L.permute(st)
         L.combine(stream=st)
 

@@ -34,7 +34,8 @@ UE_ERR_DEVICE_BOUNDS, UE_ERR_TIMEOUT, UE_ERR_UNSUPPORTED = 4, 5, 6
 
 # every symbol include/ue.h declares
 EXPORTS = ("ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count", "ue_gate_count",
-           "ue_plan", "ue_plan_ex", "ue_reroute", "ue_reroute_ex", "ue_locality_split",
+           "ue_plan", "ue_plan_ex", "ue_reroute", "ue_plan_reroute", "ue_reroute_ex",
+           "ue_locality_split",
            "ue_reroute_local", "ue_permute", "ue_combine", "ue_combine_backward",
            "ue_permute_backward", "ue_weight_sync", "ue_grad_reduce", "ue_reroute_noalloc",
            "ue_debug_set_lookback_limit", "ue_debug_drop_first_publish")
@@ -102,6 +103,7 @@ def load_library(path: str | None = None):
     lib.ue_plan_ex.argtypes = [vp, vp, ctypes.POINTER(ue_plan_opts), ctypes.POINTER(ue_placement),
                                vp]
     lib.ue_reroute.argtypes = [vp, vp, ctypes.POINTER(ue_placement), vp, vp, vp]
+    lib.ue_plan_reroute.argtypes = [vp, vp, vp, ctypes.POINTER(ue_placement), vp, vp, vp]
     lib.ue_reroute_ex.argtypes = [vp, vp, ctypes.POINTER(ue_placement), i32, vp, vp, vp]
     lib.ue_locality_split.argtypes = [vp, vp, ctypes.POINTER(ue_placement), vp, vp, vp]
     lib.ue_reroute_local.argtypes = [vp, vp, vp, ctypes.POINTER(ue_placement), vp, vp, vp, vp,
@@ -225,6 +227,12 @@ def ue_reroute(ctx, idx, plan: ue_placement, phys_slot, dest_row, stream=None):
                                                 _stream(stream)))
 
 
+def ue_plan_reroute(ctx, load_e, idx, plan: ue_placement, phys_slot, dest_row, stream=None):
+    _ok("ue_plan_reroute",
+        load_library().ue_plan_reroute(ctx, _ptr(load_e), _ptr(idx), ctypes.byref(plan),
+                                       _ptr(phys_slot), _ptr(dest_row), _stream(stream)))
+
+
 def ue_permute(ctx, hidden, dest_row, dispatch, stream=None):
     _ok("ue_permute", load_library().ue_permute(ctx, _ptr(hidden), _ptr(dest_row),
                                                 _ptr(dispatch), _stream(stream)))
@@ -286,7 +294,7 @@ __all__ = ["ue_init", "ue_destroy", "ue_get_error", "ue_gate_topk", "ue_count", 
            "ue_plan_ex", "ue_reroute_ex", "ue_locality_split", "ue_reroute_local",
            "ue_plan_opts", "plan_opts", "UE_SOLVER_GREEDY", "UE_SOLVER_BISECT",
            "UE_ORDER_PREFIX", "UE_ORDER_INTERLEAVE",
-           "ue_reroute", "ue_permute", "ue_combine", "ue_combine_backward",
+           "ue_reroute", "ue_plan_reroute", "ue_permute", "ue_combine", "ue_combine_backward",
            "ue_permute_backward", "ue_weight_sync", "ue_grad_reduce", "ue_reroute_noalloc",
            "ue_debug_set_lookback_limit",
            "ue_debug_drop_first_publish", "ue_config", "ue_placement", "make_config",

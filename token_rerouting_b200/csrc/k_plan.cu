@@ -51,6 +51,9 @@
 // slot order. The count of co-located copies does not depend on the order of
 // placement and is taken from the final slots. The rest of the CTA writes the
 // outputs and scans the slot offsets at the end.
+// The kernel lets a dependent launch start at once (programmatic dependent
+// launch): a reroute launched that way does its plan-free part, counting its
+// tiles and looking back, on the other SMs while this one CTA runs.
 #include "ue_internal.cuh"
 
 namespace ue {
@@ -131,6 +134,9 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
     const int warp = tid >> 5;
     const int lane = tid & 31;
 
+    // a reroute launched as this kernel's programmatic dependent may start
+    // now: it counts its tiles and looks back while the plan runs
+    pdl_trigger();
     if (tid == 0) {
         sQ = 0ull;
         sUsedPicks = 0;

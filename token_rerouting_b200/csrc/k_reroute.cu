@@ -21,25 +21,32 @@
 //
 // Design (B200): a single-pass stable counting sort. Each CTA takes a tile
 // of 512 threads x 7 to 32 pairs by an atomic ticket (so every tile it waits
-// on is already running) and works in two halves on named barriers: warps
-// 0-7 copy the tile's ids into shared memory (cp.async), count them per warp
-// sub-range of the output phase and publish its per-expert counts at once,
-// then arrive at its group of 16 tiles; warps 8-15 meanwhile rebuild the
-// plan's copy table (at most 512 entries). The group's last arrival, whose
-// members have all published, writes each member's exclusive prefix inside
-// the group into the member's word and the group's sum into the group's
-// word, then looks back over the groups before it (each group word is
-// published by a tile with a lower ticket) to the nearest inclusive prefix,
-// and publishes the group's inclusive prefix. A tile's exclusive prefix per expert is its
-// own word plus the previous group's inclusive prefix: two loads per expert
-// once they are out, so few tiles read the same words.
+// on is already running). Its warps copy the tile's ids into shared memory
+// (cp.async), count them per warp sub-range of the output phase, publish the
+// tile's per-expert counts at once and arrive at its group of 16 tiles. The
+// group's last arrival, whose members have all published, writes each
+// member's exclusive prefix inside the group into the member's word and the
+// group's sum into the group's word, then looks back over the groups before
+// it (each group word is published by a tile with a lower ticket) to the
+// nearest inclusive prefix, and publishes the group's inclusive prefix.
+// Meanwhile every warp ranks each pair of its sub-range among the earlier
+// pairs of its expert (the lanes holding the same id come from eight or nine
+// ballots over the id's bits, then a running count per expert). Then, side
+// by side on named barriers, warps 0-7 find the tile's exclusive prefix per
+// expert: its own word plus the previous group's inclusive prefix, two loads
+// per expert once they are out, so few tiles read the same words; warps 8-15
+// rebuild the plan's copy table (at most 512 entries).
 // Every wait is bounded: when it runs out the waiter records UE_ERR_TIMEOUT,
 // publishes an error flag where others wait on it, and its tile writes
-// nothing. Finally each warp re-walks its pairs in order, ranking equal ids
-// within 32 lanes (the lanes holding the same id come from eight or nine
-// ballots over the id's bits), and writes the physical slot and dispatch
-// row; for floor-form quotas the copy index comes from one exact
-// multiply-high by a per-expert reciprocal, otherwise from a binary search.
+// nothing. Finally each warp takes its pairs, whose occurrence index is the
+// tile's prefix plus the pair's offset in the tile, and writes the physical
+// slot and dispatch row; for floor-form quotas the copy index comes from one
+// exact multiply-high by a per-expert reciprocal, otherwise from a binary
+// search.
+// Only the copy table and that last phase read the plan. Launched as the
+// plan kernel's programmatic dependent, the tiles copy, count, publish, rank
+// and look back while the plan runs; warps 8-15 wait for the plan to
+// complete before they read it.
 // The status words carry the launch's tag, so nothing is cleared between
 // launches: words of earlier launches read as "not yet published". The last
 // CTA to finish resets the ticket and the counter and advances the epoch;
@@ -273,6 +280,8 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         } pro;
     } u;
     __shared__ int s_wsum[kWarps];
+    __shared__ int s_pre[kMaxE];  // the tile's exclusive prefix per expert
+    __shared__ int4 s_fast[kMaxE]; // copy of each expert's first pair in the tile
     __shared__ int s_tile;
     __shared__ uint32_t s_tag;
     __shared__ int s_fail;
@@ -304,133 +313,196 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     const int gfirst = grp * kRerouteGroup;
     const int members = min(kRerouteGroup, ntiles - gfirst);
 
-    // Two halves of the CTA work side by side, each with its own barrier:
-    // warps 0-7 stage, count and publish the tile and arrive at its group;
-    // warps 8-15 rebuild the copy table from the plan, which does not depend
-    // on the tile.
-    if (tid < kHalf) {
-        // ---- stage the tile and count it per warp sub-range ----
-        for (int x = tid; x < kWarps * kMaxE; x += kHalf) (&s_wh[0][0])[x] = 0;
-        // the ids go straight to shared memory (cp.async, all copies in
-        // flight at once); the count below checks them
-        if (kOrder != kOrderInterleave && (reinterpret_cast<uintptr_t>(idx) & 15u) == 0) {
-            for (int c4 = tid; c4 < kTileP / 4; c4 += kHalf) {
-                const int x = 4 * c4;
-                if (x + 4 <= cnt_tile) {
-                    copy_async16(&s_idx[x], idx + t0 + x);
-                } else {
+    // ---- stage the tile and count it per warp sub-range (every warp) ----
+    for (int x = tid; x < kWarps * kMaxE; x += kThreads) (&s_wh[0][0])[x] = 0;
+    // the ids go straight to shared memory (cp.async, all copies in
+    // flight at once); the count below checks them
+    if (kOrder != kOrderInterleave && (reinterpret_cast<uintptr_t>(idx) & 15u) == 0) {
+        for (int c4 = tid; c4 < kTileP / 4; c4 += kThreads) {
+            const int x = 4 * c4;
+            if (x + 4 <= cnt_tile) {
+                copy_async16(&s_idx[x], idx + t0 + x);
+            } else {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        s_idx[x + k] = x + k < cnt_tile ? __ldg(idx + t0 + x + k) : -1;
-                }
-            }
-        } else {
-            for (int x = tid; x < kTileP; x += kHalf) {
-                if (x < cnt_tile) copy_async4(&s_idx[x], idx + pair_at<kOrder>(t0 + x, ord));
-                else s_idx[x] = -1;
+                for (int k = 0; k < 4; ++k)
+                    s_idx[x + k] = x + k < cnt_tile ? __ldg(idx + t0 + x + k) : -1;
             }
         }
-        copy_async_wait_all();
-        half_sync(1);
-        // warp w counts the sub-ranges of output warps 2w and 2w + 1
-#pragma unroll
-        for (int sub = 0; sub < 2; ++sub) {
-            const int ow = 2 * warp + sub;
+    } else {
+        for (int x = tid; x < kTileP; x += kThreads) {
+            if (x < cnt_tile) copy_async4(&s_idx[x], idx + pair_at<kOrder>(t0 + x, ord));
+            else s_idx[x] = -1;
+        }
+    }
+    copy_async_wait_all();
+    __syncthreads();
 #pragma unroll 4
-            for (int rd = 0; rd < kPer; ++rd) {
-                const int x = ow * kPerWarpP + rd * 32 + lane;
-                int e = s_idx[x];
-                if (x < cnt_tile && (unsigned)e >= (unsigned)E) {
-                    // an id out of range: reported and skipped from here on
-                    raise_error(err, UE_ERR_DEVICE_BOUNDS,
-                                (int)min(pair_at<kOrder>(t0 + x, ord), (int64_t)INT_MAX));
-                    e = -1;
-                    s_idx[x] = -1;
-                }
-                if (e >= 0) atomicAdd_block(reinterpret_cast<int*>(&s_wh[ow][0]) + (e >> 1),
-                                            (e & 1) ? (1 << 16) : 1);
-            }
+    for (int rd = 0; rd < kPer; ++rd) {
+        const int x = warp * kPerWarpP + rd * 32 + lane;
+        int e = s_idx[x];
+        if (x < cnt_tile && (unsigned)e >= (unsigned)E) {
+            // an id out of range: reported and skipped from here on
+            raise_error(err, UE_ERR_DEVICE_BOUNDS,
+                        (int)min(pair_at<kOrder>(t0 + x, ord), (int64_t)INT_MAX));
+            e = -1;
+            s_idx[x] = -1;
         }
-        half_sync(1);
+        if (e >= 0) atomicAdd_block(reinterpret_cast<int*>(&s_wh[warp][0]) + (e >> 1),
+                                    (e & 1) ? (1 << 16) : 1);
+    }
+    __syncthreads();
 
-        // ---- publish this tile's counts and arrive at its group ----
-        if (tid < E) {
-            int acc = 0;
-            for (int w = 0; w < kWarps; ++w) {
-                const int t = s_wh[w][tid];
-                s_wh[w][tid] = (short)acc;
-                acc += t;
-            }
-            if (!(drop_first && tile == 0))
-                st_relaxed(sc.status + (size_t)tile * E + tid,
-                           status_word(tag, kFlagAggregate, (uint32_t)acc));
+    // ---- publish this tile's counts and arrive at its group ----
+    if (tid < E) {
+        int acc = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            const int t = s_wh[w][tid];
+            s_wh[w][tid] = (short)acc;
+            acc += t;
         }
-        half_sync(1);
-        if (tid == 0)
-            s_fin = add_acq_rel(&sc.gcount[grp], 1u) == (uint32_t)(members - 1) ? 1 : 0;
-        half_sync(1);
-        if (s_fin) {
-            // the last tile of the group to arrive (its members published their
-            // counts before they arrived): each member's exclusive prefix inside
-            // the group goes into the member's own word (flag: prefix), and the
-            // group's sum into the group's word (flag: aggregate)
-            if (tid < E) {
-                unsigned long long v[kRerouteGroup];
-    #pragma unroll
-                for (int i = 0; i < kRerouteGroup; ++i)
-                    v[i] = i < members ? ld_relaxed(sc.status + (size_t)(gfirst + i) * E + tid) : 0ull;
-                uint32_t run = 0, flag = kFlagAggregate;
-                int64_t polls = 0;
-    #pragma unroll
-                for (int i = 0; i < kRerouteGroup; ++i) {
-                    if (i < members && flag == kFlagAggregate) {
-                        if (wait_word(sc.status + (size_t)(gfirst + i) * E + tid, tag, v[i], polls,
-                                      spin_limit)) {
-                            st_relaxed(sc.status + (size_t)(gfirst + i) * E + tid,
-                                       status_word(tag, kFlagPrefix, run));
-                            run += (uint32_t)v[i] & kValueMask;
-                        } else {
-                            raise_error(err, UE_ERR_TIMEOUT, gfirst + i);
-                            flag = kFlagError;
-                        }
-                    }
-                }
-                if (flag == kFlagError) {
-                    for (int i = 0; i < members; ++i)
+        if (!(drop_first && tile == 0))
+            st_relaxed(sc.status + (size_t)tile * E + tid,
+                       status_word(tag, kFlagAggregate, (uint32_t)acc));
+    }
+    __syncthreads();
+    if (tid == 0)
+        s_fin = add_acq_rel(&sc.gcount[grp], 1u) == (uint32_t)(members - 1) ? 1 : 0;
+    __syncthreads();
+    if (s_fin) {
+        // the last tile of the group to arrive (its members published their
+        // counts before they arrived): each member's exclusive prefix inside
+        // the group goes into the member's own word (flag: prefix), and the
+        // group's sum into the group's word (flag: aggregate)
+        if (tid < E) {
+            unsigned long long v[kRerouteGroup];
+#pragma unroll
+            for (int i = 0; i < kRerouteGroup; ++i)
+                v[i] = i < members ? ld_relaxed(sc.status + (size_t)(gfirst + i) * E + tid) : 0ull;
+            uint32_t run = 0, flag = kFlagAggregate;
+            int64_t polls = 0;
+#pragma unroll
+            for (int i = 0; i < kRerouteGroup; ++i) {
+                if (i < members && flag == kFlagAggregate) {
+                    if (wait_word(sc.status + (size_t)(gfirst + i) * E + tid, tag, v[i], polls,
+                                  spin_limit)) {
                         st_relaxed(sc.status + (size_t)(gfirst + i) * E + tid,
-                                   status_word(tag, kFlagError, 0u));
-                }
-                st_relaxed(sc.gstatus + (size_t)grp * E + tid, status_word(tag, flag, run));
-                // then the group's inclusive prefix: its sum plus the sums of the
-                // groups before it, back to the nearest group whose inclusive
-                // prefix is out (decoupled look-back over groups, each of whose
-                // words is published by a tile with a lower ticket)
-                if (flag == kFlagAggregate) {
-                    uint32_t pre = 0;
-                    int gb = grp - 1;
-                    bool done = gb < 0;
-                    while (!done) {
-                        unsigned long long w = ld_relaxed(sc.gstatus + (size_t)gb * E + tid);
-                        if (!wait_word(sc.gstatus + (size_t)gb * E + tid, tag, w, polls, spin_limit)) {
-                            raise_error(err, UE_ERR_TIMEOUT, gb);
-                            flag = kFlagError;
-                            break;
-                        }
-                        const uint32_t f = (uint32_t)w >> 30;
-                        if (f == kFlagError) {
-                            flag = kFlagError;
-                            break;
-                        }
-                        pre += (uint32_t)w & kValueMask;
-                        done = f == kFlagPrefix || --gb < 0;
+                                   status_word(tag, kFlagPrefix, run));
+                        run += (uint32_t)v[i] & kValueMask;
+                    } else {
+                        raise_error(err, UE_ERR_TIMEOUT, gfirst + i);
+                        flag = kFlagError;
                     }
-                    st_relaxed(sc.gstatus + (size_t)grp * E + tid,
-                               status_word(tag, flag == kFlagError ? kFlagError : kFlagPrefix,
-                                           pre + run));
                 }
             }
-            // every member has arrived: ready for the next launch
-            if (tid == 0) sc.gcount[grp] = 0u;
+            if (flag == kFlagError) {
+                for (int i = 0; i < members; ++i)
+                    st_relaxed(sc.status + (size_t)(gfirst + i) * E + tid,
+                               status_word(tag, kFlagError, 0u));
+            }
+            st_relaxed(sc.gstatus + (size_t)grp * E + tid, status_word(tag, flag, run));
+            // then the group's inclusive prefix: its sum plus the sums of the
+            // groups before it, back to the nearest group whose inclusive
+            // prefix is out (decoupled look-back over groups, each of whose
+            // words is published by a tile with a lower ticket)
+            if (flag == kFlagAggregate) {
+                uint32_t pre = 0;
+                int gb = grp - 1;
+                bool done = gb < 0;
+                while (!done) {
+                    unsigned long long w = ld_relaxed(sc.gstatus + (size_t)gb * E + tid);
+                    if (!wait_word(sc.gstatus + (size_t)gb * E + tid, tag, w, polls, spin_limit)) {
+                        raise_error(err, UE_ERR_TIMEOUT, gb);
+                        flag = kFlagError;
+                        break;
+                    }
+                    const uint32_t f = (uint32_t)w >> 30;
+                    if (f == kFlagError) {
+                        flag = kFlagError;
+                        break;
+                    }
+                    pre += (uint32_t)w & kValueMask;
+                    done = f == kFlagPrefix || --gb < 0;
+                }
+                st_relaxed(sc.gstatus + (size_t)grp * E + tid,
+                           status_word(tag, flag == kFlagError ? kFlagError : kFlagPrefix,
+                                       pre + run));
+            }
+        }
+        // every member has arrived: ready for the next launch
+        if (tid == 0) sc.gcount[grp] = 0u;
+    }
+
+    // ---- in-tile ranks ----
+    // each warp ranks its own sub-range: a pair's offset in the tile among
+    // the pairs of its expert is the sub-range's offset plus the pairs of
+    // that expert before it in the sub-range (the lanes holding the same id,
+    // then a running count per expert); it replaces the id in shared memory
+    // as (offset << 8) | id. The ranks depend on the ids alone, so they are
+    // ready before the plan is read.
+    {
+        const unsigned lt = (1u << lane) - 1u;
+#pragma unroll 2
+        for (int rd = 0; rd < kPer; ++rd) {
+            const int x = warp * kPerWarpP + rd * 32 + lane;
+            const int e = s_idx[x];
+            const unsigned peers = same_key_lanes(e, E);
+            const int below = __popc(peers & lt);
+            const int ev = e < 0 ? 0 : e;
+            const int run = s_wh[warp][ev];
+            s_idx[x] = e < 0 ? -1 : (((run + below) << 8) | e);
+            __syncwarp();
+            // the lowest lane of each expert's group moves its count on
+            if (e >= 0 && below == 0) s_wh[warp][ev] = (short)(run + __popc(peers));
+            __syncwarp();
+        }
+    }
+
+    // Two halves of the CTA work side by side: warps 0-7 look back for the
+    // tile's exclusive prefix per expert; warps 8-15 rebuild the copy table
+    // from the plan, with their own barrier.
+    if (tid < kHalf) {
+        // ---- look back: this tile's exclusive prefix per expert ----
+        // the tile's own word (its exclusive prefix inside its group, put there
+        // by the group's last arrival) plus the inclusive prefix of the group
+        // before (or, while that is not out yet, the sums of the groups before,
+        // back to the nearest inclusive prefix)
+        if (tid < E) {
+            uint32_t excl = 0;
+            bool fail = false;
+            int64_t polls = 0;
+            const unsigned long long* own = sc.status + (size_t)tile * E + tid;
+            unsigned long long w = ld_relaxed(own);
+            // wait for the prefix flag (the tile's own count is there first)
+            while (!fail && ((uint32_t)(w >> 32) != tag || ((uint32_t)w >> 30) == kFlagInvalid ||
+                             ((uint32_t)w >> 30) == kFlagAggregate)) {
+                if (++polls > spin_limit) {
+                    raise_error(err, UE_ERR_TIMEOUT, tile);
+                    fail = true;
+                } else {
+                    __nanosleep(64);
+                    w = ld_relaxed(own);
+                }
+            }
+            if (!fail && ((uint32_t)w >> 30) == kFlagError) fail = true;
+            excl = (uint32_t)w & kValueMask;
+            int gb = grp - 1;
+            while (!fail && gb >= 0) {
+                unsigned long long gw = ld_relaxed(sc.gstatus + (size_t)gb * E + tid);
+                if (!wait_word(sc.gstatus + (size_t)gb * E + tid, tag, gw, polls, spin_limit)) {
+                    raise_error(err, UE_ERR_TIMEOUT, tile);
+                    fail = true;
+                    break;
+                }
+                const uint32_t f = (uint32_t)gw >> 30;
+                if (f == kFlagError) {
+                    fail = true;
+                    break;
+                }
+                excl += (uint32_t)gw & kValueMask;
+                gb = f == kFlagPrefix ? -1 : gb - 1;
+            }
+            if (fail) s_fail = 1;
+            s_pre[tid] = (int)excl;
         }
     } else {
         // ---- copy table of every expert, from the plan ----
@@ -439,9 +511,13 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         for (int x = bt; x < kMaxG / 32 * kMaxE / 4; x += kHalf)
             reinterpret_cast<int*>(&u.pro.cntc[0][0])[x] = 0;
         for (int e = bt; e < E; e += kHalf) u.pro.ff[e] = 1;
-        for (int x = bt; x <= P; x += kHalf) u.pro.off[x] = __ldg(plan.slot_offset + x);
-        for (int x = bt; x < P; x += kHalf) u.pro.sq[x] = __ldg(plan.slot_quota + x);
-        if (bt < G) u.pro.se[bt] = __ldg(plan.slot_expert + bt);
+        // launched after the plan kernel as its dependent, the tile gets
+        // here while the plan may still run: wait for it to complete, then
+        // read the plan through L2
+        pdl_wait();
+        for (int x = bt; x <= P; x += kHalf) u.pro.off[x] = __ldcg(plan.slot_offset + x);
+        for (int x = bt; x < P; x += kHalf) u.pro.sq[x] = __ldcg(plan.slot_quota + x);
+        if (bt < G) u.pro.se[bt] = __ldcg(plan.slot_expert + bt);
         half_sync(2);
         // slot g (one per thread: G <= kMaxG <= kHalf) takes its place among
         // its expert's replicas (ascending g): its rank inside its chunk of 32
@@ -570,49 +646,31 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
         }
     }
     __syncthreads();
-
-    // ---- look back: this tile's exclusive prefix per expert ----
-    // the tile's own word (its exclusive prefix inside its group, put there
-    // by the group's last arrival) plus the inclusive prefix of the group
-    // before (or, while that is not out yet, the sums of the groups before,
-    // back to the nearest inclusive prefix)
+    const bool lean = kOrder != kOrderLocal && s_allff;
     if (tid < E) {
-        uint32_t excl = 0;
-        bool fail = false;
-        int64_t polls = 0;
-        const unsigned long long* own = sc.status + (size_t)tile * E + tid;
-        unsigned long long w = ld_relaxed(own);
-        // wait for the prefix flag (the tile's own count is there first)
-        while (!fail && ((uint32_t)(w >> 32) != tag || ((uint32_t)w >> 30) == kFlagInvalid ||
-                         ((uint32_t)w >> 30) == kFlagAggregate)) {
-            if (++polls > spin_limit) {
-                raise_error(err, UE_ERR_TIMEOUT, tile);
-                fail = true;
-            } else {
-                __nanosleep(64);
-                w = ld_relaxed(own);
+        const int pre = s_pre[tid];
+        s_a[tid].pre = pre;
+        if (lean) {
+            // the copy holding the tile's first pair of this expert (its
+            // occurrence index is pre): the expert's pairs of the tile at
+            // in-tile offsets below `lim` all fall in it, at row row0 + offset
+            const ExpA a = s_a[tid];
+            const ExpC c = s_c[tid];
+            const ExpB bm = s_bm[tid];
+            int4 f = make_int4(-1, 0, 0, 0);  // (slot, row0, lim, -)
+            if (pre < a.L) {
+                const bool big = pre < a.thr;
+                const unsigned d = big ? (unsigned)c.b + 1u : (unsigned)c.b;
+                const unsigned x0 = big ? (unsigned)pre : (unsigned)(pre - a.thr);
+                const unsigned q = div_m32(x0, d, big ? bm.m1 : bm.m0);
+                const int j = big ? (int)q : a.rem + (int)q;
+                const int start = j * c.b + min(j, a.rem);
+                const int2 cr = s_cpr[c.cb + j];
+                const int quota = c.b + (j < a.rem ? 1 : 0);
+                f = make_int4(cr.x, cr.y + (pre - start), start + quota - pre, 0);
             }
+            s_fast[tid] = f;
         }
-        if (!fail && ((uint32_t)w >> 30) == kFlagError) fail = true;
-        excl = (uint32_t)w & kValueMask;
-        int gb = grp - 1;
-        while (!fail && gb >= 0) {
-            unsigned long long gw = ld_relaxed(sc.gstatus + (size_t)gb * E + tid);
-            if (!wait_word(sc.gstatus + (size_t)gb * E + tid, tag, gw, polls, spin_limit)) {
-                raise_error(err, UE_ERR_TIMEOUT, tile);
-                fail = true;
-                break;
-            }
-            const uint32_t f = (uint32_t)gw >> 30;
-            if (f == kFlagError) {
-                fail = true;
-                break;
-            }
-            excl += (uint32_t)gw & kValueMask;
-            gb = f == kFlagPrefix ? -1 : gb - 1;
-        }
-        if (fail) s_fail = 1;
-        s_a[tid].pre = (int)excl;
     }
     __syncthreads();
     const bool write_out = !s_fail;
@@ -621,43 +679,46 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     // the o-th pair of expert e: with floor-form quotas, copy j = o / (b+1)
     // while o < rem*(b+1), else rem + (o - rem*(b+1)) / b; otherwise the
     // last copy whose start is <= o. Row = first row of the copy + (o - start).
-    const unsigned lt = (1u << lane) - 1u;
-    if (kOrder != kOrderLocal && s_allff) {
-        // every expert has floor-form quotas: no per-round vote. A pair
-        // beyond its expert's load (ids that do not match the plan) is
-        // reported, and its rank is clamped so that the table reads stay
-        // inside the expert's copies.
+    if (lean) {
+        // every expert has floor-form quotas: most pairs take the copy of
+        // their expert's first pair in the tile from one record; the others
+        // (past that copy's end) find theirs by the division. A pair beyond
+        // its expert's load (ids that do not match the plan) is reported,
+        // and its rank is clamped so that the table reads stay inside the
+        // expert's copies.
         const unsigned t0u = (unsigned)t0;
 #pragma unroll 2
         for (int rd = 0; rd < (write_out ? kPer : 0); ++rd) {
             const int x = warp * kPerWarpP + rd * 32 + lane;
-            const int ex = s_idx[x];
-            const unsigned peers = same_key_lanes(ex, E);
-            const unsigned below = __popc(peers & lt);
+            const int v = s_idx[x];
+            const int ex = v < 0 ? -1 : (v & 255);
+            const int lo = v < 0 ? 0 : v >> 8;
             const int ev = ex < 0 ? 0 : ex;
             const unsigned i = pair_at32<kOrder>(t0u + (unsigned)x, ord);
-            const int base = s_wh[warp][ev];
-            const ExpA a = s_a[ev];
-            const ExpC c = s_c[ev];
-            const ExpB bm = s_bm[ev];
-            const int o = a.pre + base + (int)below;
-            const int oc = min(o, max(a.L - 1, 0));
-            const bool big = oc < a.thr;
-            const unsigned d = big ? (unsigned)c.b + 1u : (unsigned)c.b;
-            const unsigned x0 = big ? (unsigned)oc : (unsigned)(oc - a.thr);
-            const unsigned q = div_m32(x0, d, big ? bm.m1 : bm.m0);
-            const int j = big ? (int)q : a.rem + (int)q;
-            const int start = j * c.b + min(j, a.rem);
-            const int2 cr = s_cpr[c.cb + j];
-            int p = cr.x, row = cr.y + (oc - start);
-            if (ex < 0 || o >= a.L) {
-                if (ex >= 0) raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(i, (unsigned)INT_MAX));
-                p = -1;
-                row = -1;
+            const int4 f = s_fast[ev];
+            int p = f.x, row = f.y + lo;
+            if (ex < 0 || lo >= f.z) {
+                const ExpA a = s_a[ev];
+                const ExpC c = s_c[ev];
+                const ExpB bm = s_bm[ev];
+                const int o = a.pre + lo;
+                const int oc = min(o, max(a.L - 1, 0));
+                const bool big = oc < a.thr;
+                const unsigned d = big ? (unsigned)c.b + 1u : (unsigned)c.b;
+                const unsigned x0 = big ? (unsigned)oc : (unsigned)(oc - a.thr);
+                const unsigned q = div_m32(x0, d, big ? bm.m1 : bm.m0);
+                const int j = big ? (int)q : a.rem + (int)q;
+                const int start = j * c.b + min(j, a.rem);
+                const int2 cr = s_cpr[c.cb + j];
+                p = cr.x;
+                row = cr.y + (oc - start);
+                if (ex < 0 || o >= a.L) {
+                    if (ex >= 0)
+                        raise_error(err, UE_ERR_DEVICE_BOUNDS, (int)min(i, (unsigned)INT_MAX));
+                    p = -1;
+                    row = -1;
+                }
             }
-            __syncwarp();
-            if (ex >= 0 && below == 0u) s_wh[warp][ev] = (short)(base + (int)__popc(peers));
-            __syncwarp();
             if (x < cnt_tile) {
                 phys_slot[i] = p;
                 dest_row[i] = row;
@@ -667,15 +728,13 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
 #pragma unroll 2
         for (int rd = 0; rd < (write_out ? kPer : 0); ++rd) {
             const int x = warp * kPerWarpP + rd * 32 + lane;
-            const int ex = s_idx[x];
-            const unsigned peers = same_key_lanes(ex, E);
-            const unsigned below = __popc(peers & lt);  // same expert, lower lanes
+            const int v = s_idx[x];
+            const int ex = v < 0 ? -1 : (v & 255);
             const int ev = ex < 0 ? 0 : ex;             // a safe index for the loads
             const int64_t i = pair_at<kOrder>(t0 + x, ord);
-            const int base = s_wh[warp][ev];
             const ExpA a = s_a[ev];
             const ExpC c = s_c[ev];
-            const int o = a.pre + base + (int)below;
+            const int o = a.pre + (v < 0 ? 0 : v >> 8);
             int p = -1, row = -1;
             if (kOrder != kOrderLocal && __all_sync(kFull, ex < 0 || (a.rem >= 0 && o < a.L))) {
                 // every lane of the round has floor-form quotas: no branches
@@ -727,10 +786,6 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
                     row = s_cpr[ci].y + (o - s_cs[ci]);
                 }
             }
-            __syncwarp();
-            // the lowest lane of each expert's group moves the warp's count on
-            if (ex >= 0 && below == 0u) s_wh[warp][ev] = (short)(base + (int)__popc(peers));
-            __syncwarp();
             if (x < cnt_tile) {
                 phys_slot[i] = p;
                 dest_row[i] = row;
@@ -825,13 +880,21 @@ template <int kOrder, int kPer>
 cudaError_t launch_tiles(const Sizes& z, const int32_t* idx, const ue_placement& plan,
                          const OrderArgs& ord, int32_t* phys_slot, int32_t* dest_row,
                          const RerouteScratch& sc, int64_t spin_limit, int drop_first, int* err,
-                         cudaStream_t st)
+                         cudaStream_t st, bool pdl)
 {
     const int64_t tiles = (z.Q + kThreads * kPer - 1) / (kThreads * kPer);
-    reroute_kernel<kOrder, kPer><<<(unsigned)tiles, kThreads, kThreads * kPer * sizeof(int), st>>>(
-        idx, z.Q, z.R, z.E, z.S, plan, ord, phys_slot, dest_row, sc, spin_limit, drop_first,
-        err);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)tiles);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kThreads * kPer * sizeof(int);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, reroute_kernel<kOrder, kPer>, idx, z.Q, z.R, z.E, z.S, plan,
+                              ord, phys_slot, dest_row, sc, spin_limit, drop_first, err);
 }
 
 // pairs per thread of the tile sizes on offer (tile = 512 * kPer)
@@ -841,13 +904,13 @@ template <int kOrder>
 cudaError_t launch_order(const Sizes& z, int tile, const int32_t* idx, const ue_placement& plan,
                          const OrderArgs& ord, int32_t* phys_slot, int32_t* dest_row,
                          const RerouteScratch& sc, int64_t spin_limit, int drop_first, int* err,
-                         cudaStream_t st)
+                         cudaStream_t st, bool pdl)
 {
     switch (tile) {
 #define UE_CASE(P)                                                                          \
     case kThreads * P:                                                                      \
         return launch_tiles<kOrder, P>(z, idx, plan, ord, phys_slot, dest_row, sc,          \
-                                       spin_limit, drop_first, err, st);
+                                       spin_limit, drop_first, err, st, pdl);
         UE_REROUTE_PER(UE_CASE)
 #undef UE_CASE
     default:
@@ -918,15 +981,15 @@ cudaError_t launch_reroute(const Sizes& z, int tile, const int32_t* idx,
 cudaError_t launch_reroute_order(const Sizes& z, int tile, const int32_t* idx,
                                  const ue_placement& plan, int order, int32_t* phys_slot,
                                  int32_t* dest_row, const RerouteScratch& sc, int64_t spin_limit,
-                                 int drop_first, int* err, cudaStream_t st)
+                                 int drop_first, int* err, cudaStream_t st, bool after_plan)
 {
     if (z.Q == 0) return cudaSuccess;
     const OrderArgs ord = make_order(z);
     if (order == kOrderInterleave)
         return launch_order<kOrderInterleave>(z, tile, idx, plan, ord, phys_slot, dest_row, sc,
-                                              spin_limit, drop_first, err, st);
+                                              spin_limit, drop_first, err, st, after_plan);
     return launch_order<kOrderPrefix>(z, tile, idx, plan, ord, phys_slot, dest_row, sc,
-                                      spin_limit, drop_first, err, st);
+                                      spin_limit, drop_first, err, st, after_plan);
 }
 
 cudaError_t launch_reroute_local(const Sizes& z, int tile, const int32_t* idx,
@@ -946,7 +1009,7 @@ cudaError_t launch_reroute_local(const Sizes& z, int tile, const int32_t* idx,
     ord.rowb = rowb;
     ord.quota = src_quota;
     return launch_order<kOrderLocal>(z, tile, idx, plan, ord, phys_slot, dest_row, sc,
-                                     spin_limit, drop_first, err, st);
+                                     spin_limit, drop_first, err, st, false);
 }
 
 }  // namespace ue

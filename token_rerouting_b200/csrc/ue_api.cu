@@ -260,6 +260,23 @@ ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
                                         ctx->d_err, as_stream(stream)));
 }
 
+ue_status ue_plan_reroute(ue_ctx* ctx, const int32_t* load_e, const int32_t* idx,
+                          const ue_placement* plan, int32_t* phys_slot, int32_t* dest_row,
+                          void* stream)
+{
+    if (!ctx_ok(ctx) || !aligned(load_e, 4) || !aligned(idx, 4) || !placement_ok(ctx, plan) ||
+        !aligned(phys_slot, 4) || !aligned(dest_row, 4))
+        return UE_ERR_INVALID_ARG;
+    if (use_device(ctx) != UE_OK) return UE_ERR_CUDA;
+    const cudaStream_t st = as_stream(stream);
+    const cudaError_t ce = ue::launch_plan(ctx->z, load_e, 0, *plan, ctx->d_err, st);
+    if (ce != cudaSuccess) return from_cuda(ce);
+    return from_cuda(ue::launch_reroute_order(ctx->z, ctx->rtile, idx, *plan, UE_ORDER_PREFIX,
+                                              phys_slot, dest_row, rscratch(ctx),
+                                              ctx->spin_limit, ctx->drop_first, ctx->d_err, st,
+                                              true));
+}
+
 ue_status ue_reroute_ex(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan, int32_t order,
                         int32_t* phys_slot, int32_t* dest_row, void* stream)
 {

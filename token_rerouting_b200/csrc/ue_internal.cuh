@@ -33,6 +33,21 @@ __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v)
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start once the kernel before it in the stream has run
+// pdl_trigger() in every CTA (or exited); pdl_wait() then blocks the calling
+// thread until that kernel has completed and its writes are visible. Both
+// are no-ops for kernels launched the ordinary way.
+__device__ __forceinline__ void pdl_trigger()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 constexpr int kWarp = 32;
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -156,11 +171,16 @@ cudaError_t launch_reroute(const Sizes& z, int tile, const int32_t* idx,
                            const ue_placement& plan, int32_t* phys_slot, int32_t* dest_row,
                            const RerouteScratch& sc, int64_t spin_limit, int drop_first, int* err,
                            cudaStream_t st);
-// order: 0 global (r, t, k), 1 interleaved (t, r, k)
+// order: 0 global (r, t, k), 1 interleaved (t, r, k). after_plan: launched
+// as a programmatic dependent of the plan kernel just before it in the
+// stream, so that the tiles count and look back while the plan runs and read
+// the plan only once it has completed (the kernel before the plan must have
+// completed ordinarily: the ids are read early).
 cudaError_t launch_reroute_order(const Sizes& z, int tile, const int32_t* idx,
                                  const ue_placement& plan, int order, int32_t* phys_slot,
                                  int32_t* dest_row, const RerouteScratch& sc, int64_t spin_limit,
-                                 int drop_first, int* err, cudaStream_t st);
+                                 int drop_first, int* err, cudaStream_t st,
+                                 bool after_plan = false);
 // locality order: builds the [R][P] tables `first` and `rowb`, then reroutes
 cudaError_t launch_reroute_local(const Sizes& z, int tile, const int32_t* idx,
                                  const int32_t* load_re, const ue_placement& plan,

@@ -12,7 +12,7 @@ from __future__ import annotations
 from . import (make_config, placement, ue_combine, ue_count, ue_destroy, ue_gate_count,
                ue_gate_topk,
                ue_get_error, ue_init, ue_locality_split, ue_permute, ue_plan, ue_plan_ex,
-               ue_reroute, ue_reroute_ex, ue_reroute_local)
+               ue_plan_reroute, ue_reroute, ue_reroute_ex, ue_reroute_local)
 
 
 class Layer:
@@ -72,6 +72,12 @@ class Layer:
     def reroute(self, stream=None):
         ue_reroute(self.ctx, self.idx, self.plan, self.phys_slot, self.dest_row, stream)
 
+    def plan_reroute(self, stream=None):
+        """Plan then reroute in one call, the reroute's plan-free part
+        overlapping the plan kernel (ue_plan_reroute)."""
+        ue_plan_reroute(self.ctx, self.load_e, self.idx, self.plan, self.phys_slot,
+                        self.dest_row, stream)
+
     # -- planner variants ("Performance Tuning / Replication planning") -----
     def plan_ex(self, opts, stream=None):
         """ue_plan_ex with a ue_plan_opts (see token_rerouting_b200.plan_opts)."""
@@ -95,16 +101,20 @@ class Layer:
         ue_combine(self.ctx, self.dispatch if y is None else y, self.dest_row, self.w,
                    self.out, stream)
 
-    def run_routing(self, stream=None, fused=True):
+    def run_routing(self, stream=None, fused=True, overlap=True):
         """gate -> count -> plan -> reroute; with fused=True the gate and the
-        count are one call (ue_gate_count)."""
+        count are one call (ue_gate_count), with overlap=True the plan and
+        the reroute are one call (ue_plan_reroute)."""
         if fused:
             self.gate_count(stream)
         else:
             self.gate(stream)
             self.count(stream)
-        self.plan_step(stream)
-        self.reroute(stream)
+        if overlap:
+            self.plan_reroute(stream)
+        else:
+            self.plan_step(stream)
+            self.reroute(stream)
 
     def run(self, y=None, stream=None):
         """The whole path: gate -> count -> plan -> reroute -> permute ->
