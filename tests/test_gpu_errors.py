@@ -138,3 +138,26 @@ def test_variant_calls_reject_bad_arguments(layer):
         ue.ue_reroute_local(layer.ctx, layer.idx, layer.load_re, layer.plan, layer.src_quota,
                             layer.src_offset, layer.phys_slot, layer.dest_row.data_ptr() + 1)
     assert layer.error() == ue.UE_OK
+
+
+def test_overlapped_plan_and_reroute_report_errors_and_recover(layer):
+    """ue_plan_reroute (the reroute launched as the plan kernel's dependent):
+    a look-back wait that runs out and an id out of range are reported as
+    by the separate calls, and the context then runs clean."""
+    w = synth.custom(R, T, E, K, S, d, cid=505)
+    logits = synth.logits(w)
+    gh.load_inputs(layer, logits)
+    layer.run_routing()
+    assert layer.error() == ue.UE_OK
+    ue.ue_debug_set_lookback_limit(layer.ctx, 1000)
+    ue.ue_debug_drop_first_publish(layer.ctx, True)
+    layer.plan_reroute()
+    assert layer.error() == ue.UE_ERR_TIMEOUT
+    ue.ue_debug_drop_first_publish(layer.ctx, False)
+    ue.ue_debug_set_lookback_limit(layer.ctx, 1 << 22)
+    check_clean_run(layer, logits)
+    layer.idx[5, 3] = E + 1
+    layer.plan_reroute()
+    assert layer.error() == ue.UE_ERR_DEVICE_BOUNDS
+    assert int(layer.dest_row[5, 3]) == -1 and int(layer.phys_slot[5, 3]) == -1
+    check_clean_run(layer, logits)

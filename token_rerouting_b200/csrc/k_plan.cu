@@ -44,7 +44,7 @@
 // l owns ranks l, l+32, ... and their slots, so every load change lands in
 // the lane that owns the rank). Per iteration: the stop test as a vote (is
 // any load above floor(51 Q / (50 R))?) and the least loaded rank with a free
-// slot as one `redux` min of (load << 7 | r) when Q < 2^25 (three reductions
+// slot as one `redux` min of (load << 7 | r) when Q < 2^25 (two reductions
 // otherwise), the placement in r*'s lowest free slot, and the new quotas of
 // e*'s copies: the master's goes from ceil(L/(c-1)) to ceil(L/c); a first
 // replica takes floor(L/2); later replicas are found by ballots in ascending
@@ -291,32 +291,34 @@ plan_kernel(const int32_t* __restrict__ load_e, int R, int E, int S, unsigned mi
             // reductions (iters + 1 <= G always: the loop stops once every
             // slot is used)
             const Pick pk_next = sPick[min(iters + 1, kMaxG)];
-            unsigned maxl = 0u, bestl = 0xffffffffu, bestr = 0xffffffffu;
+            // the stop test as a vote: is any load above stop_max?
+            bool over = false;
+            unsigned bestl = 0xffffffffu, bestr = 0xffffffffu;
             int rstar;
             if (packed) {
                 unsigned key = 0xffffffffu;
 #pragma unroll
                 for (int j = 0; j < NJR; ++j) {
-                    maxl = max(maxl, load[j]);
+                    over = over || load[j] > stop_max;
                     if (used[j] < S) key = min(key, (load[j] << 7) | (unsigned)(lane + 32 * j));
                 }
-                maxl = __reduce_max_sync(kFull, maxl);
+                const bool any_over = __any_sync(kFull, over);
                 key = __reduce_min_sync(kFull, key);
-                if (maxl <= stop_max) break;
+                if (!any_over) break;
                 if (key == 0xffffffffu) break;  // no free slot anywhere
                 rstar = (int)(key & 127u);
             } else {
 #pragma unroll
                 for (int j = 0; j < NJR; ++j) {
-                    maxl = max(maxl, load[j]);
+                    over = over || load[j] > stop_max;
                     if (used[j] < S && load[j] < bestl) {
                         bestl = load[j];
                         bestr = (unsigned)(lane + 32 * j);
                     }
                 }
-                maxl = __reduce_max_sync(kFull, maxl);
+                const bool any_over = __any_sync(kFull, over);
                 const unsigned ml = __reduce_min_sync(kFull, bestl);
-                if (maxl <= stop_max) break;
+                if (!any_over) break;
                 if (ml == 0xffffffffu) break;  // no free slot anywhere
                 rstar = (int)__reduce_min_sync(kFull, bestl == ml ? bestr : 0xffffffffu);
             }
