@@ -310,7 +310,6 @@ __device__ __forceinline__ void top_desc(uint32_t (&k)[VPL])
 
 template <int NCH4, int NT>
 struct FastRow {
-    static constexpr int VPL = 4 * NCH4 + NT;
     float4 c4[NCH4 > 0 ? NCH4 : 1];
     float t1[NT > 0 ? NT : 1];
 
