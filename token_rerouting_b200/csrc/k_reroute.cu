@@ -77,7 +77,8 @@ __device__ __forceinline__ void copy_async_wait_all()
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// barrier of one half of the CTA (named barriers 1 and 2; 0 is __syncthreads)
+// barrier of one half of the CTA (a named barrier other than 0, which
+// __syncthreads uses)
 __device__ __forceinline__ void half_sync(int id)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kHalf) : "memory");
