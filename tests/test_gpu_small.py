@@ -163,3 +163,23 @@ def test_reroute_from_ids_not_16_byte_aligned(R, T, E, K, S):
             np.testing.assert_array_equal(dest.cpu().numpy(), o["dest_row"])
     finally:
         L.close()
+
+
+@pytest.mark.parametrize("R,T,E,K,S,seed", [(3, 1, 6, 1, 2, 0), (4, 1, 8, 1, 4, 3),
+                                            (5, 1, 10, 1, 3, 0)])
+def test_replicas_with_zero_quota(R, T, E, K, S, seed):
+    """A layout the greedy cannot balance (the master of a hot expert shares
+    its rank with another master that keeps the remainder) goes on placing
+    copies until the slots run out: experts end with more copies than pairs,
+    so some copies get a quota of 0 (floor(L/c) = 0). The reroute's record of
+    each expert's first copy in the tile and its division path must skip
+    those copies as the oracle does."""
+    rng = np.random.default_rng(seed)
+    logits = rng.normal(size=(R * T, E)).astype(np.float32)
+    logits[:, 0] += 4.0
+    logits[:, 1] += 2.0
+    o = oracle.run_path(logits, R, T, S, K)
+    L = o["load_e"]
+    nc = np.asarray(o["plan"].n_copies)
+    assert ((nc > L) & (L > 0)).any()
+    run_case(R, T, E, K, S, 8, logits)
