@@ -851,7 +851,9 @@ def run_routing_row(args, w):
     a small device footprint, for kernel captures). Each call timed alone as
     replays of a CUDA graph of back-to-back launches, CUDA events on the
     replay stream. The separate count call (ue_count, the same counts from
-    idx) is timed beside them but not part of the routing total."""
+    idx) is timed beside them but not part of the routing total. Also timed
+    the same way: the plan and the reroute overlapped (ue_plan_reroute), and
+    the whole routing chain as launched, with and without that overlap."""
     import torch
 
     import token_rerouting_b200 as ue
