@@ -40,9 +40,10 @@
 // publishes an error flag where others wait on it, and its tile writes
 // nothing. Finally each warp takes its pairs, whose occurrence index is the
 // tile's prefix plus the pair's offset in the tile, and writes the physical
-// slot and dispatch row; for floor-form quotas the copy index comes from one
-// exact multiply-high by a per-expert reciprocal, otherwise from a binary
-// search.
+// slot and dispatch row. Per expert the tile keeps the copy that holds its
+// first pair of that expert; most pairs fall in it. The others find their
+// copy by one exact multiply-high by a per-expert reciprocal for floor-form
+// quotas, otherwise by a binary search over the copy starts.
 // Only the copy table and that last phase read the plan. Launched as the
 // plan kernel's programmatic dependent, the tiles copy, count, publish, rank
 // and look back while the plan runs; warps 8-15 wait for the plan to
@@ -651,24 +652,33 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
     if (tid < E) {
         const int pre = s_pre[tid];
         s_a[tid].pre = pre;
-        if (lean) {
+        if (kOrder != kOrderLocal) {
             // the copy holding the tile's first pair of this expert (its
             // occurrence index is pre): the expert's pairs of the tile at
             // in-tile offsets below `lim` all fall in it, at row row0 + offset
             const ExpA a = s_a[tid];
             const ExpC c = s_c[tid];
-            const ExpB bm = s_bm[tid];
             int4 f = make_int4(-1, 0, 0, 0);  // (slot, row0, lim, -)
             if (pre < a.L) {
-                const bool big = pre < a.thr;
-                const unsigned d = big ? (unsigned)c.b + 1u : (unsigned)c.b;
-                const unsigned x0 = big ? (unsigned)pre : (unsigned)(pre - a.thr);
-                const unsigned q = div_m32(x0, d, big ? bm.m1 : bm.m0);
-                const int j = big ? (int)q : a.rem + (int)q;
-                const int start = j * c.b + min(j, a.rem);
+                int j, start, end;
+                if (a.rem >= 0) {
+                    // floor-form quotas: the copy by one division
+                    const ExpB bm = s_bm[tid];
+                    const bool big = pre < a.thr;
+                    const unsigned d = big ? (unsigned)c.b + 1u : (unsigned)c.b;
+                    const unsigned x0 = big ? (unsigned)pre : (unsigned)(pre - a.thr);
+                    const unsigned q = div_m32(x0, d, big ? bm.m1 : bm.m0);
+                    j = big ? (int)q : a.rem + (int)q;
+                    start = j * c.b + min(j, a.rem);
+                    end = start + c.b + (j < a.rem ? 1 : 0);
+                } else {
+                    // other quotas (c.b copies): the last copy starting at or before pre
+                    j = last_at_most(c.b, pre, [&](int jj) { return s_cs[c.cb + jj]; });
+                    start = s_cs[c.cb + j];
+                    end = j + 1 < c.b ? s_cs[c.cb + j + 1] : a.L;
+                }
                 const int2 cr = s_cpr[c.cb + j];
-                const int quota = c.b + (j < a.rem ? 1 : 0);
-                f = make_int4(cr.x, cr.y + (pre - start), start + quota - pre, 0);
+                f = make_int4(cr.x, cr.y + (pre - start), end - pre, 0);
             }
             s_fast[tid] = f;
         }
@@ -735,9 +745,19 @@ reroute_kernel(const int32_t* __restrict__ idx, int64_t Q, int R, int E, int S,
             const int64_t i = pair_at<kOrder>(t0 + x, ord);
             const ExpA a = s_a[ev];
             const ExpC c = s_c[ev];
-            const int o = a.pre + (v < 0 ? 0 : v >> 8);
+            const int lo = v < 0 ? 0 : v >> 8;
+            const int o = a.pre + lo;
             int p = -1, row = -1;
-            if (kOrder != kOrderLocal && __all_sync(kFull, ex < 0 || (a.rem >= 0 && o < a.L))) {
+            const int4 f = s_fast[ev];
+            if (kOrder != kOrderLocal && __all_sync(kFull, ex < 0 || lo < f.z)) {
+                // every pair of the round lies in the copy of its expert's
+                // first pair in the tile
+                if (ex >= 0) {
+                    p = f.x;
+                    row = f.y + lo;
+                }
+            } else if (kOrder != kOrderLocal &&
+                       __all_sync(kFull, ex < 0 || (a.rem >= 0 && o < a.L))) {
                 // every lane of the round has floor-form quotas: no branches
                 const ExpB bm = s_bm[ev];
                 const bool big = o < a.thr;
