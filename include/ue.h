@@ -97,7 +97,10 @@ typedef struct ue_ctx ue_ctx; /* opaque */
 
 /* Create a context for `cfg` on CUDA device `device` (made current) and
  * allocate its scratch once: the error word, the reroute's look-back status
- * words (ceil(Q/8192)*E 64-bit words plus a ticket, a counter and an epoch),
+ * words (ceil(Q/tile)*E 64-bit words, a tile being 512 threads x 7 to 32
+ * pairs, the smallest size whose tiles are all resident on the device at
+ * once; a word per group of 16 tiles and expert, a counter per group, a
+ * ticket, a counter and an epoch),
  * the locality order's two int32 [R][P] tables, a row of d zero bf16 values
  * (the combine reads it in place of a row out of range) and the gradient
  * reduction's int32 lists of replicated experts and their slots (at most
@@ -231,7 +234,8 @@ ue_status ue_plan_ex(ue_ctx* ctx, const int32_t* load_e, const ue_plan_opts* opt
  * first, then replicas by ascending g): the o-th pair of expert e goes to
  * the copy whose quota range holds o, at row slot_offset[p] + (o - start).
  * dest_row is a permutation of [0, Q). Single pass: a stable counting sort
- * with a decoupled look-back scan over tiles of 8192 pairs; its waits are
+ * with a decoupled look-back scan over tiles of 3584 to 16384 pairs (the
+ * smallest size whose tiles are all resident at once); its waits are
  * bounded and end with UE_ERR_TIMEOUT. Ids outside [0, E) set
  * UE_ERR_DEVICE_BOUNDS. */
 ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
