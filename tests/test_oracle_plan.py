@@ -212,3 +212,43 @@ def test_reroute_invariants_random(R, T, E, K, S):
     check_plan_invariants(out["load_e"], R, S, out["plan"])
     check_reroute_determined(out["idx"], R, E, S, out["plan"], out["phys_slot"],
                              out["dest_row"])
+
+
+def test_plan_that_cannot_balance_places_zero_quota_copies():
+    """Worked by hand: R = 2, E = 2 (one master per rank), S = 3, loads
+    L = (3, 0). Q = 3 over 2 ranks can never reach max <= 1.02 * 1.5, so the
+    greedy places a copy of expert 0 (the only ratio above 0) in every slot:
+    r* = 1, 1, 0, 1, 0, 0 (rank loads (3,0) (2,1) (1,2) (2,1) (2,1) (3,0)).
+    With c copies in copy order (master, then ascending g) the quotas are
+    floor(3/c) + [j < 3 mod c]: from c = 4 on, every copy past the third
+    gets 0, and the last placements move rank 1's pair back to rank 0, so
+    the makespan ends where it began. Co-located copies: three on rank 0
+    (beside the master) and two on rank 1 (after its first copy)."""
+    pl = oracle.plan(np.array([3, 0], dtype=np.int32), 2, 3)
+    assert pl.slot_expert.tolist() == [0, 0, 0, 0, 0, 0]
+    assert pl.n_copies.tolist() == [7, 1]
+    assert pl.slot_quota.tolist() == [1, 1, 1, 0, 0, 0, 0, 0]
+    assert pl.slot_offset.tolist() == [0, 1, 2, 3, 3, 3, 3, 3, 3]
+    assert pl.rank_load.tolist() == [3, 0]
+    assert pl.stats.tolist() == [6, 3, 3, 5]
+
+
+@pytest.mark.parametrize("R,E,S,seed", [(3, 6, 2, 0), (4, 8, 4, 3), (5, 10, 3, 0)])
+def test_reroute_with_zero_quota_copies(R, E, S, seed):
+    """Layouts the greedy cannot balance (the hot expert's master shares its
+    rank with a master that keeps the remainder), one token per rank, K = 1:
+    experts end with more copies than pairs; the reroute still fills the
+    copies with a positive quota in copy order and sends nothing to the
+    others."""
+    rng = np.random.default_rng(seed)
+    logits = rng.normal(size=(R, E)).astype(np.float32)
+    logits[:, 0] += 4.0
+    logits[:, 1] += 2.0
+    out = oracle.run_path(logits, R, 1, S, 1)
+    pl = out["plan"]
+    L = out["load_e"]
+    assert ((pl.n_copies > L) & (L > 0)).any()
+    check_plan_invariants(L, R, S, pl)
+    check_reroute_determined(out["idx"], R, E, S, pl, out["phys_slot"], out["dest_row"])
+    used = np.bincount(out["phys_slot"].ravel(), minlength=R * (E // R + S))
+    assert (used[pl.slot_quota == 0] == 0).all()
