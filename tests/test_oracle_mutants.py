@@ -78,6 +78,10 @@ MUTANTS = {
                               "    for (int32_t r = 0; r < R; ++r) {\n        for (int32_t t = 0; t < T; ++t) {"),
     "local_row_without_source_offset": ("dest_row[i] = src_offset[(int64_t)r * P + found] + (int32_t)(o - start);",
                                         "dest_row[i] = src_offset[found] + (int32_t)(o - start);"),
+    "greedy_needs_a_pair_per_copy": ("if ((int64_t)load_e[e] < (int64_t)min_tokens * (n_copies[e] + 1)) continue;",
+                                     "if ((int64_t)load_e[e] < (int64_t)(min_tokens > 0 ? min_tokens : 1) * (n_copies[e] + 1)) continue;"),
+    "colocation_counts_masters_only": ("        for (int32_t s = 0; s < S; ++s)\n            if (slot_expert[rstar * S + s] == estar) hosts = 1;\n",
+                                       ""),
     "grad_reduce_skips_master": ("out[(int64_t)e * numel + i] = (double)master[(int64_t)e * numel + i];",
                                  "out[(int64_t)e * numel + i] = 0.0;"),
 }
@@ -96,6 +100,7 @@ def run_pins(golden_dir):
         ("hand_plans", lambda: tp.test_hand_worked_plans(golden_dir)),
         ("plan_invariants", lambda: tp.test_plan_invariants_random(8, 64, 2, 1.2)),
         ("plan_hot", tp.test_plan_single_hot_expert_closed_form),
+        ("plan_unbalanceable", tp.test_plan_that_cannot_balance_places_zero_quota_copies),
         ("hand_reroute", lambda: tp.test_reroute_hand_worked(golden_dir)),
         ("reroute_invariants", lambda: tp.test_reroute_invariants_random(4, 33, 16, 3, 2)),
         ("permute", tr.test_permute_definition_small),
