@@ -82,6 +82,8 @@ MUTANTS = {
                                      "if ((int64_t)load_e[e] < (int64_t)(min_tokens > 0 ? min_tokens : 1) * (n_copies[e] + 1)) continue;"),
     "colocation_counts_masters_only": ("        for (int32_t s = 0; s < S; ++s)\n            if (slot_expert[rstar * S + s] == estar) hosts = 1;\n",
                                        ""),
+    "reroute_replica_end_inclusive": ("if (o < start + slot_quota[p]) found = p;",
+                                      "if (o <= start + slot_quota[p]) found = p;"),
     "grad_reduce_skips_master": ("out[(int64_t)e * numel + i] = (double)master[(int64_t)e * numel + i];",
                                  "out[(int64_t)e * numel + i] = 0.0;"),
 }
@@ -103,6 +105,7 @@ def run_pins(golden_dir):
         ("plan_unbalanceable", tp.test_plan_that_cannot_balance_places_zero_quota_copies),
         ("hand_reroute", lambda: tp.test_reroute_hand_worked(golden_dir)),
         ("reroute_invariants", lambda: tp.test_reroute_invariants_random(4, 33, 16, 3, 2)),
+        ("reroute_zero_quota", lambda: tp.test_reroute_with_zero_quota_copies(4, 8, 4, 3)),
         ("permute", tr.test_permute_definition_small),
         ("combine_exact", tr.test_combine_exact_dyadic_case),
         ("combine_identity", tr.test_combine_identity_experts_reproduce_hidden),
