@@ -84,6 +84,10 @@ MUTANTS = {
                                        ""),
     "reroute_replica_end_inclusive": ("if (o < start + slot_quota[p]) found = p;",
                                       "if (o <= start + slot_quota[p]) found = p;"),
+    "topk_softmax_over_k_plus_one": ("for (int32_t k = 0; k < K; ++k) z += exp((double)row[k].v - v0);",
+                                     "for (int32_t k = 0; k <= K && k < E; ++k) z += exp((double)row[k].v - v0);"),
+    "combine_drops_last_k": ("out[j * d + c] = 0.0;\n        for (int32_t k = 0; k < K; ++k) {",
+                             "out[j * d + c] = 0.0;\n        for (int32_t k = 0; k + 1 < K; ++k) {"),
     "grad_reduce_skips_master": ("out[(int64_t)e * numel + i] = (double)master[(int64_t)e * numel + i];",
                                  "out[(int64_t)e * numel + i] = 0.0;"),
 }
