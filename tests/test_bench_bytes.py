@@ -81,3 +81,15 @@ def test_threaded_cpu_baseline_equals_the_oracle():
         bench.check_threaded_slice(w, lg, hd, w.T, res)
     pairs, secs, n = bench.threaded_oracle_slices(w, lg, hd, 128, 0.0, 2, 4)
     assert pairs == w.R * 128 * w.K and n == 1 and secs > 0
+
+
+@pytest.mark.parametrize("name,launches", [
+    ("prefill_ep40_e160", 5), ("qwen3_layer_r64_e128", 5), ("dsv3_layer_r64_e256", 5),
+    ("sweep_48x8_r64_e128", 5), ("pages_ep64_e256_t8k", 5), ("small_r8_e64", 6),
+])
+def test_kernel_launches_per_step(name, launches):
+    """The `gpu_launches` claim: five kernels a step where the gate takes the
+    count in (K = 8, E a multiple of 32 from 64 to 256), gate, count, plan,
+    reroute, permute and combine otherwise (the small layer has K = 4). The
+    plan and the reroute stay two kernels when one call launches both."""
+    assert bench.kernels_per_step(synth.WORKLOADS[name]) == launches
