@@ -113,13 +113,17 @@ typedef struct ue_ctx ue_ctx; /* opaque */
  * On error *out is set to NULL. */
 ue_status ue_init(const ue_config* cfg, int device, ue_ctx** out);
 
-/* Free the context's scratch (synchronises the device first). NULL is
- * accepted and ignored. */
+/* Free the context's scratch (synchronises the device first); the end of
+ * the Manager's life ("Interface / 1. Initialization"). NULL is accepted
+ * and ignored. Returns UE_OK, UE_ERR_INVALID_ARG for a pointer that is not
+ * a live context, or UE_ERR_CUDA if the synchronisation failed (the
+ * context is freed in every case but the first two). */
 ue_status ue_destroy(ue_ctx* ctx);
 
 /* Synchronise `stream`, then read and clear the context's device error
- * word. Returns UE_OK, UE_ERR_DEVICE_BOUNDS, UE_ERR_TIMEOUT, or UE_ERR_CUDA
- * if the synchronisation itself failed. */
+ * word (the pages have no counterpart: their calls raise in Python). Returns
+ * UE_OK, UE_ERR_DEVICE_BOUNDS, UE_ERR_TIMEOUT, or UE_ERR_CUDA if the
+ * synchronisation itself failed. */
 ue_status ue_get_error(ue_ctx* ctx, void* stream);
 
 /* Router gating ("Interface / 2. Forward and backward": probs, routing_map
@@ -130,7 +134,9 @@ ue_status ue_get_error(ue_ctx* ctx, void* stream);
  *          go to the lower expert id. Logits must be finite.
  *   w      fp32 [N][K]: softmax over the K selected logits,
  *          w_k = exp(v_k - v_0) / sum_j exp(v_j - v_0), evaluated in fp64
- *          and rounded once to fp32. */
+ *          and rounded once to fp32.
+ * Errors: host-side only (null or misaligned pointers); any finite logits
+ * are valid input. */
 ue_status ue_gate_topk(ue_ctx* ctx, const float* logits, int32_t* idx,
                        float* w, void* stream);
 
@@ -170,7 +176,8 @@ ue_status ue_gate_count(ue_ctx* ctx, const float* logits, int32_t* idx, float* w
  * the lowest e) and give it a copy in the lowest free slot of the least
  * loaded rank that has one (ties to the lowest r).
  * Writes every array of `out` (device pointers, see ue_placement). Runs as
- * a single CTA. */
+ * a single CTA. A negative entry of load_e sets UE_ERR_DEVICE_BOUNDS and
+ * counts as 0. */
 ue_status ue_plan(ue_ctx* ctx, const int32_t* load_e, const ue_placement* out,
                   void* stream);
 
@@ -241,7 +248,8 @@ ue_status ue_plan_ex(ue_ctx* ctx, const int32_t* load_e, const ue_plan_opts* opt
 ue_status ue_reroute(ue_ctx* ctx, const int32_t* idx, const ue_placement* plan,
                      int32_t* phys_slot, int32_t* dest_row, void* stream);
 
-/* ue_plan then ue_reroute on one stream, overlapped: the reroute kernel is
+/* ue_plan then ue_reroute on one stream ("Interface / 2. Forward and
+ * backward": update_placement, then reroute), overlapped: the reroute kernel is
  * launched as a programmatic dependent of the plan kernel, so its tiles copy,
  * count and look back over idx on the other SMs while the plan's single CTA
  * runs, and read the plan only after the plan kernel has completed. The
@@ -346,7 +354,9 @@ ue_status ue_combine_backward(ue_ctx* ctx, const float* dout, const uint16_t* y,
                               const int32_t* dest_row, const float* w, uint16_t* dy,
                               float* dw, void* stream);
 
-/* Backward of the permute: dhidden[n] = sum_k ddispatch[dest_row[n*K+k]],
+/* Backward of the permute ("Interface / 2. Forward and backward": the
+ * backward pass returns dispatch gradients to the tokens that sent them):
+ * dhidden[n] = sum_k ddispatch[dest_row[n*K+k]],
  * fp32 [N][d] (16-byte aligned), k ascending from 0; ddispatch bf16 [Q][d].
  * Rows outside [0, Q) are skipped and set UE_ERR_DEVICE_BOUNDS. */
 ue_status ue_permute_backward(ue_ctx* ctx, const uint16_t* ddispatch,
@@ -375,7 +385,9 @@ ue_status ue_weight_sync(ue_ctx* ctx, const ue_placement* plan, const void* mast
  *                    place: master[e] = master[e] + replicas[g1] + ... over
  *                    e's replica slots in ascending g, added in that order,
  *                    so the result is the same on every run.
- *   numel_per_expert > 0 and a multiple of 4. */
+ *   numel_per_expert > 0 and a multiple of 4.
+ * A slot_expert entry >= E sets UE_ERR_DEVICE_BOUNDS and that slot is
+ * skipped. */
 ue_status ue_grad_reduce(ue_ctx* ctx, const ue_placement* plan, const float* replica_grads,
                          float* master_grads, int64_t numel_per_expert, void* stream);
 
