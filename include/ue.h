@@ -154,9 +154,10 @@ ue_status ue_gate_topk(ue_ctx* ctx, const float* logits, int32_t* idx,
 ue_status ue_count(ue_ctx* ctx, const int32_t* idx, int32_t* load_re,
                    int32_t* load_e, void* stream);
 
-/* ue_gate_topk and ue_count in one call: the same idx, w, load_re and load_e
- * as the two calls in sequence (same arguments, same layouts, the same
- * errors). For K = 8 and E a multiple of 32 from 64 to 256 the histogram is
+/* ue_gate_topk and ue_count in one call ("Interface / 2. Forward and
+ * backward": the router's routing; "UltraEP" README intro: the exact
+ * post-gating load): the same idx, w, load_re and load_e as the two calls in
+ * sequence (same arguments, same layouts, the same errors). For K = 8 and E a multiple of 32 from 64 to 256 the histogram is
  * taken inside the gate kernel (each CTA adds its picks to a shared
  * histogram per source rank and its bins to the outputs at the end), so
  * idx is not read back; other shapes run the two kernels. Uses context
@@ -203,7 +204,8 @@ typedef struct {
 
 enum { UE_SOLVER_GREEDY = 0, UE_SOLVER_BISECT = 1 };
 
-/* Replication plan with a choice of planner. Arguments as for ue_plan.
+/* Replication plan with a choice of planner ("Performance Tuning /
+ * Replication planning"). Arguments as for ue_plan.
  *   UE_SOLVER_GREEDY: the ue_plan rule, where only experts with
  *     L_e >= min_tokens * (c_e + 1) may take a copy (each copy keeps at
  *     least min_tokens pairs); the greedy also stops when no expert may.
@@ -302,7 +304,8 @@ ue_status ue_reroute_ex(ue_ctx* ctx, const int32_t* idx, const ue_placement* pla
 ue_status ue_locality_split(ue_ctx* ctx, const int32_t* load_re, const ue_placement* plan,
                             int32_t* src_quota, int32_t* src_offset, void* stream);
 
-/* Reroute under the locality-aware split: source rank r hands its pairs of
+/* Reroute under the locality-aware split ("Performance Tuning / Replication
+ * planning": per-rank quota decomposition): source rank r hands its pairs of
  * expert e, in its own order (t, k), to e's copies in copy order,
  * src_quota[r][p] pairs each, at rows src_offset[r][p], src_offset[r][p]+1,
  * ... The arrays are those ue_locality_split wrote for this plan and load_re

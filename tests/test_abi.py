@@ -105,3 +105,21 @@ def test_init_without_gpu_fails_cleanly(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="not found"):
         ue.load_library(str(tmp_path / "libue.so"))
+
+
+def test_header_documents_every_entry_point():
+    """Every entry point ue.h declares sits under a comment that states its
+    error behaviour (an error code, or errors "as for" another call) and
+    names its source on the pages, or says that the pages have none."""
+    text = open(os.path.join(ROOT, "include", "ue.h")).read()
+    for name in ue.EXPORTS:
+        m = re.search(r"ue_status\s+" + name + r"\s*\(", text)
+        assert m, name
+        end = text.rfind("*/", 0, m.start())
+        start = text.rfind("/*", 0, end)
+        between = text[end + 2:m.start()]
+        # only other prototypes may stand between the comment and this one
+        assert re.fullmatch(r"(\s|ue_status\s+\w+\s*\([^;]*\);)*", between), name
+        doc = text[start:end]
+        assert re.search(r"UE_ERR|[Ee]rrors?\b", doc), f"{name}: no error behaviour"
+        assert re.search(r'"[A-Z][^"]+"|README|no counterpart', doc), f"{name}: no source"
